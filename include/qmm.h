@@ -1,0 +1,231 @@
+/*
+ * qmm.h -- C ABI of the block-quantized weight matmul library (libqmm.so).
+ *
+ * The library runs LLM inference matmuls directly on ggml-style block-quantized
+ * weights on an NVIDIA B200 (sm_100a). Weights are never dequantized to a
+ * separate buffer: each kernel decodes the blocks as it streams them.
+ *
+ * ---------------------------------------------------------------------------
+ * Block formats (ggml style; weights stay in this layout end to end --
+ * "Lumen v0.2.0 -- Q8-native decode", section "Phase 7.D -- Q8-native fused
+ * matmul"):
+ *
+ *   Q8_0 (34 bytes / 32 weights): uint16 d (IEEE fp16 bits, little-endian),
+ *        then int8 qs[32]. Weight j = qs[j] * d.
+ *   Q4_0 (18 bytes / 32 weights): uint16 d (fp16 bits), then uint8 qs[16].
+ *        Weight j (j < 16) = ((qs[j] & 15) - 8) * d,
+ *        weight j+16      = ((qs[j] >> 4) - 8) * d.
+ *
+ * A weight matrix W holds N rows (output features) of K/32 blocks each,
+ * row-major, K contiguous: block b of row n starts at byte
+ * (n * (K/32) + b) * block_bytes. There is no padding between rows.
+ *
+ * Dense operands are row-major: X[m][k] at X + m*K + k, Y[m][n] at Y + m*N + n.
+ * Every matmul computes Y[m][n] = sum_k X[m][k] * W[n][k].
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions shared by every entry point:
+ *   - All buffer pointers are DEVICE pointers owned by the caller. The library
+ *     allocates no memory and frees none.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; nothing synchronises the host.
+ *   - Arguments are validated on the host before any CUDA call. A call that
+ *     returns an error has launched nothing and written nothing.
+ *   - `block` must be 32 (QMM_ERR_BLOCK otherwise).
+ *   - Sizes are int64_t. Negative sizes are QMM_ERR_SHAPE. M == 0 or N == 0 is
+ *     a valid empty call that launches nothing. K must be a multiple of 32;
+ *     K == 0 makes every output an empty sum (written as 0; the gate/up
+ *     output is silu(0) * 0 = 0).
+ *   - A pointer may be NULL only if the buffer it names is empty.
+ *   - W, Wg, Wu, X and QX must be 16-byte aligned; Y and DX 4-byte aligned
+ *     (QMM_ERR_ALIGN). torch / cudaMalloc allocations satisfy both.
+ *   - Inputs are assumed finite; NaN / Inf propagation is unspecified.
+ *   - The device must be compute capability 10.0 (B200 class); otherwise
+ *     QMM_ERR_DEVICE.
+ *   - Launch failures are returned as QMM_ERR_CUDA with the CUDA error text in
+ *     qmm_last_error_string().
+ *   - A kernel that waits too long on one of its own pipeline barriers (about
+ *     two seconds) stops, records the fact in a device status word and returns
+ *     instead of hanging; qmm_device_status() reads and clears that word.
+ *   - Calls are thread-safe. The entry points keep no state between calls.
+ *
+ * Tolerances the library is tested to (per output, S = sum_k |w_k * x_k|):
+ *   fp32-accumulated paths: |y - exact| <= 1e-5 * S;
+ *   bf16 tensor-core prefill: |y - exact| <= 4e-3 * S;
+ *   activation codes and int32 block dots: bit-exact.
+ */
+#ifndef QMM_H
+#define QMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t == struct CUstream_st * */
+typedef struct CUstream_st *qmm_stream_t;
+
+typedef enum {
+  QMM_OK = 0,
+  QMM_ERR_NULL = 1,         /* required pointer is NULL                       */
+  QMM_ERR_SHAPE = 2,        /* negative size, K % 32 != 0, M or K too large  */
+  QMM_ERR_BLOCK = 3,        /* block != 32                                    */
+  QMM_ERR_ALIGN = 4,        /* pointer not aligned as documented              */
+  QMM_ERR_DTYPE = 5,        /* unknown weight type                            */
+  QMM_ERR_DEVICE = 6,       /* current device is not compute capability 10.x  */
+  QMM_ERR_CUDA = 7,         /* a CUDA runtime call failed                      */
+  QMM_ERR_DEVICE_CHECK = 8  /* a kernel recorded a device-side failure         */
+} qmm_status;
+
+typedef enum { QMM_Q8_0 = 0, QMM_Q4_0 = 1 } qmm_wtype;
+
+#define QMM_BLOCK 32
+#define QMM_Q8_0_BLOCK_BYTES 34
+#define QMM_Q4_0_BLOCK_BYTES 18
+/* Largest M of the decode entry points (qmm_q8_gemv, qmm_q8q8_gemv,
+ * qmm_q4_swiglu_gateup). */
+#define QMM_MAX_DECODE_M 8
+/* Largest K of every entry point. */
+#define QMM_MAX_K 32768
+
+/*
+ * qmm_q8_gemv -- decode GEMV / small-M matmul on Q8_0 weights, fp32 activations.
+ *
+ * Defined by "Lumen v0.2.0 -- Q8-native decode", section "Phase 7.D --
+ * Q8-native fused matmul": the per-block fp16 scale d is broadcast over its 32
+ * weights, the K direction is reduced block by block and one output per row is
+ * written; there is no load-time dequantisation.
+ *
+ *   Y[m][n] = sum_b d[n][b] * sum_j qs[n][b][j] * X[m][32b + j]   (fp32 accumulation)
+ *
+ *   M      1 .. QMM_MAX_DECODE_M tokens (0 = empty call)
+ *   N      output features (rows of W), >= 0
+ *   K      reduction length, multiple of 32, <= QMM_MAX_K
+ *   W      N * K/32 Q8_0 blocks (device, read only, 16-byte aligned)
+ *   X      M x K fp32 (device, read only, 16-byte aligned)
+ *   Y      M x N fp32 (device, written)
+ */
+qmm_status qmm_q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
+                       float *Y, qmm_stream_t stream);
+
+/*
+ * qmm_quantize_act_q8 -- quantise fp32 activations to Q8 codes per 32-block.
+ *
+ * The activation-quantisation step of the Q8xQ8 path ("Lumen v0.4.0 --
+ * shape-aware VNNI/fp32 hybrid dispatch", section "Phase 7.M -- Q8xQ8 AVX2 int
+ * dot"). For every block of 32 consecutive activations of a row:
+ *   amax = max_j |x_j|;  d = amax / 127  (IEEE binary32 division, round to nearest even);
+ *   q_j  = round_half_away_from_zero(x_j / d)  (binary32 division), clamped to [-127, 127];
+ *   if d == 0, every q_j = 0.
+ *
+ *   M, K   rows and row length (K multiple of 32, <= QMM_MAX_K); M >= 0
+ *   X      M x K fp32 (device, read only, 16-byte aligned)
+ *   QX     M x K int8 codes (device, written, 16-byte aligned)
+ *   DX     M x K/32 fp32 scales d (device, written)
+ * The codes and scales are bit-exact functions of X.
+ */
+qmm_status qmm_quantize_act_q8(int64_t M, int64_t K, int block, const float *X, int8_t *QX,
+                               float *DX, qmm_stream_t stream);
+
+/*
+ * qmm_q8q8_gemv -- Q8_0 weights times Q8-quantised activations.
+ *
+ * "Lumen v0.4.0", section "Phase 7.M -- Q8xQ8 AVX2 int dot": each block's dot
+ * product of int8 weight codes and int8 activation codes is an exact int32,
+ * which is then scaled by both block scales and accumulated in fp32:
+ *
+ *   isum[m][n][b] = sum_j qs[n][b][j] * QX[m][32b + j]           (exact int32)
+ *   Y[m][n]       = sum_b (d[n][b] * DX[m][b]) * isum[m][n][b]   (fp32)
+ *
+ *   M      1 .. QMM_MAX_DECODE_M (0 = empty call)
+ *   W      N * K/32 Q8_0 blocks (16-byte aligned); QX M x K int8 (16-byte
+ *          aligned); DX M x K/32 fp32 -- as written by qmm_quantize_act_q8
+ *   Y      M x N fp32 (written)
+ */
+qmm_status qmm_q8q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W,
+                         const int8_t *QX, const float *DX, float *Y, qmm_stream_t stream);
+
+/*
+ * qmm_q4_swiglu_gateup -- fused gate/up projection with SwiGLU on Q4_0 weights.
+ *
+ * "LSE v0.4.16", section "Combined M8 Q4 gate/up execution": one launch reads
+ * one shared activation panel X, accumulates the gate and up projections in
+ * independent fp32 accumulators and writes only
+ *
+ *   Y[m][n] = silu(g) * u,  g = sum_k X[m][k] Wg[n][k],  u = sum_k X[m][k] Wu[n][k],
+ *   silu(g) = g / (1 + exp(-g)).
+ *
+ * No gate (or up) temporary is written to memory.
+ *
+ *   M       1 .. QMM_MAX_DECODE_M (0 = empty call)
+ *   Wg, Wu  N * K/32 Q4_0 blocks each (16-byte aligned)
+ *   X       M x K fp32 (16-byte aligned)
+ *   Y       M x N fp32 (written)
+ */
+qmm_status qmm_q4_swiglu_gateup(int64_t M, int64_t N, int64_t K, int block, const void *Wg,
+                                const void *Wu, const float *X, float *Y, qmm_stream_t stream);
+
+/*
+ * qmm_quant_matmul_prefill -- prefill panel Y = X . W^T on the tensor cores.
+ *
+ * "LSE v0.4.16", section "Retained optimizations and compatibility" (M1024
+ * prefill panels): a many-token matmul against block-quantized weights. The
+ * blocks are decoded to bf16 (w = q*d rounded to nearest even) in shared
+ * memory and multiplied by bf16 activations with fp32 accumulation on the
+ * tcgen05 tensor cores.
+ *
+ *   wtype   QMM_Q8_0 or QMM_Q4_0 (QMM_ERR_DTYPE otherwise)
+ *   M       tokens, >= 0
+ *   W       N * K/32 blocks of `wtype` (16-byte aligned)
+ *   X       M x K bf16 bit patterns (uint16_t, 16-byte aligned)
+ *   Y       M x N fp32 (written)
+ */
+qmm_status qmm_quant_matmul_prefill(int wtype, int64_t M, int64_t N, int64_t K, int block,
+                                    const void *W, const uint16_t *X, float *Y,
+                                    qmm_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Test and utility exports (not on the hot path).                           */
+
+/*
+ * qmm_q8q8_block_dots -- the exact int32 block dots of qmm_q8q8_gemv, written
+ * out: isum[(m*N + n)*(K/32) + b] (M x N x K/32 int32, device, written).
+ * Computed by the same device code as qmm_q8q8_gemv; used to test the integer
+ * part bit-exactly.
+ */
+qmm_status qmm_q8q8_block_dots(int64_t M, int64_t N, int64_t K, int block, const void *W,
+                               const int8_t *QX, int32_t *isum, qmm_stream_t stream);
+
+/*
+ * qmm_q4_gateup_unfused -- the unfused counterpart of qmm_q4_swiglu_gateup:
+ * writes the gate and up projections G, U (M x N fp32 each) with two separate
+ * projection launches, then Y = silu(G) * U with a third launch. Each
+ * projection uses the same accumulation code and order as the fused kernel,
+ * so Y matches qmm_q4_swiglu_gateup bit for bit ("LSE v0.4.16", section
+ * "Combined M8 Q4 gate/up execution": exact outputs preserved).
+ */
+qmm_status qmm_q4_gateup_unfused(int64_t M, int64_t N, int64_t K, int block, const void *Wg,
+                                 const void *Wu, const float *X, float *G, float *U, float *Y,
+                                 qmm_stream_t stream);
+
+/* Text of the last error raised on the calling host thread ("" if none). */
+const char *qmm_last_error_string(void);
+
+/* Library version string, e.g. "qmm 0.1.0 sm_100a". */
+const char *qmm_version(void);
+
+/*
+ * qmm_device_status -- synchronises the current device, then reads and clears
+ * the device-side status word that kernels set when a bounded wait gives up.
+ * *bits receives the word (0 = no failure recorded). Returns QMM_OK, or
+ * QMM_ERR_CUDA if the synchronisation itself failed.
+ */
+qmm_status qmm_device_status(uint32_t *bits);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMM_H */
