@@ -1,0 +1,506 @@
+"""Benchmark: Qwen2.5-0.5B-shaped M=1 decode step on Q8_0 weights, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-components]
+
+One step = the 121 weight matmuls of one decode token (24 layers x {qkv 896->1152,
+wo 896->896, gate 896->4864, up 896->4864, down 4864->896} + lm_head 896->151936),
+each a qmm_q8_gemv call (M=1, Q8_0 blocks, fp32 activations), stream-ordered and
+replayed as one CUDA graph with programmatic dependent launch. Weights are seeded
+synthetic tensors with the shapes of that model (no trained weights are used);
+they total 524,833,792 bytes per step, more than the 126 MB L2, so no flush is
+needed between steps. value = decode tokens/s (steps/s) summed over ranks.
+
+Under torchrun (N > 1) every rank decodes its own sequence on its own copy of
+the weights (data-parallel replicas, weak scaling); the only collective is the
+max-over-ranks reduction of the measured time.
+
+`--impl reference` times the CPU oracle (oracle/) on the host cores on a bounded
+sample of the same workload and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as syn  # noqa: E402
+
+METRIC = "Q8_0/Q4_0 GEMV HBM GB/s (% of B200 peak); decode-step tok/s equiv; prefill TFLOP/s"
+UNIT = "tok/s"
+WORKLOAD = ("Qwen2.5-0.5B-shaped M=1 decode step: 121 Q8_0 GEMVs (24 x qkv 896->1152, wo 896->896, "
+            "gate/up 896->4864, down 4864->896, + lm_head 896->151936)")
+
+
+def step_bytes():
+    """Algorithmic bytes of one decode step: weight blocks + fp32 x read + fp32 y written."""
+    w = x = y = 0
+    for _, n, k in syn.decode_step_shapes():
+        w += n * (k // 32) * 34
+        x += k * 4
+        y += n * 4
+    return w, x, y
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(units_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: units processed by all ranks / slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1000.0)
+
+
+# --------------------------------------------------------------------------- clocks
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    def __init__(self, torch_device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml as nv
+            import torch
+
+            nv.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            self.h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self._reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.ok = True
+        except Exception as e:  # noqa: BLE001 - report, do not fail the bench
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM), int(self._reasons(self.h)),
+                                     nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0))
+            except Exception:  # noqa: BLE001
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "error": getattr(self, "err", "")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        bits = 0
+        for _, b, _ in self.samples:
+            bits |= b
+        reasons = [name for bit, name in REASON_BITS.items() if bits & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples),
+                "power_w_max": round(max(s[2] for s in self.samples), 1)}
+
+
+# --------------------------------------------------------------------------- the decode-step workload
+
+class DecodeStep:
+    """121 Q8_0 weight matrices resident in HBM, their activations and outputs."""
+
+    def __init__(self, seed: int, device, keep_host: bool):
+        import torch
+
+        self.shapes = syn.decode_step_shapes()
+        self.host_w = [] if keep_host else None
+        self.host_x = []
+        self.W = []
+        xs = []
+        for i, (_, n, k) in enumerate(self.shapes):
+            g = syn.rng(syn.sub_seed(seed, i))
+            wb, _, _ = syn.q8_0_weights(g, n, k)
+            x = syn.act_f32(g, 1, k)
+            self.W.append(torch.from_numpy(wb).to(device))
+            if keep_host:
+                self.host_w.append(wb)
+            self.host_x.append(x)
+            xs.append(x.reshape(-1))
+        self.x_offsets = np.cumsum([0] + [x.size for x in xs])
+        self.y_offsets = np.cumsum([0] + [n for _, n, _ in self.shapes])
+        self.host_xcat = torch.from_numpy(np.concatenate(xs)).pin_memory()
+        self.X = self.host_xcat.to(device)
+        self.Y = torch.zeros(int(self.y_offsets[-1]), dtype=torch.float32, device=device)
+        self.host_logits = torch.empty(self.shapes[-1][1], dtype=torch.float32).pin_memory()
+
+    def launch(self, qmm, stream_handle: int, flags: int):
+        lib = qmm.lib
+        xp, yp = self.X.data_ptr(), self.Y.data_ptr()
+        for i, (_, n, k) in enumerate(self.shapes):
+            st = lib.qmm_q8_gemv_ex(1, n, k, 32, self.W[i].data_ptr(), xp + 4 * int(self.x_offsets[i]),
+                                    yp + 4 * int(self.y_offsets[i]), flags, stream_handle)
+            if st != 0:
+                raise qmm.QmmError(st, "qmm_q8_gemv_ex")
+
+    def logits(self):
+        return self.Y[int(self.y_offsets[-2]):int(self.y_offsets[-1])]
+
+
+def capture(fn, stream):
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn(torch.cuda.current_stream().cuda_stream)
+    return g
+
+
+def time_graph(graph, stream, reps: int) -> float:
+    """Average ms of one replay over `reps` back-to-back replays (CUDA events on `stream`)."""
+    import torch
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+# --------------------------------------------------------------------------- components (rank 0, N=1)
+
+def component_single_gemv(qmm, dev_peak_gbs, n=1152, k=896, reps_graph=4):
+    """Single GEMV (M=1, K=896, N=1152): back-to-back launches over rotating weight copies
+    totalling > 2x L2, so every launch streams its weights from HBM."""
+    import torch
+
+    props = torch.cuda.get_device_properties(0)
+    l2 = getattr(props, "L2_cache_size", 126 * 2**20)
+    wbytes = n * (k // 32) * 34
+    copies = max(8, int(2.2 * l2 // wbytes) + 1)
+    g = syn.rng(0)
+    wb, _, _ = syn.q8_0_weights(g, n, k)
+    x = torch.from_numpy(syn.act_f32(g, 1, k)).cuda()
+    W0 = torch.from_numpy(wb).cuda()
+    Ws = [W0.clone() for _ in range(copies)]
+    Y = torch.empty(n, device="cuda")
+    s = torch.cuda.Stream()
+    out = {}
+    for name, flags in (("graph_pdl_early_weights", qmm.QMM_FLAG_EARLY_WEIGHTS), ("graph_pdl", 0)):
+        def fn(h, flags=flags):
+            for w in Ws:
+                st = qmm.lib.qmm_q8_gemv_ex(1, n, k, 32, w.data_ptr(), x.data_ptr(), Y.data_ptr(), flags, h)
+                assert st == 0
+        fn(s.cuda_stream)
+        torch.cuda.synchronize()
+        gr = capture(fn, s)
+        time_graph(gr, s, 2)
+        ms = time_graph(gr, s, reps_graph) / copies
+        bytes_ = wbytes + k * 4 + n * 4
+        out[name] = {"us_per_gemv": round(ms * 1e3, 3), "GB_s": round(bytes_ / ms / 1e6, 1),
+                     "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4)}
+        del gr
+    out["bytes_per_gemv"] = wbytes + k * 4 + n * 4
+    out["note"] = f"{copies} rotating weight copies (> 2x L2) in one CUDA graph"
+    return out
+
+
+def component_lm_head(qmm, step: DecodeStep, dev_peak_gbs, reps=20):
+    """The largest GEMV of the step alone (lm_head 896->151936, 145 MB of blocks)."""
+    import torch
+
+    n, k = step.shapes[-1][1], step.shapes[-1][2]
+    s = torch.cuda.Stream()
+    W = step.W[-1]
+    xp = step.X.data_ptr() + 4 * int(step.x_offsets[-2])
+    yp = step.Y.data_ptr() + 4 * int(step.y_offsets[-2])
+
+    def fn(h):
+        assert qmm.lib.qmm_q8_gemv_ex(1, n, k, 32, W.data_ptr(), xp, yp, 0, h) == 0
+    fn(s.cuda_stream)
+    gr = capture(fn, s)
+    time_graph(gr, s, 3)
+    ms = time_graph(gr, s, reps)
+    bytes_ = n * (k // 32) * 34 + k * 4 + n * 4
+    return {"us": round(ms * 1e3, 2), "GB_s": round(bytes_ / ms / 1e6, 1),
+            "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4), "bytes": bytes_}
+
+
+# --------------------------------------------------------------------------- CPU oracle baseline
+
+def oracle_step_sample(step_w, step_x, shapes, frac: float, threads: int):
+    """Run the oracle on the first ceil(frac * N) rows of every GEMV of a step, with
+    `threads` host threads over disjoint row windows. Returns seconds."""
+    import oracle
+
+    jobs = []
+    for i, (_, n, k) in enumerate(shapes):
+        rows = max(1, int(np.ceil(frac * n)))
+        per = max(1, (rows + threads - 1) // threads)
+        for r0 in range(0, rows, per):
+            jobs.append((i, n, r0, min(rows, r0 + per)))
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda j: oracle.gemv(syn.Q8_0, step_w[j[0]], step_x[j[0]], j[1], window=(0, 1, j[2], j[3])),
+                    jobs))
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(step_w, step_x, shapes, budget_s: float = 10.0):
+    threads = os.cpu_count() or 1
+    t_probe = oracle_step_sample(step_w, step_x, shapes, 0.01, threads)
+    full_est = t_probe / 0.01
+    frac = min(1.0, max(0.01, budget_s / max(full_est, 1e-9)))
+    t = oracle_step_sample(step_w, step_x, shapes, frac, threads)
+    return {"value": round(frac / t, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"first {frac:.1%} of the rows of all 121 GEMVs of one step (fp64 C oracle, "
+                      f"{threads} threads over row windows), {t:.1f} s; tok/s = fraction / time"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle timed on a bounded sample of the decode step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+
+    oracle.build()
+    shapes = syn.decode_step_shapes()
+    host_w, host_x = [], []
+    for i, (_, n, k) in enumerate(shapes):
+        g = syn.rng(syn.sub_seed(args.seed, i))
+        host_w.append(syn.q8_0_weights(g, n, k)[0])
+        host_x.append(syn.act_f32(g, 1, k))
+    threads = os.cpu_count() or 1
+    t_probe = oracle_step_sample(host_w, host_x, shapes, 0.01, threads)
+    full_est = t_probe / 0.01
+    total_budget = 150.0
+    per_step = total_budget / (args.steps + args.warmup)
+    frac = min(1.0, max(1e-4, per_step / max(full_est, 1e-9)))
+    for _ in range(args.warmup):
+        oracle_step_sample(host_w, host_x, shapes, frac, threads)
+    t = 0.0
+    for _ in range(args.steps):
+        t += oracle_step_sample(host_w, host_x, shapes, frac, threads)
+    value = args.steps * frac / t
+    sample = (f"each step: first {frac:.3%} of the rows of all 121 GEMVs (fp64 C oracle, {threads} threads over "
+              f"row windows); tok/s = steps * fraction / time")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * t / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- traffic from the committed ncu summary
+
+def committed_traffic(kernel_src: str, summary: str):
+    """DRAM bytes per launch recorded in a profiles/ summary, if the kernel source
+    is unchanged since (the summary records the source's sha1)."""
+    try:
+        text = open(os.path.join(ROOT, "profiles", summary)).read()
+        src = open(os.path.join(ROOT, "decode_gemv_qmm_b200", "csrc", kernel_src), "rb").read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_step:\s*([0-9]+)", text)
+    h = re.search(r"kernel_source_sha1:\s*([0-9a-f]{40})", text)
+    if not m or not h or h.group(1) != hashlib.sha1(src).hexdigest():
+        return None
+    return int(m.group(1))
+
+
+# --------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="qmm", choices=["qmm", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+
+    rank, world, local_rank = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    import decode_gemv_qmm_b200 as qmm
+
+    pk = peaks()
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    step = DecodeStep(args.seed, device, keep_host=want_cpu)
+    stream = torch.cuda.Stream()
+    flags = qmm.QMM_FLAG_EARLY_WEIGHTS
+    step.launch(qmm, stream.cuda_stream, flags)  # first call outside capture
+    torch.cuda.synchronize()
+    graph = capture(lambda h: step.launch(qmm, h, flags), stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    # warm-up
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+    torch.cuda.synchronize()
+
+    # timed region: K steps, barrier + synchronize on both sides
+    sampler = ClockSampler(torch.cuda.current_device())
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms_total, world, device)
+    ms_step = ms_max / args.steps
+    value = aggregate(args.steps, world, ms_max)
+
+    # e2e: host activations -> device, the step, logits -> host (pinned), every step
+    h2d = step.host_xcat.numel() * 4
+    d2h = step.host_logits.numel() * 4
+    logits = step.logits()
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(10, min(args.steps, 2000))
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            step.X.copy_(step.host_xcat, non_blocking=True)
+            graph.replay()
+            step.host_logits.copy_(logits, non_blocking=True)
+        f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, device)
+    e2e_value = aggregate(e2e_steps, world, e2e_ms)
+
+    wb, xb, yb = step_bytes()
+    bytes_step = wb + xb + yb
+    launches = len(step.shapes)
+    achieved_gbs = bytes_step / (ms_step * 1e6)
+    traffic = committed_traffic("q8_gemv.cu", "q8_gemv_decode_step.md")
+    roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved_gbs / pk["hbm_gbs"], 4),
+                "traffic": (round(traffic / launches) if traffic else None),
+                "kernel": "q8_gemv_kernel<1>",
+                "per_launch": {"algorithmic_bytes": round(bytes_step / launches),
+                               "avg_duration_us": round(ms_step * 1e3 / launches, 3)},
+                "peak_source": pk["source"], "vs_8TBs_spec": round(achieved_gbs / 8000.0, 4)}
+    clocks = sampler.summary()
+
+    components = None
+    if rank == 0 and world == 1 and not args.no_components:
+        components = {"lm_head_896x151936": component_lm_head(qmm, step, pk["hbm_gbs"]),
+                      "single_gemv_896x1152": component_single_gemv(qmm, pk["hbm_gbs"])}
+
+    cpu = None
+    if want_cpu:
+        cpu = cpu_baseline(step.host_w, step.host_x, step.shapes)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "M": 1, "weight_format": "Q8_0", "bytes_per_step": bytes_step,
+                           "l2": "inputs larger than L2 (524,833,792 weight bytes per step; no flush)",
+                           "launch": "CUDA graph of 121 qmm_q8_gemv_ex calls, programmatic dependent launch, "
+                                     "QMM_FLAG_EARLY_WEIGHTS",
+                           "parallelism": f"dp{world} (independent decode per rank)"},
+                "GB_s": round(achieved_gbs, 1), "roofline": roofline, "clocks": clocks,
+                "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h,
+                        "how": "pinned host activations copied in, graph replay, logits copied out, every step"},
+                "gpu_launches": launches * args.steps, "cpu_baseline": cpu, "components": components}
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

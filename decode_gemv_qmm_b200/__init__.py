@@ -1,0 +1,170 @@
+"""Python binding of libqmm.so: block-quantized weight matmul on B200 (sm_100a).
+
+Argument marshalling only -- every step of every operation runs in the CUDA
+kernels of libqmm.so. Functions carry the names of the C entry points
+(include/qmm.h) and take torch tensors for device buffers; PyTorch supplies
+device memory and streams, nothing else. Importing this package fails loudly
+if the library has not been built (``python -m decode_gemv_qmm_b200.build``);
+there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqmm.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m decode_gemv_qmm_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+QMM_OK, QMM_ERR_NULL, QMM_ERR_SHAPE, QMM_ERR_BLOCK, QMM_ERR_ALIGN = 0, 1, 2, 3, 4
+QMM_ERR_DTYPE, QMM_ERR_DEVICE, QMM_ERR_CUDA, QMM_ERR_DEVICE_CHECK = 5, 6, 7, 8
+STATUS_NAMES = {0: "QMM_OK", 1: "QMM_ERR_NULL", 2: "QMM_ERR_SHAPE", 3: "QMM_ERR_BLOCK", 4: "QMM_ERR_ALIGN",
+                5: "QMM_ERR_DTYPE", 6: "QMM_ERR_DEVICE", 7: "QMM_ERR_CUDA", 8: "QMM_ERR_DEVICE_CHECK"}
+QMM_Q8_0, QMM_Q4_0 = 0, 1
+QMM_FLAG_EARLY_WEIGHTS = 1
+BLOCK = 32
+MAX_DECODE_M = 8
+MAX_K = 32768
+
+_i64, _int, _u32, _p = ctypes.c_int64, ctypes.c_int, ctypes.c_uint32, ctypes.c_void_p
+_SIGS = {
+    "qmm_q8_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _p],
+    "qmm_q8_gemv_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _u32, _p],
+    "qmm_quantize_act_q8": [_i64, _i64, _int, _p, _p, _p, _p],
+    "qmm_q8q8_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
+    "qmm_q4_swiglu_gateup": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
+    "qmm_quant_matmul_prefill": [_int, _i64, _i64, _i64, _int, _p, _p, _p, _p],
+    "qmm_q8q8_block_dots": [_i64, _i64, _i64, _int, _p, _p, _p, _p],
+    "qmm_q4_gateup_unfused": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p],
+}
+for _name, _args in _SIGS.items():
+    _f = getattr(lib, _name, None)
+    if _f is not None:
+        _f.argtypes = _args
+        _f.restype = ctypes.c_int
+lib.qmm_last_error_string.restype = ctypes.c_char_p
+lib.qmm_last_error_string.argtypes = []
+lib.qmm_version.restype = ctypes.c_char_p
+lib.qmm_version.argtypes = []
+lib.qmm_device_status.restype = ctypes.c_int
+lib.qmm_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+
+
+class QmmError(RuntimeError):
+    def __init__(self, status: int, fn: str):
+        self.status = status
+        msg = lib.qmm_last_error_string().decode(errors="replace")
+        super().__init__(f"{fn}: {STATUS_NAMES.get(status, status)}: {msg}")
+
+
+def _check(status: int, fn: str):
+    if status != QMM_OK:
+        raise QmmError(status, fn)
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def version() -> str:
+    return lib.qmm_version().decode()
+
+
+def device_status() -> int:
+    """Synchronise and read-and-clear the kernels' device status word (0 = clean)."""
+    bits = ctypes.c_uint32(0)
+    _check(lib.qmm_device_status(ctypes.byref(bits)), "qmm_device_status")
+    return bits.value
+
+
+def _out(Y, shape, device, dtype=torch.float32):
+    if Y is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    return Y
+
+
+def qmm_q8_gemv(W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None = None, *,
+                block: int = BLOCK, flags: int = 0, stream=None) -> torch.Tensor:
+    """Y[M, N] = X[M, K] . dequant(W)^T for Q8_0 blocks W (uint8, N*K/32*34 bytes)."""
+    M, K = X.shape
+    Y = _out(Y, (M, N), X.device)
+    if flags:
+        st = lib.qmm_q8_gemv_ex(M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), flags, _stream(stream))
+    else:
+        st = lib.qmm_q8_gemv(M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), _stream(stream))
+    _check(st, "qmm_q8_gemv")
+    return Y
+
+
+def qmm_quantize_act_q8(X: torch.Tensor, QX: torch.Tensor | None = None, DX: torch.Tensor | None = None, *,
+                        block: int = BLOCK, stream=None):
+    """(QX int8[M, K], DX fp32[M, K/32]) = per-32-block Q8 quantisation of X."""
+    M, K = X.shape
+    QX = _out(QX, (M, K), X.device, torch.int8)
+    DX = _out(DX, (M, K // BLOCK), X.device)
+    _check(lib.qmm_quantize_act_q8(M, K, block, _ptr(X), _ptr(QX), _ptr(DX), _stream(stream)),
+           "qmm_quantize_act_q8")
+    return QX, DX
+
+
+def qmm_q8q8_gemv(W: torch.Tensor, QX: torch.Tensor, DX: torch.Tensor, N: int, Y: torch.Tensor | None = None, *,
+                  block: int = BLOCK, stream=None) -> torch.Tensor:
+    M, K = QX.shape
+    Y = _out(Y, (M, N), QX.device)
+    _check(lib.qmm_q8q8_gemv(M, N, K, block, _ptr(W), _ptr(QX), _ptr(DX), _ptr(Y), _stream(stream)),
+           "qmm_q8q8_gemv")
+    return Y
+
+
+def qmm_q8q8_block_dots(W: torch.Tensor, QX: torch.Tensor, N: int, isum: torch.Tensor | None = None, *,
+                        block: int = BLOCK, stream=None) -> torch.Tensor:
+    M, K = QX.shape
+    isum = _out(isum, (M, N, K // BLOCK), QX.device, torch.int32)
+    _check(lib.qmm_q8q8_block_dots(M, N, K, block, _ptr(W), _ptr(QX), _ptr(isum), _stream(stream)),
+           "qmm_q8q8_block_dots")
+    return isum
+
+
+def qmm_q4_swiglu_gateup(Wg: torch.Tensor, Wu: torch.Tensor, X: torch.Tensor, N: int,
+                         Y: torch.Tensor | None = None, *, block: int = BLOCK, stream=None) -> torch.Tensor:
+    M, K = X.shape
+    Y = _out(Y, (M, N), X.device)
+    _check(lib.qmm_q4_swiglu_gateup(M, N, K, block, _ptr(Wg), _ptr(Wu), _ptr(X), _ptr(Y), _stream(stream)),
+           "qmm_q4_swiglu_gateup")
+    return Y
+
+
+def qmm_q4_gateup_unfused(Wg, Wu, X, N, G=None, U=None, Y=None, *, block: int = BLOCK, stream=None):
+    M, K = X.shape
+    G, U, Y = (_out(t, (M, N), X.device) for t in (G, U, Y))
+    _check(lib.qmm_q4_gateup_unfused(M, N, K, block, _ptr(Wg), _ptr(Wu), _ptr(X), _ptr(G), _ptr(U), _ptr(Y),
+                                     _stream(stream)), "qmm_q4_gateup_unfused")
+    return G, U, Y
+
+
+def qmm_quant_matmul_prefill(wtype: int, W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None = None,
+                             *, block: int = BLOCK, stream=None) -> torch.Tensor:
+    """Y[M, N] = bf16 X[M, K] . bf16(dequant(W))^T with fp32 accumulation (tensor cores)."""
+    M, K = X.shape
+    Y = _out(Y, (M, N), X.device)
+    _check(lib.qmm_quant_matmul_prefill(wtype, M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), _stream(stream)),
+           "qmm_quant_matmul_prefill")
+    return Y

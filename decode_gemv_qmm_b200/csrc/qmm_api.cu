@@ -1,0 +1,154 @@
+// qmm_api.cu -- the extern "C" entry points of libqmm.so: argument validation
+// (host only, before any CUDA call), device checks and dispatch to the
+// kernel launchers. The operations themselves are defined in include/qmm.h.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+#include <string>
+
+#include "qmm_internal.h"
+
+namespace qmm {
+
+static thread_local std::string t_last_error;
+
+qmm_status set_error(qmm_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+qmm_status cuda_check(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return QMM_OK;
+  return set_error(QMM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+DevInfo g_dev[kMaxDevices];
+bool g_dev_known[kMaxDevices];
+
+// Attributes of the current device (queried once per device, then cached).
+qmm_status current_device(DevInfo *out) {
+  int d = -1;
+  cudaError_t e = cudaGetDevice(&d);
+  if (e != cudaSuccess) return cuda_check(e, "cudaGetDevice");
+  if (d < 0 || d >= kMaxDevices) return set_error(QMM_ERR_DEVICE, "device ordinal %d out of range", d);
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (!g_dev_known[d]) {
+      DevInfo info;
+      info.device = d;
+      e = cudaDeviceGetAttribute(&info.cc_major, cudaDevAttrComputeCapabilityMajor, d);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&info.cc_minor, cudaDevAttrComputeCapabilityMinor, d);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, d);
+      if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&info.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, d);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&info.l2_bytes, cudaDevAttrL2CacheSize, d);
+      if (e != cudaSuccess) return cuda_check(e, "cudaDeviceGetAttribute");
+      g_dev[d] = info;
+      g_dev_known[d] = true;
+    }
+    *out = g_dev[d];
+  }
+  if (out->cc_major != 10 || out->cc_minor != 0)
+    return set_error(QMM_ERR_DEVICE, "device %d has compute capability %d.%d; this library is built for sm_100a (10.0)",
+                     d, out->cc_major, out->cc_minor);
+  return QMM_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Common checks of (M, N, K, block). `max_m` < 0 means unbounded M.
+qmm_status check_shape(const char *fn, int64_t M, int64_t N, int64_t K, int block, int64_t max_m) {
+  if (block != QMM_BLOCK) return set_error(QMM_ERR_BLOCK, "%s: block=%d, only 32 is supported", fn, block);
+  if (M < 0 || N < 0 || K < 0)
+    return set_error(QMM_ERR_SHAPE, "%s: negative size M=%lld N=%lld K=%lld", fn, (long long)M, (long long)N,
+                     (long long)K);
+  if (K % QMM_BLOCK != 0) return set_error(QMM_ERR_SHAPE, "%s: K=%lld is not a multiple of 32", fn, (long long)K);
+  if (K > QMM_MAX_K) return set_error(QMM_ERR_SHAPE, "%s: K=%lld exceeds %d", fn, (long long)K, QMM_MAX_K);
+  if (max_m >= 0 && M > max_m)
+    return set_error(QMM_ERR_SHAPE, "%s: M=%lld exceeds %lld", fn, (long long)M, (long long)max_m);
+  if (N > (int64_t(1) << 40)) return set_error(QMM_ERR_SHAPE, "%s: N=%lld too large", fn, (long long)N);
+  return QMM_OK;
+}
+
+qmm_status check_ptr(const char *fn, const char *name, const void *p, bool needed, uintptr_t align) {
+  if (!needed) return QMM_OK;
+  if (p == nullptr) return set_error(QMM_ERR_NULL, "%s: %s is NULL", fn, name);
+  if (!aligned(p, align))
+    return set_error(QMM_ERR_ALIGN, "%s: %s=%p is not %u-byte aligned", fn, name, p, (unsigned)align);
+  return QMM_OK;
+}
+
+#define QMM_TRY(expr)                  \
+  do {                                 \
+    qmm_status _st = (expr);           \
+    if (_st != QMM_OK) return _st;     \
+  } while (0)
+
+qmm_status zero_fill(float *Y, int64_t count, cudaStream_t s) {
+  return cuda_check(cudaMemsetAsync(Y, 0, static_cast<size_t>(count) * sizeof(float), s), "cudaMemsetAsync");
+}
+
+}  // namespace
+
+static qmm_status q8_gemv_impl(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
+                               float *Y, qmm_stream_t stream, uint32_t user_flags) {
+  const char *fn = "qmm_q8_gemv";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, N, K, block, QMM_MAX_DECODE_M));
+  if (user_flags & ~uint32_t(QMM_FLAG_EARLY_WEIGHTS))
+    return set_error(QMM_ERR_SHAPE, "%s: unknown flags 0x%x", fn, user_flags);
+  if (M == 0 || N == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "W", W, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "X", X, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "Y", Y, true, 4));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return zero_fill(Y, M * N, s);
+  uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
+  return launch_q8_gemv(dev, static_cast<int>(M), N, static_cast<int>(K), W, X, Y, s, flags);
+}
+
+}  // namespace qmm
+
+using namespace qmm;
+
+extern "C" {
+
+QMM_API qmm_status qmm_q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
+                               float *Y, qmm_stream_t stream) {
+  return q8_gemv_impl(M, N, K, block, W, X, Y, stream, 0u);
+}
+
+QMM_API qmm_status qmm_q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
+                                  float *Y, uint32_t flags, qmm_stream_t stream) {
+  return q8_gemv_impl(M, N, K, block, W, X, Y, stream, flags);
+}
+
+QMM_API const char *qmm_last_error_string(void) { return t_last_error.c_str(); }
+
+QMM_API const char *qmm_version(void) { return "qmm 0.1.0 sm_100a"; }
+
+QMM_API qmm_status qmm_device_status(uint32_t *bits) {
+  if (bits == nullptr) return set_error(QMM_ERR_NULL, "qmm_device_status: bits is NULL");
+  *bits = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_check(e, "cudaDeviceSynchronize");
+  uint32_t b = 0;
+  e = q8_gemv_status(&b);
+  if (e != cudaSuccess) return cuda_check(e, "status read");
+  *bits |= b;
+  return QMM_OK;
+}
+
+}  // extern "C"

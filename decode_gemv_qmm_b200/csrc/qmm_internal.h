@@ -1,0 +1,38 @@
+// qmm_internal.h -- host-side declarations shared by the C-ABI layer and the
+// kernel files (launchers, device info, error recording). Not installed.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qmm.h"
+
+namespace qmm {
+
+struct DevInfo {
+  int device = -1;
+  int sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  int smem_optin = 0;  // max dynamic shared memory per block (opt-in)
+  int l2_bytes = 0;
+};
+
+// Launch options carried from the entry points to the launchers.
+enum : uint32_t {
+  kLaunchPdl = 1u,            // launch with programmatic stream serialization
+  kPrefetchBeforeWait = 2u,   // stream W before the preceding grid has finished
+};
+
+// Record an error message for qmm_last_error_string() and return `st`.
+qmm_status set_error(qmm_status st, const char *fmt, ...);
+// Translate a CUDA error (cudaSuccess -> QMM_OK).
+qmm_status cuda_check(cudaError_t e, const char *what);
+
+// ---- launchers (arguments already validated; sizes > 0) -------------------
+qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
+                          float *Y, cudaStream_t stream, uint32_t flags);
+
+// Device status word of each kernel file: read and clear (synchronous).
+cudaError_t q8_gemv_status(uint32_t *bits);
+
+}  // namespace qmm

@@ -64,6 +64,12 @@
 extern "C" {
 #endif
 
+#if defined(__GNUC__)
+#define QMM_API __attribute__((visibility("default")))
+#else
+#define QMM_API
+#endif
+
 struct CUstream_st; /* cudaStream_t == struct CUstream_st * */
 typedef struct CUstream_st *qmm_stream_t;
 
@@ -90,6 +96,13 @@ typedef enum { QMM_Q8_0 = 0, QMM_Q4_0 = 1 } qmm_wtype;
 /* Largest K of every entry point. */
 #define QMM_MAX_K 32768
 
+/* Option of the *_ex entry points: start streaming the weight blocks before
+ * the preceding kernel in the stream has finished (programmatic dependent
+ * launch; activations are still read only after it has finished). Only valid
+ * when that preceding kernel does not write the weight buffer -- true for
+ * model weights, which are written once at load time. */
+#define QMM_FLAG_EARLY_WEIGHTS 1u
+
 /*
  * qmm_q8_gemv -- decode GEMV / small-M matmul on Q8_0 weights, fp32 activations.
  *
@@ -107,8 +120,13 @@ typedef enum { QMM_Q8_0 = 0, QMM_Q4_0 = 1 } qmm_wtype;
  *   X      M x K fp32 (device, read only, 16-byte aligned)
  *   Y      M x N fp32 (device, written)
  */
-qmm_status qmm_q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
-                       float *Y, qmm_stream_t stream);
+QMM_API qmm_status qmm_q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W,
+                               const float *X, float *Y, qmm_stream_t stream);
+
+/* qmm_q8_gemv with options: flags is 0 or QMM_FLAG_EARLY_WEIGHTS (unknown bits
+ * are QMM_ERR_SHAPE). qmm_q8_gemv(...) == qmm_q8_gemv_ex(..., 0, stream). */
+QMM_API qmm_status qmm_q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                  const float *X, float *Y, uint32_t flags, qmm_stream_t stream);
 
 /*
  * qmm_quantize_act_q8 -- quantise fp32 activations to Q8 codes per 32-block.
@@ -126,7 +144,7 @@ qmm_status qmm_q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W
  *   DX     M x K/32 fp32 scales d (device, written)
  * The codes and scales are bit-exact functions of X.
  */
-qmm_status qmm_quantize_act_q8(int64_t M, int64_t K, int block, const float *X, int8_t *QX,
+QMM_API qmm_status qmm_quantize_act_q8(int64_t M, int64_t K, int block, const float *X, int8_t *QX,
                                float *DX, qmm_stream_t stream);
 
 /*
@@ -144,7 +162,7 @@ qmm_status qmm_quantize_act_q8(int64_t M, int64_t K, int block, const float *X, 
  *          aligned); DX M x K/32 fp32 -- as written by qmm_quantize_act_q8
  *   Y      M x N fp32 (written)
  */
-qmm_status qmm_q8q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W,
+QMM_API qmm_status qmm_q8q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W,
                          const int8_t *QX, const float *DX, float *Y, qmm_stream_t stream);
 
 /*
@@ -164,7 +182,7 @@ qmm_status qmm_q8q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void 
  *   X       M x K fp32 (16-byte aligned)
  *   Y       M x N fp32 (written)
  */
-qmm_status qmm_q4_swiglu_gateup(int64_t M, int64_t N, int64_t K, int block, const void *Wg,
+QMM_API qmm_status qmm_q4_swiglu_gateup(int64_t M, int64_t N, int64_t K, int block, const void *Wg,
                                 const void *Wu, const float *X, float *Y, qmm_stream_t stream);
 
 /*
@@ -182,7 +200,7 @@ qmm_status qmm_q4_swiglu_gateup(int64_t M, int64_t N, int64_t K, int block, cons
  *   X       M x K bf16 bit patterns (uint16_t, 16-byte aligned)
  *   Y       M x N fp32 (written)
  */
-qmm_status qmm_quant_matmul_prefill(int wtype, int64_t M, int64_t N, int64_t K, int block,
+QMM_API qmm_status qmm_quant_matmul_prefill(int wtype, int64_t M, int64_t N, int64_t K, int block,
                                     const void *W, const uint16_t *X, float *Y,
                                     qmm_stream_t stream);
 
@@ -195,7 +213,7 @@ qmm_status qmm_quant_matmul_prefill(int wtype, int64_t M, int64_t N, int64_t K, 
  * Computed by the same device code as qmm_q8q8_gemv; used to test the integer
  * part bit-exactly.
  */
-qmm_status qmm_q8q8_block_dots(int64_t M, int64_t N, int64_t K, int block, const void *W,
+QMM_API qmm_status qmm_q8q8_block_dots(int64_t M, int64_t N, int64_t K, int block, const void *W,
                                const int8_t *QX, int32_t *isum, qmm_stream_t stream);
 
 /*
@@ -206,15 +224,15 @@ qmm_status qmm_q8q8_block_dots(int64_t M, int64_t N, int64_t K, int block, const
  * so Y matches qmm_q4_swiglu_gateup bit for bit ("LSE v0.4.16", section
  * "Combined M8 Q4 gate/up execution": exact outputs preserved).
  */
-qmm_status qmm_q4_gateup_unfused(int64_t M, int64_t N, int64_t K, int block, const void *Wg,
+QMM_API qmm_status qmm_q4_gateup_unfused(int64_t M, int64_t N, int64_t K, int block, const void *Wg,
                                  const void *Wu, const float *X, float *G, float *U, float *Y,
                                  qmm_stream_t stream);
 
 /* Text of the last error raised on the calling host thread ("" if none). */
-const char *qmm_last_error_string(void);
+QMM_API const char *qmm_last_error_string(void);
 
 /* Library version string, e.g. "qmm 0.1.0 sm_100a". */
-const char *qmm_version(void);
+QMM_API const char *qmm_version(void);
 
 /*
  * qmm_device_status -- synchronises the current device, then reads and clears
@@ -222,7 +240,7 @@ const char *qmm_version(void);
  * *bits receives the word (0 = no failure recorded). Returns QMM_OK, or
  * QMM_ERR_CUDA if the synchronisation itself failed.
  */
-qmm_status qmm_device_status(uint32_t *bits);
+QMM_API qmm_status qmm_device_status(uint32_t *bits);
 
 #ifdef __cplusplus
 }
