@@ -8,43 +8,53 @@
 //
 //   Y[m][n] = sum_b d[n][b] * sum_j q[n][b][j] * X[m][32b + j]
 //
-// B200 design (HBM-bound stream of 34-byte blocks):
-//  * Each CTA owns a contiguous range of rows, i.e. a contiguous byte range of
-//    W. One thread streams it through a ring of shared-memory stages with 1-D
-//    bulk copies (cp.async.bulk, completion on an mbarrier). Copies are widened
-//    to 16-byte boundaries; the <16-byte tail of the whole matrix is copied
-//    with plain loads so nothing past the end of W is read.
-//  * Lane l of a warp owns block column c = 32*window + l and keeps the 32
-//    activations of that column in registers for the whole kernel; warps of a
-//    CTA split the K blocks into 32-column windows (split-K across warps) and
-//    the rows of a stage. A lane reads its block from shared memory with nine
-//    aligned 32-bit loads and funnel shifts (blocks are only 2-byte aligned).
+// B200 design (a stream of 34-byte blocks; HBM-bound when the integer pipe
+// keeps up):
+//  * Each CTA owns a contiguous range of rows = a contiguous byte range of W.
+//    A producer warp streams it through a ring of shared-memory stages with
+//    1-D bulk copies (cp.async.bulk, completion counted on a "full" mbarrier);
+//    consumer warps release a stage through an "empty" mbarrier, so warps
+//    never wait for each other. Copies are widened to 16-byte boundaries; the
+//    <16-byte tail of the whole matrix is copied with plain loads so nothing
+//    past the end of W is read.
+//  * Lane l of a consumer warp owns block column c = 32*window + l and keeps
+//    the 32 activations of that column in registers; consumer warps split the
+//    K blocks into 32-column windows (split-K across warps) and the rows of a
+//    stage. A lane reads its 2-byte-aligned block with nine aligned 32-bit
+//    shared loads and funnel shifts.
 //  * int8 -> fp32 without a conversion instruction: the code byte (biased by
-//    128) is placed in the mantissa of 2^23 with one byte-permute, and one
-//    packed fp32x2 add removes 2^23 + 128 exactly. The products use packed
-//    fp32x2 FMAs. Each block is summed in four fp32 chains, scaled by d,
-//    then reduced across the warp (shuffles) and across windows (shared
-//    memory) in a fixed order, so results are deterministic.
+//    128) is placed in the mantissa of 2^23 by one byte-permute, and a packed
+//    fp32x2 add removes 2^23 + 128 exactly; products use packed fp32x2 FMAs.
+//    (On sm_100 the byte permute issues at half rate, so it bounds the
+//    kernel; everything else is kept off the integer pipe where possible.)
+//  * A warp processes RG rows at a time (independent chains for latency
+//    hiding) and reduces their partial sums across lanes with one
+//    reduce-scatter butterfly. Windows of a row are summed by the producer
+//    warp in a fixed order, so results are deterministic.
 //  * Programmatic dependent launch: with the "early weights" option the ring
 //    is filled before griddepcontrol.wait (W must not be written by the
-//    preceding kernel); X and Y are touched only after it.
+//    preceding kernel); X and Y are touched only after it. The CTA footprint
+//    is small enough for two launches to share an SM.
 #include <algorithm>
 
 #include "qmm_common.cuh"
 #include "qmm_internal.h"
+#include "qmm_tmap.h"
 
 namespace qmm {
 namespace {
 
 static __device__ uint32_t g_q8_gemv_status;
 
-constexpr int kMaxWarps = 16;
 constexpr int kMaxStages = 8;
-constexpr int kStageTarget = 32 * 1024;  // bytes of W per stage (aim)
-constexpr int kSmemBudget = 100 * 1024;  // two CTAs of consecutive launches fit one SM
-constexpr int kBarBytes = 128;           // mbarrier area at the start of shared memory
+constexpr int kStageTarget = 16 * 1024;  // bytes of W per stage (aim)
+constexpr int kSmemBudget = 96 * 1024;   // two CTAs of consecutive launches fit one SM
+constexpr int kBarBytes = 256;           // full[8] + empty[8] mbarriers
+constexpr int kMaxConsumerWarps = 16;
+constexpr int kPanelBytes = 32 * 1024;  // activation panel kept in shared memory up to this size (256 rows)
 
-struct Params {
+struct alignas(64) Params {
+  CUtensorMap xmap;  // X viewed as (M*K/32) rows of 128 bytes, 128-byte swizzle
   const uint8_t *W;
   const float *X;
   float *Y;
@@ -57,116 +67,246 @@ struct Params {
   int stages;
   int stage_bytes;
   int stage_off;
+  int xs_off;  // byte offset of the activation panel in shared memory (0 = no panel)
+  int xs_rows;  // rows of 32 activations in the panel (M * K / 32)
   int cg;  // 32-column windows = ceil(KB / 32)
-  int cs;  // column slots (warps side by side along K)
-  int rs;  // row slots (warps side by side along N)
+  int cs;  // column slots (consumer warps side by side along K)
+  int rs;  // row slots (consumer warps side by side along N)
   int prefetch_before_wait;
 };
 
-// d * sum_j q_j x_j for one Q8_0 block at `blk` (2-byte aligned, shared memory).
+// Convert four int8 codes (one 32-bit word) and multiply-accumulate them
+// against four activations held as two float2 pairs.
+__device__ __forceinline__ void fma4(uint32_t qword, const float2 &x01, const float2 &x23, float2 &a01,
+                                     float2 &a23) {
+  const float2 neg_bias = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
+  const uint32_t q4 = qword ^ 0x80808080u;                        // bytes q + 128
+  float2 f01 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7440u)),
+                           __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7441u)));
+  float2 f23 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7442u)),
+                           __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7443u)));
+  f01 = __fadd2_rn(f01, neg_bias);  // exact: 2^23 + 128 + q - (2^23 + 128) = q
+  f23 = __fadd2_rn(f23, neg_bias);
+  a01 = __ffma2_rn(f01, x01, a01);
+  a23 = __ffma2_rn(f23, x23, a23);
+}
+
+// d * sum_j q_j x_j of one Q8_0 block at shared address `sa` (2-byte aligned)
+// for MP activation rows. Each 4-weight word feeds its own accumulator pair;
+// the pairs are summed in a fixed tree, which keeps the dependent chain short.
 template <int MP>
-__device__ __forceinline__ void q8_block_dot(const uint8_t *blk, const float2 (&x2)[MP][16],
-                                             float (&out)[MP]) {
-  const uint32_t mis = static_cast<uint32_t>(reinterpret_cast<uintptr_t>(blk)) & 2u;
-  const uint32_t *wp = reinterpret_cast<const uint32_t *>(blk - mis);
+__device__ __forceinline__ void q8_block_dot(uint32_t sa, const float2 (&x2)[MP][16], float (&out)[MP]) {
+  const uint32_t mis = sa & 2u;
+  const uint32_t wa = sa - mis;
   uint32_t w[9];
 #pragma unroll
-  for (int k = 0; k < 9; ++k) w[k] = wp[k];
+  for (int k = 0; k < 9; ++k) w[k] = lds_u32(wa + 4 * k);
   const uint32_t r8 = mis << 3;  // 0 or 16: bit offset of d inside w[0]
   const float d = half_bits_to_float(__funnelshift_rc(w[0], w[1], r8));
   const uint32_t sh = 16u + r8;  // 16 or 32: bit offset of qs inside (w[i+1]:w[i])
-  const float2 neg_bias = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
-  float2 acc[MP][2];
 #pragma unroll
-  for (int m = 0; m < MP; ++m) acc[m][0] = acc[m][1] = make_float2(0.f, 0.f);
+  for (int m = 0; m < MP; ++m) {
+    float2 a[8], b[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t q4 = __funnelshift_rc(w[i], w[i + 1], sh) ^ 0x80808080u;  // bytes q + 128
-    float2 f01 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7440u)),
-                             __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7441u)));
-    float2 f23 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7442u)),
-                             __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7443u)));
-    f01 = __fadd2_rn(f01, neg_bias);  // exact: 2^23 + 128 + q - (2^23 + 128) = q
-    f23 = __fadd2_rn(f23, neg_bias);
-#pragma unroll
-    for (int m = 0; m < MP; ++m) {
-      acc[m][0] = __ffma2_rn(f01, x2[m][2 * i], acc[m][0]);
-      acc[m][1] = __ffma2_rn(f23, x2[m][2 * i + 1], acc[m][1]);
+    for (int i = 0; i < 8; ++i) {
+      a[i] = b[i] = make_float2(0.f, 0.f);
+      fma4(__funnelshift_rc(w[i], w[i + 1], sh), x2[m][2 * i], x2[m][2 * i + 1], a[i], b[i]);
     }
-  }
 #pragma unroll
-  for (int m = 0; m < MP; ++m)
-    out[m] = d * ((acc[m][0].x + acc[m][0].y) + (acc[m][1].x + acc[m][1].y));
+    for (int st = 1; st < 8; st *= 2) {
+#pragma unroll
+      for (int i = 0; i < 8; i += 2 * st) {
+        a[i] = __fadd2_rn(a[i], a[i + st]);
+        b[i] = __fadd2_rn(b[i], b[i + st]);
+      }
+    }
+    const float2 t = __fadd2_rn(a[0], b[0]);
+    out[m] = d * (t.x + t.y);
+  }
 }
 
-template <int MP>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) q8_gemv_kernel(const __grid_constant__ Params p) {
+// Reduce V per-lane values over the 32 lanes with a reduce-scatter butterfly:
+// afterwards lane l holds the total of value index vidx(l) (V in {1, 2, 4}).
+template <int V>
+__device__ __forceinline__ float warp_reduce_scatter(float (&v)[V], int lane) {
+  if constexpr (V == 4) {
+    const bool hi16 = lane & 16;
+    float k0 = hi16 ? v[2] : v[0], k1 = hi16 ? v[3] : v[1];
+    const float s0 = hi16 ? v[0] : v[2], s1 = hi16 ? v[1] : v[3];
+    k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    const bool hi8 = lane & 8;
+    float k = hi8 ? k1 : k0;
+    k += __shfl_xor_sync(0xffffffffu, hi8 ? k0 : k1, 8);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+    return k;  // value index ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1)
+  } else if constexpr (V == 2) {
+    const bool hi16 = lane & 16;
+    float k = hi16 ? v[1] : v[0];
+    k += __shfl_xor_sync(0xffffffffu, hi16 ? v[0] : v[1], 16);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+    return k;  // value index (lane >> 4) & 1
+  } else {
+    float k = v[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+    return k;
+  }
+}
+template <int V>
+__device__ __forceinline__ int scatter_index(int lane) {
+  if constexpr (V == 4) return ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+  if constexpr (V == 2) return (lane >> 4) & 1;
+  return 0;
+}
+template <int V>
+__device__ __forceinline__ bool scatter_writer(int lane) {
+  if constexpr (V == 4) return (lane & 7) == 0;
+  if constexpr (V == 2) return (lane & 15) == 0;
+  return lane == 0;
+}
+
+// MP activation rows per pass (1 or 2); RG weight rows per warp step.
+template <int MP, int RG>
+__global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *empty = full + kMaxStages;
+  uint64_t *xbar = empty + kMaxStages;
   float *red = reinterpret_cast<float *>(smem + kBarBytes);
   uint8_t *stage_mem = smem + p.stage_off;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nconsumer = p.cs * p.rs;
   const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * p.N / p.grid;
   const int64_t r_end = static_cast<int64_t>(blockIdx.x + 1) * p.N / p.grid;
   const int nrows = static_cast<int>(r_end - r_begin);
   const int nchunks = (nrows + p.rows_chunk - 1) / p.rows_chunk;
   const int S = p.stages;
+  const int red_stride = p.M * p.cg * p.rows_chunk;  // floats of partials per stage
 
+  // Let the next launch in the stream start its prologue (weight prefetch) as
+  // soon as SM resources allow; its own griddepcontrol.wait still orders it.
+  pdl_launch_dependents();
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], nconsumer);
+    }
+    mbar_init(xbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
 
-  // Producer (thread 0): copy the bytes of chunk `c` into stage c % S.
-  uint64_t policy = 0;
-  int issued = 0;
-  auto issue = [&](int c) {
-    const int s = c % S;
-    const int64_t r0 = r_begin + static_cast<int64_t>(c) * p.rows_chunk;
-    const int64_t r1 = min(r0 + p.rows_chunk, r_end);
-    const int64_t b0 = r0 * p.row_bytes, b1 = r1 * p.row_bytes;
-    const int64_t a0 = b0 & ~int64_t(15);
-    int64_t a1 = (b1 + 15) & ~int64_t(15);
-    const int64_t lim = p.total_bytes & ~int64_t(15);
-    uint8_t *dst = stage_mem + static_cast<int64_t>(s) * p.stage_bytes;
-    if (a1 > lim) {  // last chunk of W: bytes past the last 16-byte boundary by hand
-      for (int64_t t = lim; t < b1; ++t) dst[t - a0] = p.W[t];
-      a1 = lim;
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint64_t policy = 0;
+    auto issue = [&](int c) {
+      const int s = c % S;
+      const int64_t r0 = r_begin + static_cast<int64_t>(c) * p.rows_chunk;
+      const int64_t r1 = min(r0 + p.rows_chunk, r_end);
+      const int64_t b0 = r0 * p.row_bytes, b1 = r1 * p.row_bytes;
+      const int64_t a0 = b0 & ~int64_t(15);
+      int64_t a1 = (b1 + 15) & ~int64_t(15);
+      const int64_t lim = p.total_bytes & ~int64_t(15);
+      uint8_t *dst = stage_mem + static_cast<int64_t>(s) * p.stage_bytes;
+      if (a1 > lim) {  // last chunk of W: bytes past the last 16-byte boundary by hand
+        for (int64_t t = lim; t < b1; ++t) dst[t - a0] = p.W[t];
+        a1 = lim;
+      }
+      const uint32_t bytes = static_cast<uint32_t>(a1 - a0);
+      mbar_arrive_expect_tx(&full[s], bytes);
+      if (bytes) bulk_g2s(dst, p.W + a0, bytes, &full[s], policy);
+    };
+    // Sum the window partials of chunk c (all consumers have released it).
+    auto finish = [&](int c) {
+      if (p.cg == 1) return;
+      const int s = c % S;
+      const int64_t r0 = r_begin + static_cast<int64_t>(c) * p.rows_chunk;
+      const int rows = static_cast<int>(min(static_cast<int64_t>(p.rows_chunk), r_end - r0));
+      const float *rb = red + s * red_stride;
+      for (int t = lane; t < p.M * rows; t += 32) {
+        const int m = t / rows, rl = t - m * rows;
+        const float *src = rb + m * p.cg * p.rows_chunk + rl;
+        float v = src[0];
+        for (int cw = 1; cw < p.cg; ++cw) v += src[cw * p.rows_chunk];
+        p.Y[static_cast<int64_t>(m) * p.N + r0 + rl] = v;
+      }
+    };
+    // The activation panel: one 2-D TMA load with the 128-byte swizzle, issued
+    // as soon as the preceding grid has finished (X may be its output).
+    auto issue_x = [&]() {
+      if (p.xs_off) {
+        mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(p.xs_rows) * 128u);
+        tma_load_2d(smem + p.xs_off, &p.xmap, 0, 0, xbar);
+      }
+    };
+    const int prologue = min(S, nchunks);
+    if (p.prefetch_before_wait) {
+      if (lane == 0) {
+        policy = l2_evict_first_policy();
+        for (int c = 0; c < prologue; ++c) issue(c);
+      }
+      pdl_wait();
+      if (lane == 0) issue_x();
+    } else {
+      pdl_wait();
+      if (lane == 0) {
+        issue_x();
+        policy = l2_evict_first_policy();
+        for (int c = 0; c < prologue; ++c) issue(c);
+      }
     }
-    const uint32_t bytes = static_cast<uint32_t>(a1 - a0);
-    mbar_arrive_expect_tx(&full[s], bytes);
-    if (bytes) bulk_g2s(dst, p.W + a0, bytes, &full[s], policy);
-  };
-  const int prologue = min(S, nchunks);
-  if (p.prefetch_before_wait) {
-    if (tid == 0) {
-      policy = l2_evict_first_policy();
-      for (; issued < prologue; ++issued) issue(issued);
+    bool ok = true;
+    int issued = prologue;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      // chunk c is released once every consumer warp arrived on empty[c % S]
+      ok = mbar_wait(&empty[c % S], static_cast<uint32_t>(c / S) & 1u);
+      if (!ok) break;
+      __syncwarp();
+      finish(c);
+      __syncwarp();
+      if (lane == 0 && issued < nchunks) {
+        issue(issued);
+        ++issued;
+      }
     }
-    pdl_wait();
-  } else {
-    pdl_wait();
-    if (tid == 0) {
-      policy = l2_evict_first_policy();
-      for (; issued < prologue; ++issued) issue(issued);
+    if (!ok && lane == 0) {  // error path: record, then drain copies still in flight
+      atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+      for (int c = max(0, issued - S); c < issued; ++c)
+        if (!mbar_wait(&full[c % S], static_cast<uint32_t>(c / S) & 1u))
+          atomicOr(&g_q8_gemv_status, kDevTimeoutDrain);
     }
+    return;
   }
-  pdl_launch_dependents();
 
-  const int cs_w = warp % p.cs, rs_w = warp / p.cs;
+  // -------------------------------------------------------------- consumers
+  pdl_wait();
+  const int cwarp = warp - 1;
+  const int cs_w = cwarp % p.cs, rs_w = cwarp / p.cs;
+  // Activation panel (when present): row r = m * KB + c holds the 32
+  // activations of block column c of token m; the TMA's 128-byte swizzle puts
+  // 16-byte unit u of row r at unit u ^ (r & 7), so the eight lanes of a
+  // shared-memory phase (consecutive c) read eight different bank groups.
+  const bool xs = p.xs_off != 0;
+  const uint32_t xs_sa = smem_u32(smem) + p.xs_off;
+  if (xs && !mbar_wait(xbar, 0)) {
+    if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+    return;
+  }
   float2 x2[MP][16];
   auto load_x = [&](int m0, int cw) {
     const int c = cw * 32 + lane;
 #pragma unroll
     for (int m = 0; m < MP; ++m) {
       if (c < p.KB && m0 + m < p.M) {
-        const float4 *src =
-            reinterpret_cast<const float4 *>(p.X + static_cast<int64_t>(m0 + m) * p.K + c * 32);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float4 v = __ldg(src + j);
+          const int row = (m0 + m) * p.KB + c;
+          const float4 v = xs ? lds_f4(xs_sa + 16u * (row * 8 + (j ^ (row & 7))))
+                              : __ldg(reinterpret_cast<const float4 *>(p.X + static_cast<int64_t>(m0 + m) * p.K) + 8 * c + j);
           x2[m][2 * j] = make_float2(v.x, v.y);
           x2[m][2 * j + 1] = make_float2(v.z, v.w);
         }
@@ -179,75 +319,71 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) q8_gemv_kernel(const __grid
   const bool x_cached = (p.cg == p.cs) && (p.M <= MP);
   if (x_cached) load_x(0, cs_w);
 
-  bool bad = false;
-  int chunk = 0;
-  for (; chunk < nchunks; ++chunk) {
-    const int s = chunk % S;
-    const bool ok = mbar_wait(&full[s], static_cast<uint32_t>(chunk / S) & 1u);
-    if (!ok) bad = true;
-    const int64_t r0 = r_begin + static_cast<int64_t>(chunk) * p.rows_chunk;
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = c % S;
+    if (!mbar_wait(&full[s], static_cast<uint32_t>(c / S) & 1u)) {
+      if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+      return;  // the producer times out on this warp's missing arrival and drains
+    }
+    const int64_t r0 = r_begin + static_cast<int64_t>(c) * p.rows_chunk;
     const int rows = static_cast<int>(min(static_cast<int64_t>(p.rows_chunk), r_end - r0));
-    const int64_t byte0 = r0 * p.row_bytes;
-    const uint8_t *base = stage_mem + static_cast<int64_t>(s) * p.stage_bytes + (byte0 & 15);
-    float *redb = red + (chunk & 1) * p.M * p.cg * p.rows_chunk;
-    if (ok) {
-      for (int m0 = 0; m0 < p.M; m0 += MP) {
-        for (int cw = cs_w; cw < p.cg; cw += p.cs) {
-          if (!x_cached) load_x(m0, cw);
-          const int c = cw * 32 + lane;
-          const bool act = c < p.KB;
-          for (int rl = rs_w; rl < rows; rl += p.rs) {
-            float part[MP];
-            if (act) {
-              q8_block_dot<MP>(base + static_cast<int64_t>(rl) * p.row_bytes + 34 * c, x2, part);
-            } else {
+    const uint32_t base = smem_u32(stage_mem) + s * p.stage_bytes + static_cast<uint32_t>((r0 * p.row_bytes) & 15);
+    float *rb = red + s * red_stride;
+    for (int m0 = 0; m0 < p.M; m0 += MP) {
+      for (int cw = cs_w; cw < p.cg; cw += p.cs) {
+        if (!x_cached) load_x(m0, cw);
+        const int col = cw * 32 + lane;
+        const bool act = col < p.KB;
+        // Lanes past the last block column and rows past the chunk compute on a
+        // valid in-bounds block and discard the result: no branch, so the RG
+        // block dots of a step can be interleaved by the scheduler.
+        const uint32_t col_off = 34u * static_cast<uint32_t>(act ? col : p.KB - 1);
+        for (int rl = rs_w * RG; rl < rows; rl += p.rs * RG) {
+          float part[RG * MP];
 #pragma unroll
-              for (int m = 0; m < MP; ++m) part[m] = 0.f;
-            }
+          for (int g = 0; g < RG; ++g) {
+            const bool ok = act && rl + g < rows;
+            const int row = min(rl + g, rows - 1);
+            float o[MP];
+            q8_block_dot<MP>(base + static_cast<uint32_t>(row * p.row_bytes) + col_off, x2, o);
 #pragma unroll
-            for (int m = 0; m < MP; ++m) {
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) part[m] += __shfl_xor_sync(0xffffffffu, part[m], o);
-            }
-            if (lane == 0) {
-#pragma unroll
-              for (int m = 0; m < MP; ++m) {
-                if (m0 + m < p.M) {
-                  if (p.cg == 1)
-                    p.Y[static_cast<int64_t>(m0 + m) * p.N + r0 + rl] = part[m];
-                  else
-                    redb[((m0 + m) * p.cg + cw) * p.rows_chunk + rl] = part[m];
-                }
-              }
+            for (int m = 0; m < MP; ++m) part[g * MP + m] = ok ? o[m] : 0.f;
+          }
+          const float tot = warp_reduce_scatter<RG * MP>(part, lane);
+          if (scatter_writer<RG * MP>(lane)) {
+            const int v = scatter_index<RG * MP>(lane);
+            const int g = v / MP, m = m0 + v % MP;
+            if (rl + g < rows && m < p.M) {
+              if (p.cg == 1)
+                p.Y[static_cast<int64_t>(m) * p.N + r0 + rl + g] = tot;
+              else
+                rb[(m * p.cg + cw) * p.rows_chunk + rl + g] = tot;
             }
           }
         }
       }
     }
-    if (__syncthreads_or(bad)) break;  // uniform exit if any thread gave up
-    if (tid == 0 && issued < nchunks) {
-      issue(issued);  // refill the stage everyone just finished with
-      ++issued;
-    }
-    if (p.cg > 1) {  // sum the windows of each row in a fixed order
-      for (int t = tid; t < p.M * rows; t += blockDim.x) {
-        const int m = t / rows, rl = t - m * rows;
-        const float *src = redb + m * p.cg * p.rows_chunk + rl;
-        float v = src[0];
-        for (int cw = 1; cw < p.cg; ++cw) v += src[cw * p.rows_chunk];
-        p.Y[static_cast<int64_t>(m) * p.N + r0 + rl] = v;
-      }
-    }
-  }
-  if (chunk < nchunks && tid == 0) {  // error path: record, then drain copies in flight
-    atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
-    for (int c = chunk; c < issued; ++c)
-      if (!mbar_wait(&full[c % S], static_cast<uint32_t>(c / S) & 1u))
-        atomicOr(&g_q8_gemv_status, kDevTimeoutDrain);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
 }
 
 int align_up(int64_t v, int a) { return static_cast<int>((v + a - 1) / a * a); }
+
+template <int MP, int RG>
+cudaError_t launch(const cudaLaunchConfig_t &cfg, const Params &p) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    int optin = 0;
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaError_t e = cudaFuncSetAttribute(q8_gemv_kernel<MP, RG>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  return cudaLaunchKernelEx(&cfg, q8_gemv_kernel<MP, RG>, p);
+}
 
 }  // namespace
 
@@ -264,13 +400,27 @@ qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
   p.row_bytes = 34ll * p.KB;
   p.total_bytes = N * p.row_bytes;
   p.cg = (p.KB + 31) / 32;
-  p.cs = std::min(p.cg, kMaxWarps);
-  p.rs = std::max(1, kMaxWarps / p.cs);
-  const int threads = p.cs * p.rs * 32;
-  p.grid = static_cast<int>(std::min<int64_t>(N, dev.sms));
+  // consumer warps: the K windows side by side, then rows
+  // Small problems: few rows per CTA, so a lean CTA (more launches resident
+  // per SM under programmatic dependent launch); large problems: two CTAs per SM.
+  const int64_t rows_one_wave = (N + dev.sms - 1) / dev.sms;
+  p.cs = std::min(p.cg, kMaxConsumerWarps);
+  p.rs = p.cs > 1 ? std::max(1, 10 / p.cs) : (rows_one_wave <= 16 ? 4 : 8);
+  const int nconsumer = p.cs * p.rs;
+  const int threads = (nconsumer + 1) * 32;
+  const int64_t ctas_per_sm = rows_one_wave >= 128 ? 2 : 1;
+  p.grid = static_cast<int>(std::min<int64_t>(N, dev.sms * ctas_per_sm));
   const int64_t rows_max = (N + p.grid - 1) / p.grid;
+  // rows per warp step: more rows amortise the cross-lane reduction, but every
+  // row-slot warp should get work when a CTA owns only a few rows
+  int rg = 1;
+  if (M == 1) {
+    if (rows_max >= 4ll * p.rs * 2) rg = 4;
+    else if (rows_max >= 2ll * p.rs) rg = 2;
+  }
   int64_t rc = std::max<int64_t>(1, kStageTarget / p.row_bytes);
-  if (rc >= p.rs) rc = rc / p.rs * p.rs;
+  const int64_t quantum = static_cast<int64_t>(p.rs) * rg;
+  rc = (rc >= quantum) ? rc / quantum * quantum : quantum;
   rc = std::min<int64_t>(rc, rows_max);
   p.rows_chunk = static_cast<int>(rc);
   // data + up to 15 bytes of alignment slack in front + over-read of the last block
@@ -279,8 +429,20 @@ qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
   int S = std::max(1, kSmemBudget / p.stage_bytes);
   S = static_cast<int>(std::min<int64_t>({S, kMaxStages, nchunks_max}));
   p.stages = S;
-  const int red_bytes = p.cg > 1 ? 2 * M * p.cg * p.rows_chunk * 4 : 0;
-  p.stage_off = kBarBytes + align_up(red_bytes, 128);
+  const int red_bytes = p.cg > 1 ? S * M * p.cg * p.rows_chunk * 4 : 0;
+  const int64_t xs_bytes = static_cast<int64_t>(M) * K * 4;
+  const bool panel = xs_bytes <= kPanelBytes;
+  p.xs_off = panel ? align_up(kBarBytes + red_bytes, 1024) : 0;  // 128-byte swizzle needs 1024-byte alignment
+  p.xs_rows = panel ? static_cast<int>(xs_bytes / 128) : 0;
+  p.stage_off = panel ? align_up(p.xs_off + xs_bytes, 128) : kBarBytes + align_up(red_bytes, 128);
+  if (panel) {
+    const uint64_t dims[2] = {32, static_cast<uint64_t>(p.xs_rows)};
+    const uint64_t strides[1] = {128};
+    const uint32_t box[2] = {32, static_cast<uint32_t>(p.xs_rows)};
+    qmm_status st = encode_tiled(&p.xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, X, dims, strides, box,
+                                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != QMM_OK) return st;
+  }
   const size_t smem = static_cast<size_t>(p.stage_off) + static_cast<size_t>(S) * p.stage_bytes;
   if (smem > static_cast<size_t>(dev.smem_optin))
     return set_error(QMM_ERR_SHAPE, "q8_gemv: K=%d needs %zu bytes of shared memory", K, smem);
@@ -297,15 +459,10 @@ qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (M == 1) {
-    e = cudaFuncSetAttribute(q8_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, q8_gemv_kernel<1>, p);
-  } else {
-    e = cudaFuncSetAttribute(q8_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, q8_gemv_kernel<2>, p);
-  }
+  if (M > 1) e = launch<2, 1>(cfg, p);
+  else if (rg == 4) e = launch<1, 4>(cfg, p);
+  else if (rg == 2) e = launch<1, 2>(cfg, p);
+  else e = launch<1, 1>(cfg, p);
   return cuda_check(e, "q8_gemv launch");
 }
 
