@@ -38,6 +38,7 @@ _SIGS = {
     "qmm_q8_gemv_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _u32, _p],
     "qmm_quantize_act_q8": [_i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q8q8_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
+    "qmm_q8q8_gemv_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
     "qmm_q4_swiglu_gateup": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_quant_matmul_prefill": [_int, _i64, _i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q8q8_block_dots": [_i64, _i64, _i64, _int, _p, _p, _p, _p],
@@ -126,11 +127,15 @@ def qmm_quantize_act_q8(X: torch.Tensor, QX: torch.Tensor | None = None, DX: tor
 
 
 def qmm_q8q8_gemv(W: torch.Tensor, QX: torch.Tensor, DX: torch.Tensor, N: int, Y: torch.Tensor | None = None, *,
-                  block: int = BLOCK, stream=None) -> torch.Tensor:
+                  block: int = BLOCK, flags: int = 0, stream=None) -> torch.Tensor:
+    """Y[M, N] from Q8_0 blocks W and Q8 activation codes QX with block scales DX."""
     M, K = QX.shape
     Y = _out(Y, (M, N), QX.device)
-    _check(lib.qmm_q8q8_gemv(M, N, K, block, _ptr(W), _ptr(QX), _ptr(DX), _ptr(Y), _stream(stream)),
-           "qmm_q8q8_gemv")
+    if flags:
+        st = lib.qmm_q8q8_gemv_ex(M, N, K, block, _ptr(W), _ptr(QX), _ptr(DX), _ptr(Y), flags, _stream(stream))
+    else:
+        st = lib.qmm_q8q8_gemv(M, N, K, block, _ptr(W), _ptr(QX), _ptr(DX), _ptr(Y), _stream(stream))
+    _check(st, "qmm_q8q8_gemv")
     return Y
 
 

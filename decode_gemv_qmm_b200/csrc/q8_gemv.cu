@@ -8,6 +8,15 @@
 //
 //   Y[m][n] = sum_b d[n][b] * sum_j q[n][b][j] * X[m][32b + j]
 //
+// The same streaming kernel also runs the Q8xQ8 variant ("Lumen v0.4.0 --
+// shape-aware VNNI/fp32 hybrid dispatch", section "Phase 7.M -- Q8xQ8 AVX2 int
+// dot"): activations quantised to int8 per 32-block (scale DX); each block's
+// dot of weight codes and activation codes is an exact int32 (eight dp4a
+// steps over 4-byte words), scaled by d_w * d_x in fp32:
+//
+//   isum[m][n][b] = sum_j q[n][b][j] * QX[m][32b + j]   (exact)
+//   Y[m][n]       = sum_b (d[n][b] * DX[m][b]) * isum[m][n][b]
+//
 // B200 design (a stream of 34-byte blocks; HBM-bound when the integer pipe
 // keeps up):
 //  * Each CTA owns a contiguous range of rows = a contiguous byte range of W.
@@ -53,11 +62,16 @@ constexpr int kBarBytes = 256;           // full[8] + empty[8] mbarriers
 constexpr int kMaxConsumerWarps = 16;
 constexpr int kPanelBytes = 32 * 1024;  // activation panel kept in shared memory up to this size (256 rows)
 
+enum : int { kModeF32 = 0, kModeQ8 = 1, kModeQ8Dots = 2 };
+
 struct alignas(64) Params {
   CUtensorMap xmap;  // X viewed as (M*K/32) rows of 128 bytes, 128-byte swizzle
   const uint8_t *W;
-  const float *X;
+  const float *X;    // fp32 activations (kModeF32)
+  const int8_t *QX;  // int8 activation codes (kModeQ8, kModeQ8Dots)
+  const float *DX;   // per-block activation scales (kModeQ8)
   float *Y;
+  int32_t *isum;     // block dots out (kModeQ8Dots)
   int64_t N;
   int64_t row_bytes;
   int64_t total_bytes;
@@ -69,6 +83,7 @@ struct alignas(64) Params {
   int stage_off;
   int xs_off;  // byte offset of the activation panel in shared memory (0 = no panel)
   int xs_rows;  // rows of 32 activations in the panel (M * K / 32)
+  int xs_bytes;  // panel bytes
   int cg;  // 32-column windows = ceil(KB / 32)
   int cs;  // column slots (consumer warps side by side along K)
   int rs;  // row slots (consumer warps side by side along N)
@@ -125,6 +140,31 @@ __device__ __forceinline__ void q8_block_dot(uint32_t sa, const float2 (&x2)[MP]
   }
 }
 
+// Exact int32 dot of one Q8_0 block's codes with MP rows of int8 activation
+// codes (eight 4-byte words each); also returns the block's scale d.
+template <int MP>
+__device__ __forceinline__ float q8q8_block_isum(uint32_t sa, const uint32_t (&qx)[MP][8], int (&isum)[MP]) {
+  const uint32_t mis = sa & 2u;
+  const uint32_t wa = sa - mis;
+  uint32_t w[9];
+#pragma unroll
+  for (int k = 0; k < 9; ++k) w[k] = lds_u32(wa + 4 * k);
+  const uint32_t r8 = mis << 3;
+  const float d = half_bits_to_float(__funnelshift_rc(w[0], w[1], r8));
+  const uint32_t sh = 16u + r8;
+#pragma unroll
+  for (int m = 0; m < MP; ++m) {
+    int s0 = 0, s1 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      s0 = __dp4a(static_cast<int>(__funnelshift_rc(w[i], w[i + 1], sh)), static_cast<int>(qx[m][i]), s0);
+      s1 = __dp4a(static_cast<int>(__funnelshift_rc(w[i + 1], w[i + 2], sh)), static_cast<int>(qx[m][i + 1]), s1);
+    }
+    isum[m] = s0 + s1;  // |isum| <= 32 * 128 * 128 = 2^19: exact
+  }
+  return d;
+}
+
 // Reduce V per-lane values over the 32 lanes with a reduce-scatter butterfly:
 // afterwards lane l holds the total of value index vidx(l) (V in {1, 2, 4}).
 template <int V>
@@ -168,8 +208,9 @@ __device__ __forceinline__ bool scatter_writer(int lane) {
   return lane == 0;
 }
 
-// MP activation rows per pass (1 or 2); RG weight rows per warp step.
-template <int MP, int RG>
+// MODE: activation kind; MP activation rows per pass (1 or 2); RG weight rows
+// per warp step.
+template <int MODE, int MP, int RG>
 __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
@@ -202,7 +243,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    uint64_t policy = 0;
+    uint64_t policy = 0, policy_x = 0;
+    if constexpr (MODE != kModeF32) policy_x = l2_evict_last_policy();
     auto issue = [&](int c) {
       const int s = c % S;
       const int64_t r0 = r_begin + static_cast<int64_t>(c) * p.rows_chunk;
@@ -222,7 +264,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
     };
     // Sum the window partials of chunk c (all consumers have released it).
     auto finish = [&](int c) {
-      if (p.cg == 1) return;
+      if (p.cg == 1 || MODE == kModeQ8Dots) return;
       const int s = c % S;
       const int64_t r0 = r_begin + static_cast<int64_t>(c) * p.rows_chunk;
       const int rows = static_cast<int>(min(static_cast<int64_t>(p.rows_chunk), r_end - r0));
@@ -237,10 +279,14 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
     };
     // The activation panel: one 2-D TMA load with the 128-byte swizzle, issued
     // as soon as the preceding grid has finished (X may be its output).
+    // (int8 activation codes: one plain bulk copy of the M x K bytes.)
     auto issue_x = [&]() {
       if (p.xs_off) {
-        mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(p.xs_rows) * 128u);
-        tma_load_2d(smem + p.xs_off, &p.xmap, 0, 0, xbar);
+        mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(p.xs_bytes));
+        if constexpr (MODE == kModeF32)
+          tma_load_2d(smem + p.xs_off, &p.xmap, 0, 0, xbar);
+        else
+          bulk_g2s(smem + p.xs_off, p.QX, static_cast<uint32_t>(p.xs_bytes), xbar, policy_x);
       }
     };
     const int prologue = min(S, nchunks);
@@ -296,23 +342,49 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
     if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
     return;
   }
+  // Per-lane activations of its block column: fp32 values, or int8 codes
+  // (eight words) and the block's activation scale.
   float2 x2[MP][16];
+  uint32_t qx[MP][8];
+  float dxr[MP];
   auto load_x = [&](int m0, int cw) {
     const int c = cw * 32 + lane;
 #pragma unroll
     for (int m = 0; m < MP; ++m) {
-      if (c < p.KB && m0 + m < p.M) {
+      const bool valid = c < p.KB && m0 + m < p.M;
+      if constexpr (MODE == kModeF32) {
+        if (valid) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int row = (m0 + m) * p.KB + c;
-          const float4 v = xs ? lds_f4(xs_sa + 16u * (row * 8 + (j ^ (row & 7))))
-                              : __ldg(reinterpret_cast<const float4 *>(p.X + static_cast<int64_t>(m0 + m) * p.K) + 8 * c + j);
-          x2[m][2 * j] = make_float2(v.x, v.y);
-          x2[m][2 * j + 1] = make_float2(v.z, v.w);
+          for (int j = 0; j < 8; ++j) {
+            const int row = (m0 + m) * p.KB + c;
+            const float4 v = xs ? lds_f4(xs_sa + 16u * (row * 8 + (j ^ (row & 7))))
+                                : __ldg(reinterpret_cast<const float4 *>(p.X + static_cast<int64_t>(m0 + m) * p.K) + 8 * c + j);
+            x2[m][2 * j] = make_float2(v.x, v.y);
+            x2[m][2 * j + 1] = make_float2(v.z, v.w);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x2[m][j] = make_float2(0.f, 0.f);
         }
       } else {
+        if (valid) {
+          const int64_t off = static_cast<int64_t>(m0 + m) * p.K + 32 * c;
+          uint4 lo, hi;
+          if (xs) {
+            lo = lds_u4(xs_sa + static_cast<uint32_t>(off));
+            hi = lds_u4(xs_sa + static_cast<uint32_t>(off) + 16u);
+          } else {
+            lo = __ldg(reinterpret_cast<const uint4 *>(p.QX + off));
+            hi = __ldg(reinterpret_cast<const uint4 *>(p.QX + off) + 1);
+          }
+          qx[m][0] = lo.x; qx[m][1] = lo.y; qx[m][2] = lo.z; qx[m][3] = lo.w;
+          qx[m][4] = hi.x; qx[m][5] = hi.y; qx[m][6] = hi.z; qx[m][7] = hi.w;
+          dxr[m] = (MODE == kModeQ8) ? __ldg(p.DX + static_cast<int64_t>(m0 + m) * p.KB + c) : 0.f;
+        } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) x2[m][j] = make_float2(0.f, 0.f);
+          for (int j = 0; j < 8; ++j) qx[m][j] = 0u;
+          dxr[m] = 0.f;
+        }
       }
     }
   };
@@ -344,11 +416,28 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
           for (int g = 0; g < RG; ++g) {
             const bool ok = act && rl + g < rows;
             const int row = min(rl + g, rows - 1);
+            const uint32_t sa = base + static_cast<uint32_t>(row * p.row_bytes) + col_off;
             float o[MP];
-            q8_block_dot<MP>(base + static_cast<uint32_t>(row * p.row_bytes) + col_off, x2, o);
+            if constexpr (MODE == kModeF32) {
+              q8_block_dot<MP>(sa, x2, o);
+            } else {
+              int is[MP];
+              const float d = q8q8_block_isum<MP>(sa, qx, is);
+#pragma unroll
+              for (int m = 0; m < MP; ++m) {
+                if constexpr (MODE == kModeQ8Dots) {
+                  if (ok && m0 + m < p.M)
+                    p.isum[((static_cast<int64_t>(m0 + m) * p.N) + r0 + rl + g) * p.KB + col] = is[m];
+                  o[m] = 0.f;
+                } else {
+                  o[m] = (d * dxr[m]) * static_cast<float>(is[m]);
+                }
+              }
+            }
 #pragma unroll
             for (int m = 0; m < MP; ++m) part[g * MP + m] = ok ? o[m] : 0.f;
           }
+          if constexpr (MODE == kModeQ8Dots) continue;
           const float tot = warp_reduce_scatter<RG * MP>(part, lane);
           if (scatter_writer<RG * MP>(lane)) {
             const int v = scatter_index<RG * MP>(lane);
@@ -370,7 +459,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
 
 int align_up(int64_t v, int a) { return static_cast<int>((v + a - 1) / a * a); }
 
-template <int MP, int RG>
+template <int MODE, int MP, int RG>
 cudaError_t launch(const cudaLaunchConfig_t &cfg, const Params &p) {
   static bool configured[64] = {};
   int dev = 0;
@@ -378,21 +467,27 @@ cudaError_t launch(const cudaLaunchConfig_t &cfg, const Params &p) {
   if (dev >= 0 && dev < 64 && !configured[dev]) {
     int optin = 0;
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    cudaError_t e = cudaFuncSetAttribute(q8_gemv_kernel<MP, RG>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    cudaError_t e = cudaFuncSetAttribute(q8_gemv_kernel<MODE, MP, RG>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  return cudaLaunchKernelEx(&cfg, q8_gemv_kernel<MP, RG>, p);
+  return cudaLaunchKernelEx(&cfg, q8_gemv_kernel<MODE, MP, RG>, p);
 }
 
 }  // namespace
 
-qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
-                          float *Y, cudaStream_t stream, uint32_t flags) {
+namespace {
+
+template <int MODE>
+qmm_status launch_stream(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, const int8_t *QX,
+                         const float *DX, float *Y, int32_t *isum, cudaStream_t stream, uint32_t flags) {
   Params p{};
   p.W = static_cast<const uint8_t *>(W);
   p.X = X;
+  p.QX = QX;
+  p.DX = DX;
   p.Y = Y;
+  p.isum = isum;
   p.N = N;
   p.M = M;
   p.K = K;
@@ -430,12 +525,13 @@ qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
   S = static_cast<int>(std::min<int64_t>({S, kMaxStages, nchunks_max}));
   p.stages = S;
   const int red_bytes = p.cg > 1 ? S * M * p.cg * p.rows_chunk * 4 : 0;
-  const int64_t xs_bytes = static_cast<int64_t>(M) * K * 4;
+  const int64_t xs_bytes = static_cast<int64_t>(M) * K * (MODE == kModeF32 ? 4 : 1);
   const bool panel = xs_bytes <= kPanelBytes;
   p.xs_off = panel ? align_up(kBarBytes + red_bytes, 1024) : 0;  // 128-byte swizzle needs 1024-byte alignment
   p.xs_rows = panel ? static_cast<int>(xs_bytes / 128) : 0;
+  p.xs_bytes = panel ? static_cast<int>(xs_bytes) : 0;
   p.stage_off = panel ? align_up(p.xs_off + xs_bytes, 128) : kBarBytes + align_up(red_bytes, 128);
-  if (panel) {
+  if (panel && MODE == kModeF32) {
     const uint64_t dims[2] = {32, static_cast<uint64_t>(p.xs_rows)};
     const uint64_t strides[1] = {128};
     const uint32_t box[2] = {32, static_cast<uint32_t>(p.xs_rows)};
@@ -459,11 +555,28 @@ qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (M > 1) e = launch<2, 1>(cfg, p);
-  else if (rg == 4) e = launch<1, 4>(cfg, p);
-  else if (rg == 2) e = launch<1, 2>(cfg, p);
-  else e = launch<1, 1>(cfg, p);
-  return cuda_check(e, "q8_gemv launch");
+  if (M > 1) e = launch<MODE, 2, 1>(cfg, p);
+  else if (rg == 4) e = launch<MODE, 1, 4>(cfg, p);
+  else if (rg == 2) e = launch<MODE, 1, 2>(cfg, p);
+  else e = launch<MODE, 1, 1>(cfg, p);
+  return cuda_check(e, MODE == kModeF32 ? "q8_gemv launch" : "q8q8_gemv launch");
+}
+
+}  // namespace
+
+qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
+                          cudaStream_t stream, uint32_t flags) {
+  return launch_stream<kModeF32>(dev, M, N, K, W, X, nullptr, nullptr, Y, nullptr, stream, flags);
+}
+
+qmm_status launch_q8q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,
+                            const float *DX, float *Y, cudaStream_t stream, uint32_t flags) {
+  return launch_stream<kModeQ8>(dev, M, N, K, W, nullptr, QX, DX, Y, nullptr, stream, flags);
+}
+
+qmm_status launch_q8q8_block_dots(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,
+                                  int32_t *isum, cudaStream_t stream) {
+  return launch_stream<kModeQ8Dots>(dev, M, N, K, W, nullptr, QX, nullptr, nullptr, isum, stream, kLaunchPdl);
 }
 
 cudaError_t q8_gemv_status(uint32_t *bits) {

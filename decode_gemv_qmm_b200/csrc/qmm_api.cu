@@ -119,6 +119,46 @@ static qmm_status q8_gemv_impl(int64_t M, int64_t N, int64_t K, int block, const
   return launch_q8_gemv(dev, static_cast<int>(M), N, static_cast<int>(K), W, X, Y, s, flags);
 }
 
+static qmm_status quantize_impl(int64_t M, int64_t K, int block, const float *X, int8_t *QX, float *DX,
+                                qmm_stream_t stream) {
+  const char *fn = "qmm_quantize_act_q8";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, 0, K, block, -1));
+  if (M == 0 || K == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "X", X, true, 16));
+  QMM_TRY(check_ptr(fn, "QX", QX, true, 16));
+  QMM_TRY(check_ptr(fn, "DX", DX, true, 4));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  return launch_quantize_act_q8(dev, M, static_cast<int>(K), X, QX, DX, reinterpret_cast<cudaStream_t>(stream),
+                                kLaunchPdl);
+}
+
+static qmm_status q8q8_impl(int64_t M, int64_t N, int64_t K, int block, const void *W, const int8_t *QX,
+                            const float *DX, float *Y, int32_t *isum, qmm_stream_t stream, uint32_t user_flags) {
+  const char *fn = isum ? "qmm_q8q8_block_dots" : "qmm_q8q8_gemv";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, N, K, block, QMM_MAX_DECODE_M));
+  if (user_flags & ~uint32_t(QMM_FLAG_EARLY_WEIGHTS))
+    return set_error(QMM_ERR_SHAPE, "%s: unknown flags 0x%x", fn, user_flags);
+  if (M == 0 || N == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "W", W, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "QX", QX, K > 0, 16));
+  if (isum) {
+    QMM_TRY(check_ptr(fn, "isum", isum, K > 0, 4));
+  } else {
+    QMM_TRY(check_ptr(fn, "DX", DX, K > 0, 4));
+    QMM_TRY(check_ptr(fn, "Y", Y, true, 4));
+  }
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return isum ? QMM_OK : zero_fill(Y, M * N, s);
+  if (isum) return launch_q8q8_block_dots(dev, static_cast<int>(M), N, static_cast<int>(K), W, QX, isum, s);
+  uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
+  return launch_q8q8_gemv(dev, static_cast<int>(M), N, static_cast<int>(K), W, QX, DX, Y, s, flags);
+}
+
 }  // namespace qmm
 
 using namespace qmm;
@@ -133,6 +173,26 @@ QMM_API qmm_status qmm_q8_gemv(int64_t M, int64_t N, int64_t K, int block, const
 QMM_API qmm_status qmm_q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
                                   float *Y, uint32_t flags, qmm_stream_t stream) {
   return q8_gemv_impl(M, N, K, block, W, X, Y, stream, flags);
+}
+
+QMM_API qmm_status qmm_quantize_act_q8(int64_t M, int64_t K, int block, const float *X, int8_t *QX, float *DX,
+                                       qmm_stream_t stream) {
+  return quantize_impl(M, K, block, X, QX, DX, stream);
+}
+
+QMM_API qmm_status qmm_q8q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W, const int8_t *QX,
+                                 const float *DX, float *Y, qmm_stream_t stream) {
+  return q8q8_impl(M, N, K, block, W, QX, DX, Y, nullptr, stream, 0u);
+}
+
+QMM_API qmm_status qmm_q8q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, const void *W, const int8_t *QX,
+                                    const float *DX, float *Y, uint32_t flags, qmm_stream_t stream) {
+  return q8q8_impl(M, N, K, block, W, QX, DX, Y, nullptr, stream, flags);
+}
+
+QMM_API qmm_status qmm_q8q8_block_dots(int64_t M, int64_t N, int64_t K, int block, const void *W, const int8_t *QX,
+                                       int32_t *isum, qmm_stream_t stream) {
+  return q8q8_impl(M, N, K, block, W, QX, nullptr, nullptr, isum, stream, 0u);
 }
 
 QMM_API const char *qmm_last_error_string(void) { return t_last_error.c_str(); }

@@ -32,6 +32,13 @@ qmm_status cuda_check(cudaError_t e, const char *what);
 qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
                           float *Y, cudaStream_t stream, uint32_t flags);
 
+qmm_status launch_q8q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,
+                            const float *DX, float *Y, cudaStream_t stream, uint32_t flags);
+qmm_status launch_q8q8_block_dots(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,
+                                  int32_t *isum, cudaStream_t stream);
+qmm_status launch_quantize_act_q8(const DevInfo &dev, int64_t M, int K, const float *X, int8_t *QX, float *DX,
+                                  cudaStream_t stream, uint32_t flags);
+
 // Device status word of each kernel file: read and clear (synchronous).
 cudaError_t q8_gemv_status(uint32_t *bits);
 

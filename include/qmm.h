@@ -165,6 +165,11 @@ QMM_API qmm_status qmm_quantize_act_q8(int64_t M, int64_t K, int block, const fl
 QMM_API qmm_status qmm_q8q8_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W,
                          const int8_t *QX, const float *DX, float *Y, qmm_stream_t stream);
 
+/* qmm_q8q8_gemv with options (0 or QMM_FLAG_EARLY_WEIGHTS). */
+QMM_API qmm_status qmm_q8q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                    const int8_t *QX, const float *DX, float *Y, uint32_t flags,
+                                    qmm_stream_t stream);
+
 /*
  * qmm_q4_swiglu_gateup -- fused gate/up projection with SwiGLU on Q4_0 weights.
  *
