@@ -40,6 +40,7 @@ _SIGS = {
     "qmm_q8q8_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_q8q8_gemv_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
     "qmm_q4_swiglu_gateup": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
+    "qmm_q4_swiglu_gateup_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
     "qmm_quant_matmul_prefill": [_int, _i64, _i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q8q8_block_dots": [_i64, _i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q4_gateup_unfused": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p],
@@ -149,11 +150,17 @@ def qmm_q8q8_block_dots(W: torch.Tensor, QX: torch.Tensor, N: int, isum: torch.T
 
 
 def qmm_q4_swiglu_gateup(Wg: torch.Tensor, Wu: torch.Tensor, X: torch.Tensor, N: int,
-                         Y: torch.Tensor | None = None, *, block: int = BLOCK, stream=None) -> torch.Tensor:
+                         Y: torch.Tensor | None = None, *, block: int = BLOCK, flags: int = 0,
+                         stream=None) -> torch.Tensor:
+    """Y[M, N] = silu(X . Wg^T) * (X . Wu^T) for Q4_0 blocks Wg, Wu in one launch."""
     M, K = X.shape
     Y = _out(Y, (M, N), X.device)
-    _check(lib.qmm_q4_swiglu_gateup(M, N, K, block, _ptr(Wg), _ptr(Wu), _ptr(X), _ptr(Y), _stream(stream)),
-           "qmm_q4_swiglu_gateup")
+    if flags:
+        st = lib.qmm_q4_swiglu_gateup_ex(M, N, K, block, _ptr(Wg), _ptr(Wu), _ptr(X), _ptr(Y), flags,
+                                         _stream(stream))
+    else:
+        st = lib.qmm_q4_swiglu_gateup(M, N, K, block, _ptr(Wg), _ptr(Wu), _ptr(X), _ptr(Y), _stream(stream))
+    _check(st, "qmm_q4_swiglu_gateup")
     return Y
 
 

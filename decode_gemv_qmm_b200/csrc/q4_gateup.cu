@@ -1,0 +1,471 @@
+// q4_gateup.cu -- fused gate/up projection with SwiGLU on Q4_0 weights (M <= 8).
+//
+// Operation ("LSE v0.4.16", section "Combined M8 Q4 gate/up execution"): one
+// launch reads one shared activation panel X and accumulates the gate and up
+// projections in independent fp32 accumulators; only
+//     Y[m][n] = silu(g) * u,  g = X[m] . Wg[n],  u = X[m] . Wu[n],  silu(g) = g / (1 + e^-g)
+// is written -- no gate (or up) temporary ever reaches memory.
+//
+// Why tensor cores: at M = 8 every weight meets 8 activations, so on fp32
+// FMAs the kernel is ALU-bound (~40 us for the 8 x 5120 x 17408 shape against
+// ~15 us of HBM time). It is a genuine small-M matrix product, so it runs on
+// mma.sync m16n8k16 (fp16 inputs, fp32 accumulation) with
+//  * A = 16 weight rows x 16 k: Q4 nibbles q - 8 in [-8, 7] are exact in fp16
+//    (nibble -> half with one byte-permute, one mask/or and one half add);
+//  * B = 16 k x 8 tokens: each activation is split into two fp16 parts,
+//    x * s = hi + lo (hi = fp16(x s), lo = fp16(x s - hi)), with s a power of
+//    two per 32-block chosen so the block maximum lands in [2^14, 2^15): the
+//    pair carries ~22 significant bits, and the products are exact in fp32;
+//  * each 32-block gives C = A0 B0hi + A1 B1hi + A0 B0lo + A1 B1lo (four
+//    mma), then acc += (d * 2^-s) * C in fp32 -- the per-block scale applied
+//    in fp32 exactly as the method defines it.
+// Within a block the order of k is permuted (the same permutation on A and B
+// leaves the dot product unchanged) so that lane t of a quad takes qs bytes
+// 4t..4t+3 (one 32-bit word) and activations 4t..4t+3 / 16+4t..16+4t+3 (two
+// 16-byte loads).
+//
+// Data movement: a producer warp streams 8-block (256 k) stages with 2-D TMA
+// loads -- one 16-row x 144-byte box per weight tile and matrix, one
+// 8-token x 32-float box (128-byte swizzle) per block of X. Consumer warp w
+// owns block w of every stage for all of the CTA's row tiles, so its B
+// fragments are built once and reused 2 x tiles times. At the end the 8
+// warps' partial sums are added in warp order through shared memory and the
+// SwiGLU epilogue writes Y. Rows of W must be 16-byte multiples for the
+// tensor maps (K % 256 == 0); other K use the same code reading global memory
+// directly.
+//
+// qmm_q4_gateup_unfused runs the same kernel with one matrix per launch
+// (writing G, then U) and a third launch applying silu(G) * U with the same
+// device function, so the fused output equals the unfused one bit for bit.
+#include <algorithm>
+
+#include "qmm_common.cuh"
+#include "qmm_internal.h"
+#include "qmm_tmap.h"
+
+namespace qmm {
+namespace {
+
+static __device__ uint32_t g_q4_status;
+
+constexpr int kWarps = 8;            // consumer warps; warp w owns block w of each stage
+constexpr int kBlocksPerStage = 8;   // 8 Q4_0 blocks = 256 k = 144 bytes per row
+constexpr int kTilesMax = 8;         // 16-row tiles per CTA
+constexpr int kStages = 4;
+constexpr int kRowStageBytes = kBlocksPerStage * 18;             // 144
+constexpr int kTileBytes = 16 * kRowStageBytes;                  // 2304
+constexpr int kXStageBytes = kBlocksPerStage * 8 * 128;          // 8 blocks x 8 tokens x 32 floats
+constexpr int kStageBytes = kXStageBytes + 2 * kTilesMax * kTileBytes;  // 45056 (multiple of 1024)
+constexpr int kBarBytes = 1024;
+
+enum : int { kOutFused = 0, kOutProj = 1 };
+
+struct alignas(64) Params {
+  CUtensorMap tm_x;      // X: dims {K, M} fp32, box {32, 8}, 128-byte swizzle
+  CUtensorMap tm_w[2];   // Wg, Wu: dims {9 * KB (uint16), N}, box {72, 16}
+  const uint8_t *W[2];   // Wg, Wu (direct path)
+  const float *X;
+  float *Y;              // fused output, or the projection output
+  int M, K, KB;
+  int64_t N;
+  int tiles;             // 16-row tiles in total
+  int grid;
+  int nmat;              // 2 (fused) or 1 (projection)
+  int prefetch_before_wait;
+};
+
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four Q4 codes (bytes b0..b3 of v) -> exact fp16 pairs:
+//   lo01 = (lownib(b0) - 8, lownib(b1) - 8), lo23 = (lownib(b2) - 8, lownib(b3) - 8)
+//   hi01 = (hinib(b0) - 8,  hinib(b1) - 8),  hi23 = (hinib(b2) - 8,  hinib(b3) - 8)
+struct Nib4 {
+  uint32_t lo01, lo23, hi01, hi23;
+};
+__device__ __forceinline__ Nib4 q4_word_to_half2(uint32_t v) {
+  const uint32_t p01 = __byte_perm(v, 0u, 0x4140u);  // [b0, 0, b1, 0]
+  const uint32_t p23 = __byte_perm(v, 0u, 0x4342u);  // [b2, 0, b3, 0]
+  const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
+  const __half2 k16th = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
+  const __half2 km72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));   // -72
+  Nib4 r;
+  uint32_t t;
+  t = (p01 & 0x000F000Fu) | 0x64006400u;  // 1024 + n
+  __half2 h = __hsub2(*reinterpret_cast<__half2 *>(&t), k1032);
+  r.lo01 = *reinterpret_cast<uint32_t *>(&h);
+  t = (p23 & 0x000F000Fu) | 0x64006400u;
+  h = __hsub2(*reinterpret_cast<__half2 *>(&t), k1032);
+  r.lo23 = *reinterpret_cast<uint32_t *>(&h);
+  t = (p01 & 0x00F000F0u) | 0x64006400u;  // 1024 + 16 n
+  h = __hfma2(*reinterpret_cast<__half2 *>(&t), k16th, km72);  // 64 + n - 72
+  r.hi01 = *reinterpret_cast<uint32_t *>(&h);
+  t = (p23 & 0x00F000F0u) | 0x64006400u;
+  h = __hfma2(*reinterpret_cast<__half2 *>(&t), k16th, km72);
+  r.hi23 = *reinterpret_cast<uint32_t *>(&h);
+  return r;
+}
+
+// B fragments of one 32-block for this lane (token g = lane / 4, quad t = lane % 4):
+// activations 4t..4t+3 (k-step 0) and 16+4t..16+4t+3 (k-step 1), scaled by the
+// block's power of two and split into fp16 hi + lo parts.
+struct BFrag {
+  uint32_t hi0, hi1, hi2, hi3;  // k-step 0: (b0, b1); k-step 1: (b0, b1)
+  uint32_t lo0, lo1, lo2, lo3;
+  float inv_scale;
+};
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ BFrag make_bfrag(float4 x0, float4 x1) {
+  // block maximum over all 8 tokens x 32 activations (warp-wide)
+  float mx = fmaxf(fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x0.z), fabsf(x0.w))),
+                   fmaxf(fmaxf(fabsf(x1.x), fabsf(x1.y)), fmaxf(fabsf(x1.z), fabsf(x1.w))));
+  mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+  // s = 2^(14 - e) where 2^e <= mx < 2^(e+1); clamped to the normal range
+  const int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 127;
+  int sexp = 14 - e;
+  sexp = max(-100, min(100, sexp));
+  const float s = __uint_as_float(static_cast<uint32_t>(sexp + 127) << 23);
+  BFrag f;
+  f.inv_scale = __uint_as_float(static_cast<uint32_t>(127 - sexp) << 23);
+  const float v[8] = {x0.x * s, x0.y * s, x0.z * s, x0.w * s, x1.x * s, x1.y * s, x1.z * s, x1.w * s};
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    hi[i] = pack_half2(v[2 * i], v[2 * i + 1]);
+    const float2 hf = __half22float2(*reinterpret_cast<__half2 *>(&hi[i]));
+    lo[i] = pack_half2(v[2 * i] - hf.x, v[2 * i + 1] - hf.y);
+  }
+  f.hi0 = hi[0]; f.hi1 = hi[1]; f.hi2 = hi[2]; f.hi3 = hi[3];
+  f.lo0 = lo[0]; f.lo1 = lo[1]; f.lo2 = lo[2]; f.lo3 = lo[3];
+  return f;
+}
+
+// One 16-row x 32-k block tile: c = W_tile . (hi + lo), then acc += (d * 2^-s) c.
+__device__ __forceinline__ void tile_block(float (&acc)[4], uint32_t vg, uint32_t vh, float dg, float dh,
+                                           const BFrag &b) {
+  const Nib4 ng = q4_word_to_half2(vg), nh = q4_word_to_half2(vh);
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+  mma_16816(c, ng.lo01, nh.lo01, ng.lo23, nh.lo23, b.hi0, b.hi1);  // k-step 0 (low nibbles)
+  mma_16816(c, ng.hi01, nh.hi01, ng.hi23, nh.hi23, b.hi2, b.hi3);  // k-step 1 (high nibbles)
+  mma_16816(c, ng.lo01, nh.lo01, ng.lo23, nh.lo23, b.lo0, b.lo1);
+  mma_16816(c, ng.hi01, nh.hi01, ng.hi23, nh.hi23, b.lo2, b.lo3);
+  const float sg = __fmul_rn(dg, b.inv_scale), sh = __fmul_rn(dh, b.inv_scale);
+  acc[0] = __fmaf_rn(sg, c[0], acc[0]);
+  acc[1] = __fmaf_rn(sg, c[1], acc[1]);
+  acc[2] = __fmaf_rn(sh, c[2], acc[2]);
+  acc[3] = __fmaf_rn(sh, c[3], acc[3]);
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
+// DIRECT = false: TMA-fed shared-memory stages; true: reads global memory.
+template <bool DIRECT>
+__global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *empty = full + kStages;
+  uint8_t *stages = smem + kBarBytes;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * p.tiles / p.grid);
+  const int tile1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * p.tiles / p.grid);
+  const int ntiles = tile1 - tile0;
+  const int nstages = (p.KB + kBlocksPerStage - 1) / kBlocksPerStage;
+
+  pdl_launch_dependents();
+  if (!DIRECT) {
+    if (tid == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(&full[s], 1);
+        mbar_init(&empty[s], kWarps);
+      }
+      fence_mbar_init();
+    }
+    __syncthreads();
+  }
+
+  if (warp == kWarps) {
+    // -------------------------------------------------------------- producer
+    if (DIRECT) return;
+    const uint32_t wbytes = static_cast<uint32_t>(p.nmat * ntiles * kTileBytes);
+    auto issue_w = [&](int j) {  // weights of stage j (arrive + expect all bytes of the stage)
+      const int s = j % kStages;
+      uint8_t *st = stages + s * kStageBytes;
+      mbar_arrive_expect_tx(&full[s], wbytes + kXStageBytes);
+      for (int mat = 0; mat < p.nmat; ++mat)
+        for (int t = 0; t < ntiles; ++t)
+          tma_load_2d(st + kXStageBytes + (mat * kTilesMax + t) * kTileBytes, &p.tm_w[mat], 72 * j,
+                      16 * (tile0 + t), &full[s]);
+    };
+    auto issue_x = [&](int j) {
+      uint8_t *st = stages + (j % kStages) * kStageBytes;
+      for (int b = 0; b < kBlocksPerStage; ++b)
+        tma_load_2d(st + b * 1024, &p.tm_x, 32 * (j * kBlocksPerStage + b), 0, &full[j % kStages]);
+    };
+    const int prologue = min(kStages, nstages);
+    if (lane == 0) {
+      if (p.prefetch_before_wait) {
+        for (int j = 0; j < prologue; ++j) issue_w(j);
+        pdl_wait();
+        for (int j = 0; j < prologue; ++j) issue_x(j);
+      } else {
+        pdl_wait();
+        for (int j = 0; j < prologue; ++j) {
+          issue_w(j);
+          issue_x(j);
+        }
+      }
+      bool ok = true;
+      int issued = prologue;
+      for (int j = 0; j < nstages && issued < nstages; ++j) {
+        ok = mbar_wait(&empty[j % kStages], static_cast<uint32_t>(j / kStages) & 1u);
+        if (!ok) break;
+        issue_w(issued);
+        issue_x(issued);
+        ++issued;
+      }
+      if (!ok) {  // error path: record, then drain the copies still in flight
+        atomicOr(&g_q4_status, kDevTimeoutFull);
+        for (int j = max(0, issued - kStages); j < issued; ++j)
+          if (!mbar_wait(&full[j % kStages], static_cast<uint32_t>(j / kStages) & 1u))
+            atomicOr(&g_q4_status, kDevTimeoutDrain);
+      }
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- consumers
+  pdl_wait();
+  const int g = lane >> 2, t = lane & 3;
+  float acc[kTilesMax][2][4];
+#pragma unroll
+  for (int i = 0; i < kTilesMax; ++i)
+#pragma unroll
+    for (int mat = 0; mat < 2; ++mat)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[i][mat][k] = 0.f;
+
+  const int64_t row_bytes = 18ll * p.KB;
+  for (int j = 0; j < nstages; ++j) {
+    const int s = j % kStages;
+    if (!DIRECT && !mbar_wait(&full[s], static_cast<uint32_t>(j / kStages) & 1u)) {
+      if (lane == 0) atomicOr(&g_q4_status, kDevTimeoutFull);
+      return;  // the producer gives up on this warp's missing arrival and drains
+    }
+    const int kb = j * kBlocksPerStage + warp;  // this warp's block
+    if (kb < p.KB) {
+      // activations of block kb for token g
+      float4 x0, x1;
+      if (!DIRECT) {
+        const uint32_t xa = smem_u32(stages + s * kStageBytes + warp * 1024) + g * 128;
+        x0 = lds_f4(xa + 16u * (t ^ g));
+        x1 = lds_f4(xa + 16u * ((4 + t) ^ g));
+      } else if (g < p.M) {
+        const float4 *xp = reinterpret_cast<const float4 *>(p.X + static_cast<int64_t>(g) * p.K + 32 * kb);
+        x0 = __ldg(xp + t);
+        x1 = __ldg(xp + 4 + t);
+      } else {
+        x0 = x1 = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      const BFrag bf = make_bfrag(x0, x1);
+#pragma unroll
+      for (int mat = 0; mat < 2; ++mat) {
+        if (mat >= p.nmat) break;
+#pragma unroll
+        for (int i = 0; i < kTilesMax; ++i) {
+          if (i >= ntiles) break;
+          uint32_t vg, vh;
+          float dg, dh;
+          if (!DIRECT) {
+            // row r of the tile at r * 144 bytes; block `warp` at 18 * warp
+            const uint32_t tb = smem_u32(stages + s * kStageBytes + kXStageBytes + (mat * kTilesMax + i) * kTileBytes);
+            const uint32_t ag = tb + g * kRowStageBytes + 18 * warp, ah = ag + 8 * kRowStageBytes;
+            if (warp & 1) {  // block starts 2 bytes past a 4-byte boundary: qs word aligned
+              vg = lds_u32(ag + 2 + 4 * t);
+              vh = lds_u32(ah + 2 + 4 * t);
+            } else {
+              vg = __funnelshift_r(lds_u32(ag + 4 * t), lds_u32(ag + 4 * t + 4), 16);
+              vh = __funnelshift_r(lds_u32(ah + 4 * t), lds_u32(ah + 4 * t + 4), 16);
+            }
+            dg = half_bits_to_float(lds_u16(ag));
+            dh = half_bits_to_float(lds_u16(ah));
+          } else {
+            const int64_t rg = 16ll * (tile0 + i) + g, rh = rg + 8;
+            const uint8_t *Wm = p.W[mat];
+            auto word = [&](int64_t r, float &d) -> uint32_t {
+              if (r >= p.N) {
+                d = 0.f;
+                return 0x88888888u;  // nibbles 8 -> value 0
+              }
+              const uint16_t *bp = reinterpret_cast<const uint16_t *>(Wm + r * row_bytes + 18ll * kb);
+              d = half_bits_to_float(__ldg(bp));
+              return static_cast<uint32_t>(__ldg(bp + 1 + 2 * t)) | (static_cast<uint32_t>(__ldg(bp + 2 + 2 * t)) << 16);
+            };
+            vg = word(rg, dg);
+            vh = word(rh, dh);
+          }
+          tile_block(acc[i][mat], vg, vh, dg, dh, bf);
+        }
+      }
+    }
+    if (!DIRECT) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+  }
+
+  // ------------------------------------------ cross-warp sum, SwiGLU epilogue
+  // Every consumer has passed its last stage, so the stage memory is free.
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+  float4 *red = reinterpret_cast<float4 *>(stages);  // [warp][tile][mat][lane]
+#pragma unroll
+  for (int i = 0; i < kTilesMax; ++i) {
+    if (i >= ntiles) break;
+#pragma unroll
+    for (int mat = 0; mat < 2; ++mat) {
+      if (mat >= p.nmat) break;
+      red[((warp * kTilesMax + i) * 2 + mat) * 32 + lane] =
+          make_float4(acc[i][mat][0], acc[i][mat][1], acc[i][mat][2], acc[i][mat][3]);
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
+  const float *redf = reinterpret_cast<const float *>(red);
+  const int rows = ntiles * 16;
+  for (int o = tid; o < 8 * rows; o += kWarps * 32) {
+    const int tok = o / rows, rl = o - tok * rows;
+    const int i = rl >> 4, r = rl & 15;
+    const int src_lane = (r & 7) * 4 + (tok >> 1), idx = (r >> 3) * 2 + (tok & 1);
+    float v[2] = {0.f, 0.f};
+    for (int mat = 0; mat < p.nmat; ++mat) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) sum = __fadd_rn(sum, redf[(((w * kTilesMax + i) * 2 + mat) * 32 + src_lane) * 4 + idx]);
+      v[mat] = sum;
+    }
+    const int64_t n = 16ll * tile0 + rl;
+    if (tok < p.M && n < p.N) p.Y[static_cast<int64_t>(tok) * p.N + n] = (p.nmat == 2) ? silu_mul(v[0], v[1]) : v[0];
+  }
+}
+
+__global__ void silu_mul_kernel(const float *__restrict__ G, const float *__restrict__ U, float *__restrict__ Y,
+                                int64_t count) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    Y[i] = silu_mul(G[i], U[i]);
+}
+
+template <bool DIRECT>
+cudaError_t launch(const cudaLaunchConfig_t &cfg, const Params &p) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(q4_gateup_kernel<DIRECT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kBarBytes + kStages * kStageBytes + 1024);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  return cudaLaunchKernelEx(&cfg, q4_gateup_kernel<DIRECT>, p);
+}
+
+// One gate/up launch over nmat matrices (W[0], W[1]) writing Y.
+qmm_status launch_proj(const DevInfo &dev, int M, int64_t N, int K, const void *const *W, int nmat, const float *X,
+                       float *Y, cudaStream_t stream, uint32_t flags) {
+  Params p{};
+  p.M = M;
+  p.K = K;
+  p.KB = K / 32;
+  p.N = N;
+  p.X = X;
+  p.Y = Y;
+  p.nmat = nmat;
+  p.W[0] = static_cast<const uint8_t *>(W[0]);
+  p.W[1] = static_cast<const uint8_t *>(nmat > 1 ? W[1] : W[0]);
+  p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
+  const int64_t tiles = (N + 15) / 16;
+  if (tiles > (int64_t(1) << 30)) return set_error(QMM_ERR_SHAPE, "q4_gateup: N too large");
+  p.tiles = static_cast<int>(tiles);
+  p.grid = static_cast<int>(std::max<int64_t>(std::min<int64_t>(tiles, dev.sms), (tiles + kTilesMax - 1) / kTilesMax));
+  const bool direct = (p.KB % kBlocksPerStage) != 0;
+  if (!direct) {
+    const uint64_t xd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint64_t xs[1] = {static_cast<uint64_t>(K) * 4};
+    const uint32_t xb[2] = {32, 8};
+    qmm_status st = encode_tiled(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, X, xd, xs, xb, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != QMM_OK) return st;
+    for (int mat = 0; mat < 2; ++mat) {
+      const uint64_t wd[2] = {static_cast<uint64_t>(9) * p.KB, static_cast<uint64_t>(N)};
+      const uint64_t ws[1] = {static_cast<uint64_t>(18) * p.KB};
+      const uint32_t wb[2] = {72, 16};
+      st = encode_tiled(&p.tm_w[mat], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.W[mat], wd, ws, wb,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (st != QMM_OK) return st;
+    }
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3((kWarps + 1) * 32);
+  cfg.dynamicSmemBytes = direct ? static_cast<size_t>(kWarps * kTilesMax * 2 * 32 * 16 + 2048)
+                                : static_cast<size_t>(kBarBytes + kStages * kStageBytes + 1024);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(direct ? launch<true>(cfg, p) : launch<false>(cfg, p), "q4_gateup launch");
+}
+
+}  // namespace
+
+qmm_status launch_q4_gateup(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
+                            const float *X, float *Y, cudaStream_t stream, uint32_t flags) {
+  const void *W[2] = {Wg, Wu};
+  return launch_proj(dev, M, N, K, W, 2, X, Y, stream, flags);
+}
+
+qmm_status launch_q4_gateup_unfused(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
+                                    const float *X, float *G, float *U, float *Y, cudaStream_t stream) {
+  const void *Wgp[1] = {Wg}, *Wup[1] = {Wu};
+  qmm_status st = launch_proj(dev, M, N, K, Wgp, 1, X, G, stream, kLaunchPdl);
+  if (st != QMM_OK) return st;
+  st = launch_proj(dev, M, N, K, Wup, 1, X, U, stream, kLaunchPdl);
+  if (st != QMM_OK) return st;
+  const int64_t count = static_cast<int64_t>(M) * N;
+  const int grid = static_cast<int>(std::min<int64_t>((count + 255) / 256, dev.sms * 8ll));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(std::max(grid, 1));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, silu_mul_kernel, static_cast<const float *>(G),
+                                       static_cast<const float *>(U), Y, count),
+                    "silu_mul launch");
+}
+
+cudaError_t q4_gateup_status(uint32_t *bits) {
+  uint32_t zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(bits, g_q4_status, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_q4_status, &zero, sizeof(uint32_t));
+  return e;
+}
+
+}  // namespace qmm

@@ -159,6 +159,39 @@ static qmm_status q8q8_impl(int64_t M, int64_t N, int64_t K, int block, const vo
   return launch_q8q8_gemv(dev, static_cast<int>(M), N, static_cast<int>(K), W, QX, DX, Y, s, flags);
 }
 
+static qmm_status gateup_impl(int64_t M, int64_t N, int64_t K, int block, const void *Wg, const void *Wu,
+                              const float *X, float *G, float *U, float *Y, qmm_stream_t stream, bool unfused,
+                              uint32_t user_flags) {
+  const char *fn = unfused ? "qmm_q4_gateup_unfused" : "qmm_q4_swiglu_gateup";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, N, K, block, QMM_MAX_DECODE_M));
+  if (user_flags & ~uint32_t(QMM_FLAG_EARLY_WEIGHTS))
+    return set_error(QMM_ERR_SHAPE, "%s: unknown flags 0x%x", fn, user_flags);
+  if (M == 0 || N == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "Wg", Wg, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "Wu", Wu, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "X", X, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "Y", Y, true, 4));
+  if (unfused) {
+    QMM_TRY(check_ptr(fn, "G", G, true, 4));
+    QMM_TRY(check_ptr(fn, "U", U, true, 4));
+  }
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    if (unfused) {
+      QMM_TRY(zero_fill(G, M * N, s));
+      QMM_TRY(zero_fill(U, M * N, s));
+    }
+    return zero_fill(Y, M * N, s);
+  }
+  if (unfused)
+    return launch_q4_gateup_unfused(dev, static_cast<int>(M), N, static_cast<int>(K), Wg, Wu, X, G, U, Y, s);
+  uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
+  return launch_q4_gateup(dev, static_cast<int>(M), N, static_cast<int>(K), Wg, Wu, X, Y, s, flags);
+}
+
 }  // namespace qmm
 
 using namespace qmm;
@@ -195,6 +228,22 @@ QMM_API qmm_status qmm_q8q8_block_dots(int64_t M, int64_t N, int64_t K, int bloc
   return q8q8_impl(M, N, K, block, W, QX, nullptr, nullptr, isum, stream, 0u);
 }
 
+QMM_API qmm_status qmm_q4_swiglu_gateup(int64_t M, int64_t N, int64_t K, int block, const void *Wg, const void *Wu,
+                                        const float *X, float *Y, qmm_stream_t stream) {
+  return gateup_impl(M, N, K, block, Wg, Wu, X, nullptr, nullptr, Y, stream, false, 0u);
+}
+
+QMM_API qmm_status qmm_q4_swiglu_gateup_ex(int64_t M, int64_t N, int64_t K, int block, const void *Wg,
+                                           const void *Wu, const float *X, float *Y, uint32_t flags,
+                                           qmm_stream_t stream) {
+  return gateup_impl(M, N, K, block, Wg, Wu, X, nullptr, nullptr, Y, stream, false, flags);
+}
+
+QMM_API qmm_status qmm_q4_gateup_unfused(int64_t M, int64_t N, int64_t K, int block, const void *Wg, const void *Wu,
+                                         const float *X, float *G, float *U, float *Y, qmm_stream_t stream) {
+  return gateup_impl(M, N, K, block, Wg, Wu, X, G, U, Y, stream, true, 0u);
+}
+
 QMM_API const char *qmm_last_error_string(void) { return t_last_error.c_str(); }
 
 QMM_API const char *qmm_version(void) { return "qmm 0.1.0 sm_100a"; }
@@ -206,6 +255,9 @@ QMM_API qmm_status qmm_device_status(uint32_t *bits) {
   if (e != cudaSuccess) return cuda_check(e, "cudaDeviceSynchronize");
   uint32_t b = 0;
   e = q8_gemv_status(&b);
+  if (e != cudaSuccess) return cuda_check(e, "status read");
+  *bits |= b;
+  e = q4_gateup_status(&b);
   if (e != cudaSuccess) return cuda_check(e, "status read");
   *bits |= b;
   return QMM_OK;

@@ -39,7 +39,13 @@ qmm_status launch_q8q8_block_dots(const DevInfo &dev, int M, int64_t N, int K, c
 qmm_status launch_quantize_act_q8(const DevInfo &dev, int64_t M, int K, const float *X, int8_t *QX, float *DX,
                                   cudaStream_t stream, uint32_t flags);
 
+qmm_status launch_q4_gateup(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
+                            const float *X, float *Y, cudaStream_t stream, uint32_t flags);
+qmm_status launch_q4_gateup_unfused(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
+                                    const float *X, float *G, float *U, float *Y, cudaStream_t stream);
+
 // Device status word of each kernel file: read and clear (synchronous).
 cudaError_t q8_gemv_status(uint32_t *bits);
+cudaError_t q4_gateup_status(uint32_t *bits);
 
 }  // namespace qmm

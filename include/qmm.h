@@ -190,6 +190,11 @@ QMM_API qmm_status qmm_q8q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, 
 QMM_API qmm_status qmm_q4_swiglu_gateup(int64_t M, int64_t N, int64_t K, int block, const void *Wg,
                                 const void *Wu, const float *X, float *Y, qmm_stream_t stream);
 
+/* qmm_q4_swiglu_gateup with options (0 or QMM_FLAG_EARLY_WEIGHTS). */
+QMM_API qmm_status qmm_q4_swiglu_gateup_ex(int64_t M, int64_t N, int64_t K, int block, const void *Wg,
+                                           const void *Wu, const float *X, float *Y, uint32_t flags,
+                                           qmm_stream_t stream);
+
 /*
  * qmm_quant_matmul_prefill -- prefill panel Y = X . W^T on the tensor cores.
  *

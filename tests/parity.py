@@ -33,3 +33,23 @@ def assert_within(got: np.ndarray, ref: np.ndarray, S: np.ndarray, tol: float, w
         raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outputs outside tolerance; worst at {i}: "
                              f"gpu={got[i]!r} oracle={ref[i]!r} err={err[i]:.3e} bound={bound[i]:.3e}")
     return float(np.max(err / np.maximum(S, 1e-300)))
+
+
+def oracle_parallel(fn, N, *args, rows_per_job=256, threads=None):
+    """Run an oracle function over row windows on host threads (the C oracle
+    releases the GIL); returns the per-window results concatenated along N."""
+    import concurrent.futures as cf
+    import os
+    M = args[-1].shape[0]
+    jobs = [(n0, min(N, n0 + rows_per_job)) for n0 in range(0, N, rows_per_job)]
+    with cf.ThreadPoolExecutor(max_workers=threads or os.cpu_count() or 1) as ex:
+        parts = list(ex.map(lambda j: fn(*args[:-1], args[-1], N, window=(0, M, j[0], j[1])), jobs))
+    return parts
+
+
+def swiglu_tolerance(r, tol=TOL_FP32):
+    """Propagated bound for out = silu(g) u: tol (1.1 |u| S_g + |silu(g)| S_u) + 8 ulp(out)."""
+    g, u = r["g"], r["u"]
+    silu = g / (1.0 + np.exp(-g))
+    ulp = np.spacing(np.abs(r["out"]).astype(np.float32)).astype(np.float64)
+    return tol * (1.1 * np.abs(u) * r["Sg"] + np.abs(silu) * r["Su"]) + 8 * ulp
