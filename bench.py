@@ -279,6 +279,84 @@ def component_lm_head(qmm, step: DecodeStep, dev_peak_gbs, reps=20):
             "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4), "bytes": bytes_}
 
 
+def component_gateup(qmm, dev_peak_gbs, m=8, n=17408, k=5120, reps=10):
+    """Fused Q4_0 gate/up SwiGLU (M=8, K=5120, N=17408) vs the unfused path (two
+    projection launches + silu*mul); three rotating weight pairs (> L2)."""
+    import torch
+
+    g = syn.rng(3)
+    pairs = [(torch.from_numpy(syn.q4_0_weights(g, n, k)[0]).cuda(), torch.from_numpy(syn.q4_0_weights(g, n, k)[0]).cuda())
+             for _ in range(3)]
+    x = torch.from_numpy(syn.act_f32(g, m, k)).cuda()
+    Y = torch.empty(m, n, device="cuda")
+    G, U = torch.empty(m, n, device="cuda"), torch.empty(m, n, device="cuda")
+    s = torch.cuda.Stream()
+    out = {}
+
+    def fused(h):
+        for wg, wu in pairs:
+            assert qmm.lib.qmm_q4_swiglu_gateup_ex(m, n, k, 32, wg.data_ptr(), wu.data_ptr(), x.data_ptr(),
+                                                   Y.data_ptr(), qmm.QMM_FLAG_EARLY_WEIGHTS, h) == 0
+
+    def unfused(h):
+        for wg, wu in pairs:
+            assert qmm.lib.qmm_q4_gateup_unfused(m, n, k, 32, wg.data_ptr(), wu.data_ptr(), x.data_ptr(),
+                                                 G.data_ptr(), U.data_ptr(), Y.data_ptr(), h) == 0
+
+    bytes_ = 2 * n * (k // 32) * 18 + m * k * 4 + m * n * 4
+    for name, fn in (("fused", fused), ("unfused", unfused)):
+        fn(s.cuda_stream)
+        torch.cuda.synchronize()
+        gr = capture(fn, s)
+        time_graph(gr, s, 3)
+        us = time_graph(gr, s, reps) / len(pairs) * 1e3
+        out[name] = {"us": round(us, 2), "GB_s": round(bytes_ / us / 1e3, 1),
+                     "frac_hbm": round(bytes_ / us / 1e3 / dev_peak_gbs, 4)}
+        del gr
+    out["bytes"] = bytes_
+    out["flops"] = 2 * 2 * m * n * k
+    out["fused_vs_unfused_time"] = round(out["fused"]["us"] / out["unfused"]["us"] - 1.0, 4)
+    return out
+
+
+def component_prefill(qmm, pk, reps=10):
+    """Prefill panels on the tensor cores: TFLOP/s per shape (rotating weight copies
+    > L2 where the weights are small; activations bf16 N(0,1))."""
+    import torch
+
+    shapes = [("q8_m32_k896_n4864", syn.Q8_0, 32, 4864, 896), ("q8_m32_k4864_n896", syn.Q8_0, 32, 896, 4864),
+              ("q8_m1024_k896_n4864", syn.Q8_0, 1024, 4864, 896), ("q8_m1024_k4864_n896", syn.Q8_0, 1024, 896, 4864),
+              ("q4_m1024_k5120_n17408", syn.Q4_0, 1024, 17408, 5120)]
+    out = {}
+    g = syn.rng(4)
+    for name, wt, m, n, k in shapes:
+        wbytes = n * (k // 32) * (34 if wt == syn.Q8_0 else 18)
+        copies = max(1, int(3 * 126e6 // wbytes) + 1) if wbytes < 200e6 else 1
+        copies = min(copies, 64)
+        W0 = torch.from_numpy(syn.weights(g, wt, n, k)).cuda()
+        Ws = [W0] + [W0.clone() for _ in range(copies - 1)]
+        X = torch.from_numpy(syn.act_bf16_bits(g, m, k).view(np.int16)).cuda()
+        Y = torch.empty(m, n, device="cuda")
+        s = torch.cuda.Stream()
+
+        def fn(h, Ws=Ws, X=X, Y=Y, wt=wt, m=m, n=n, k=k):
+            for w in Ws:
+                assert qmm.lib.qmm_quant_matmul_prefill(wt, m, n, k, 32, w.data_ptr(), X.data_ptr(), Y.data_ptr(), h) == 0
+        fn(s.cuda_stream)
+        torch.cuda.synchronize()
+        gr = capture(fn, s)
+        time_graph(gr, s, 2)
+        us = time_graph(gr, s, reps) / len(Ws) * 1e3
+        flops = 2 * m * n * k
+        bytes_ = wbytes + m * k * 2 + m * n * 4
+        out[name] = {"us": round(us, 2), "TFLOP_s": round(flops / us / 1e6, 1),
+                     "frac_tensor_burst": round(flops / us / 1e6 / pk["bf16_tflops"], 4),
+                     "GB_s": round(bytes_ / us / 1e3, 1), "frac_hbm": round(bytes_ / us / 1e3 / pk["hbm_gbs"], 4),
+                     "weight_copies": len(Ws)}
+        del gr, Ws
+    return out
+
+
 # --------------------------------------------------------------------------- CPU oracle baseline
 
 def oracle_step_sample(step_w, step_x, shapes, frac: float, threads: int):
@@ -481,7 +559,9 @@ def main(argv=None):
     components = None
     if rank == 0 and world == 1 and not args.no_components:
         components = {"lm_head_896x151936": component_lm_head(qmm, step, pk["hbm_gbs"]),
-                      "single_gemv_896x1152": component_single_gemv(qmm, pk["hbm_gbs"])}
+                      "single_gemv_896x1152": component_single_gemv(qmm, pk["hbm_gbs"]),
+                      "q4_gateup_m8_k5120_n17408": component_gateup(qmm, pk["hbm_gbs"]),
+                      "prefill": component_prefill(qmm, pk)}
 
     cpu = None
     if want_cpu:

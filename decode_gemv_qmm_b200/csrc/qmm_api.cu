@@ -192,6 +192,24 @@ static qmm_status gateup_impl(int64_t M, int64_t N, int64_t K, int block, const 
   return launch_q4_gateup(dev, static_cast<int>(M), N, static_cast<int>(K), Wg, Wu, X, Y, s, flags);
 }
 
+static qmm_status prefill_impl(int wtype, int64_t M, int64_t N, int64_t K, int block, const void *W,
+                               const uint16_t *X, float *Y, qmm_stream_t stream) {
+  const char *fn = "qmm_quant_matmul_prefill";
+  t_last_error.clear();
+  if (wtype != QMM_Q8_0 && wtype != QMM_Q4_0) return set_error(QMM_ERR_DTYPE, "%s: unknown weight type %d", fn, wtype);
+  QMM_TRY(check_shape(fn, M, N, K, block, -1));
+  if (M > (int64_t(1) << 24)) return set_error(QMM_ERR_SHAPE, "%s: M=%lld too large", fn, (long long)M);
+  if (M == 0 || N == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "W", W, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "X", X, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "Y", Y, true, 4));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return zero_fill(Y, M * N, s);
+  return launch_prefill(dev, wtype, M, N, static_cast<int>(K), W, X, Y, s, kLaunchPdl);
+}
+
 }  // namespace qmm
 
 using namespace qmm;
@@ -244,6 +262,11 @@ QMM_API qmm_status qmm_q4_gateup_unfused(int64_t M, int64_t N, int64_t K, int bl
   return gateup_impl(M, N, K, block, Wg, Wu, X, G, U, Y, stream, true, 0u);
 }
 
+QMM_API qmm_status qmm_quant_matmul_prefill(int wtype, int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                            const uint16_t *X, float *Y, qmm_stream_t stream) {
+  return prefill_impl(wtype, M, N, K, block, W, X, Y, stream);
+}
+
 QMM_API const char *qmm_last_error_string(void) { return t_last_error.c_str(); }
 
 QMM_API const char *qmm_version(void) { return "qmm 0.1.0 sm_100a"; }
@@ -258,6 +281,9 @@ QMM_API qmm_status qmm_device_status(uint32_t *bits) {
   if (e != cudaSuccess) return cuda_check(e, "status read");
   *bits |= b;
   e = q4_gateup_status(&b);
+  if (e != cudaSuccess) return cuda_check(e, "status read");
+  *bits |= b;
+  e = prefill_status(&b);
   if (e != cudaSuccess) return cuda_check(e, "status read");
   *bits |= b;
   return QMM_OK;

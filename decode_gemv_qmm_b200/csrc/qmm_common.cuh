@@ -3,6 +3,7 @@
 // launch controls and the Q8_0 / Q4_0 block field access.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>

@@ -44,8 +44,12 @@ qmm_status launch_q4_gateup(const DevInfo &dev, int M, int64_t N, int K, const v
 qmm_status launch_q4_gateup_unfused(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
                                     const float *X, float *G, float *U, float *Y, cudaStream_t stream);
 
+qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,
+                          const uint16_t *X, float *Y, cudaStream_t stream, uint32_t flags);
+
 // Device status word of each kernel file: read and clear (synchronous).
 cudaError_t q8_gemv_status(uint32_t *bits);
 cudaError_t q4_gateup_status(uint32_t *bits);
+cudaError_t prefill_status(uint32_t *bits);
 
 }  // namespace qmm

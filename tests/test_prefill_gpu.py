@@ -1,0 +1,76 @@
+"""qmm_quant_matmul_prefill (tcgen05 tensor-core prefill panels) against the CPU oracle.
+
+The weights are decoded to bf16 on the GPU, so outputs must be within
+4e-3 * sum_k |w_k x_k| of the exact (fp64, undecoded) oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as syn
+from parity import TOL_BF16, assert_within, dev, host, oracle_parallel
+
+pytestmark = pytest.mark.gpu
+
+qmm = pytest.importorskip("decode_gemv_qmm_b200")
+
+
+def run(wtype, m, n, k, seed, window_rows=None):
+    g = syn.rng(seed)
+    W = syn.weights(g, wtype, n, k)
+    xb = syn.act_bf16_bits(g, m, k)
+    Y = qmm.qmm_quant_matmul_prefill(wtype, dev(W), dev(xb), n)
+    torch.cuda.synchronize()
+    y = host(Y)
+    return W, xb, y
+
+
+def check_full(wtype, m, n, k, seed):
+    W, xb, y = run(wtype, m, n, k, seed)
+    parts = oracle_parallel(lambda a, b, N, window: oracle.prefill(wtype, a, b, N, window=window), n, W, xb,
+                            rows_per_job=128)
+    ref = np.concatenate([p[0] for p in parts], axis=1)
+    S = np.concatenate([p[1] for p in parts], axis=1)
+    assert_within(y, ref, S, TOL_BF16, f"prefill wtype={wtype} M={m} N={n} K={k}")
+
+
+@pytest.mark.parametrize("wtype", [syn.Q8_0, syn.Q4_0])
+@pytest.mark.parametrize("m,n,k", [(16, 128, 256), (32, 256, 512), (7, 130, 256), (100, 200, 1024), (1, 1, 256),
+                                   (300, 129, 768)])
+def test_prefill_tma_weight_path(wtype, m, n, k):
+    check_full(wtype, m, n, k, seed=m + n + k)
+
+
+@pytest.mark.parametrize("wtype", [syn.Q8_0, syn.Q4_0])
+@pytest.mark.parametrize("m,n,k", [(32, 128, 896), (16, 77, 96), (5, 3, 32), (64, 257, 160)])
+def test_prefill_direct_weight_path(wtype, m, n, k):
+    check_full(wtype, m, n, k, seed=3 * m + n + k)
+
+
+def check_sampled(wtype, m, n, k, seed, n_samples=96):
+    """Full-size launch; compare every token of a spread of sampled weight rows
+    (covering several 128-row tiles, the last tile included)."""
+    W, xb, y = run(wtype, m, n, k, seed)
+    g = np.random.default_rng(seed + 1)
+    rows = np.unique(np.concatenate([g.choice(n, size=n_samples, replace=False), [0, 127, 128, n - 1]]))
+    import concurrent.futures as cf
+    import os
+    with cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+        res = list(ex.map(lambda r: oracle.prefill(wtype, W, xb, n, window=(0, m, int(r), int(r) + 1)), rows))
+    ref = np.concatenate([r[0] for r in res], axis=1)
+    S = np.concatenate([r[1] for r in res], axis=1)
+    assert_within(y[:, rows], ref, S, TOL_BF16, f"prefill wtype={wtype} M={m} N={n} K={k} (sampled rows)")
+
+
+@pytest.mark.parametrize("m", [32, 1024])
+@pytest.mark.parametrize("n,k", [(4864, 896), (896, 4864)])
+def test_prefill_q8_panels_full_size(m, n, k):
+    if m == 32:
+        check_full(syn.Q8_0, m, n, k, seed=m + n)
+    else:
+        check_sampled(syn.Q8_0, m, n, k, seed=m + n)
+
+
+def test_prefill_q4_m1024_k5120_n17408():
+    check_sampled(syn.Q4_0, 1024, 17408, 5120, seed=11, n_samples=64)
