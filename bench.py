@@ -451,6 +451,74 @@ def committed_traffic(kernel_src: str, summary: str):
     return int(m.group(1))
 
 
+# --------------------------------------------------------------------------- single-kernel cases (profiling)
+
+def run_case(spec: str, reps: int, seed: int):
+    """Launch one named kernel `reps` times back to back (eager, stream-ordered)
+    and print the average time of the last reps-1. For profiler captures; the
+    numbers it prints are not benchmark values.
+
+    gemv:N:K            qmm_q8_gemv, M=1
+    q8q8:N:K            qmm_quantize_act_q8 + qmm_q8q8_gemv, M=1
+    gateup:M:N:K        qmm_q4_swiglu_gateup
+    prefill:q8|q4:M:N:K qmm_quant_matmul_prefill
+    decode_step         the 121 GEMVs of one decode step
+    """
+    import torch
+
+    import decode_gemv_qmm_b200 as qmm
+
+    torch.cuda.set_device(0)
+    parts = spec.split(":")
+    g = syn.rng(seed)
+    launches = []
+    if parts[0] == "gemv":
+        n, k = int(parts[1]), int(parts[2])
+        W = torch.from_numpy(syn.q8_0_weights(g, n, k)[0]).cuda()
+        x = torch.from_numpy(syn.act_f32(g, 1, k)).cuda()
+        y = torch.empty(1, n, device="cuda")
+        launches.append(lambda: qmm.qmm_q8_gemv(W, x, n, y))
+    elif parts[0] == "q8q8":
+        n, k = int(parts[1]), int(parts[2])
+        W = torch.from_numpy(syn.q8_0_weights(g, n, k)[0]).cuda()
+        x = torch.from_numpy(syn.act_f32(g, 1, k)).cuda()
+        qx = torch.empty(1, k, dtype=torch.int8, device="cuda")
+        dx = torch.empty(1, k // 32, device="cuda")
+        y = torch.empty(1, n, device="cuda")
+        launches.append(lambda: (qmm.qmm_quantize_act_q8(x, qx, dx), qmm.qmm_q8q8_gemv(W, qx, dx, n, y)))
+    elif parts[0] == "gateup":
+        m, n, k = int(parts[1]), int(parts[2]), int(parts[3])
+        Wg = torch.from_numpy(syn.q4_0_weights(g, n, k)[0]).cuda()
+        Wu = torch.from_numpy(syn.q4_0_weights(g, n, k)[0]).cuda()
+        x = torch.from_numpy(syn.act_f32(g, m, k)).cuda()
+        y = torch.empty(m, n, device="cuda")
+        launches.append(lambda: qmm.qmm_q4_swiglu_gateup(Wg, Wu, x, n, y))
+    elif parts[0] == "prefill":
+        wt = syn.Q8_0 if parts[1] == "q8" else syn.Q4_0
+        m, n, k = int(parts[2]), int(parts[3]), int(parts[4])
+        W = torch.from_numpy(syn.weights(g, wt, n, k)).cuda()
+        X = torch.from_numpy(syn.act_bf16_bits(g, m, k).view(np.int16)).cuda()
+        Y = torch.empty(m, n, device="cuda")
+        launches.append(lambda: qmm.qmm_quant_matmul_prefill(wt, W, X, n, Y))
+    elif parts[0] == "decode_step":
+        step = DecodeStep(seed, torch.device("cuda", 0), keep_host=False)
+        launches.append(lambda: step.launch(qmm, torch.cuda.current_stream().cuda_stream, qmm.QMM_FLAG_EARLY_WEIGHTS))
+    else:
+        raise SystemExit(f"unknown case {spec!r}")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for r in range(reps):
+        if r == 1:
+            e0.record()
+        for f in launches:
+            f()
+    e1.record()
+    torch.cuda.synchronize()
+    if reps > 1:
+        print(json.dumps({"case": spec, "reps": reps, "us_per_rep": round(e0.elapsed_time(e1) * 1e3 / (reps - 1), 2),
+                          "note": "eager launches for profiling; not a benchmark value"}))
+    return 0
+
+
 # --------------------------------------------------------------------------- main
 
 def main(argv=None):
@@ -462,7 +530,11 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None, help="launch one named kernel (see run_case) instead of the benchmark")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args(argv)
+    if args.case:
+        return run_case(args.case, args.reps, args.seed)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
