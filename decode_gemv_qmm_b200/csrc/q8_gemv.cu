@@ -457,6 +457,180 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Resident variant (M = 1, small weight slices): a chain of dependent decode
+// GEMVs is latency-bound, and only the FMAs need the activations. So a CTA
+// loads its whole weight slice (before griddepcontrol.wait when allowed),
+// decodes every block it owns into registers as exact fp32 codes (plus the
+// block scale), and after the activations arrive does only packed FMAs, one
+// multiply by d per block, one reduce-scatter and the store.
+//
+// Warp (window cw, row slot k) owns block column 32*cw + lane of rows
+// r_begin + k + U*... (U rows, stride wpw); windows of a row are added by the
+// CTA in window order. Deterministic.
+
+struct alignas(64) RParams {
+  CUtensorMap xmap;  // X as K/32 rows of 128 bytes, 128-byte swizzle
+  const uint8_t *W;
+  float *Y;
+  int64_t N;
+  int64_t row_bytes;
+  int64_t total_bytes;
+  int K, KB;
+  int grid;
+  int cg;    // 32-column windows
+  int wpw;   // warps per window
+  int xs_off;      // swizzled activation panel (1024-aligned)
+  int red_off;     // window partials (cg > 1)
+  int w_off;       // raw weight slice
+  int max_rows;    // rows per CTA upper bound
+  int prefetch_before_wait;
+};
+
+template <int U>
+__global__ void __launch_bounds__(U == 1 ? 512 : (U == 2 ? 512 : 352), 1)
+q8_gemv_resident_kernel(const __grid_constant__ RParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *wbar = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *xbar = wbar + 1;
+  float *red = reinterpret_cast<float *>(smem + p.red_off);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * p.N / p.grid;
+  const int64_t r_end = static_cast<int64_t>(blockIdx.x + 1) * p.N / p.grid;
+  const int rows = static_cast<int>(r_end - r_begin);
+  const int64_t b0 = r_begin * p.row_bytes, b1 = r_end * p.row_bytes;
+  const int64_t a0 = b0 & ~int64_t(15);
+
+  pdl_launch_dependents();
+  if (tid == 0) {
+    mbar_init(wbar, 1);
+    mbar_init(xbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue_w = [&]() {
+    int64_t a1 = (b1 + 15) & ~int64_t(15);
+    const int64_t lim = p.total_bytes & ~int64_t(15);
+    uint8_t *dst = smem + p.w_off;
+    if (a1 > lim) {  // bytes past the last 16-byte boundary of W by hand
+      for (int64_t t = lim; t < b1; ++t) dst[t - a0] = p.W[t];
+      a1 = lim;
+    }
+    const uint32_t bytes = static_cast<uint32_t>(a1 - a0);
+    mbar_arrive_expect_tx(wbar, bytes);
+    const uint64_t pol = l2_evict_first_policy();
+    constexpr uint32_t kPiece = 8192;  // several copies in flight
+    for (uint32_t o = 0; o < bytes; o += kPiece)
+      bulk_g2s(dst + o, p.W + a0 + o, min(kPiece, bytes - o), wbar, pol);
+  };
+  auto issue_x = [&]() {
+    mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(p.KB) * 128u);
+    tma_load_2d(smem + p.xs_off, &p.xmap, 0, 0, xbar);
+  };
+  if (tid == 0) {
+    if (p.prefetch_before_wait) {
+      issue_w();
+      pdl_wait();
+      issue_x();
+    } else {
+      pdl_wait();
+      issue_x();
+      issue_w();
+    }
+  }
+
+  // ---- decode the owned blocks into registers (does not need X)
+  const int cw = warp % p.cg, k = warp / p.cg;
+  const int col = cw * 32 + lane;
+  const bool act = col < p.KB;
+  const uint32_t wbase = smem_u32(smem + p.w_off) + static_cast<uint32_t>(b0 - a0);
+  float2 wq[U][16];
+  float wd[U];
+  bool ok = mbar_wait(wbar, 0);
+  if (!ok && lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int rl = k + u * p.wpw;
+    if (ok && act && rl < rows) {
+      const uint32_t sa = wbase + static_cast<uint32_t>(rl * p.row_bytes) + 34u * col;
+      const uint32_t mis = sa & 2u, wa = sa - mis;
+      uint32_t w[9];
+#pragma unroll
+      for (int i = 0; i < 9; ++i) w[i] = lds_u32(wa + 4 * i);
+      const uint32_t r8 = mis << 3, sh = 16u + r8;
+      wd[u] = half_bits_to_float(__funnelshift_rc(w[0], w[1], r8));
+      const float2 nb = make_float2(-8388736.0f, -8388736.0f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t q4 = __funnelshift_rc(w[i], w[i + 1], sh) ^ 0x80808080u;
+        const float2 f01 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7440u)),
+                                       __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7441u)));
+        const float2 f23 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7442u)),
+                                       __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7443u)));
+        wq[u][2 * i] = __fadd2_rn(f01, nb);  // exact codes q
+        wq[u][2 * i + 1] = __fadd2_rn(f23, nb);
+      }
+    } else {
+      wd[u] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) wq[u][i] = make_float2(0.f, 0.f);
+    }
+  }
+
+  // ---- activations (after the preceding grid has finished)
+  pdl_wait();
+  float2 x2[16];
+  if (ok && !mbar_wait(xbar, 0)) {
+    ok = false;
+    if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+  }
+  if (ok && act) {
+    const uint32_t xa = smem_u32(smem + p.xs_off);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 v = lds_f4(xa + 16u * (col * 8 + (j ^ (col & 7))));
+      x2[2 * j] = make_float2(v.x, v.y);
+      x2[2 * j + 1] = make_float2(v.z, v.w);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) x2[j] = make_float2(0.f, 0.f);
+  }
+
+  // ---- products: four packed accumulators per row, then a fixed tree
+  float part[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    float2 a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = __fmul2_rn(wq[u][i], x2[i]);
+#pragma unroll
+    for (int i = 4; i < 16; ++i) a[i & 3] = __ffma2_rn(wq[u][i], x2[i], a[i & 3]);
+    const float2 t = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+    part[u] = wd[u] * (t.x + t.y);
+  }
+  if (!ok && tid == 0) {  // error path: give copies still in flight a bounded chance to land
+    if (!mbar_wait(wbar, 0) || !mbar_wait(xbar, 0)) atomicOr(&g_q8_gemv_status, kDevTimeoutDrain);
+  }
+  const float tot = warp_reduce_scatter<U>(part, lane);
+  const int ui = scatter_index<U>(lane);
+  const int rl = k + ui * p.wpw;
+  if (p.cg == 1) {
+    if (scatter_writer<U>(lane) && rl < rows) p.Y[r_begin + rl] = tot;
+    return;
+  }
+  if (scatter_writer<U>(lane) && rl < rows) red[cw * p.max_rows + rl] = tot;
+  __syncthreads();
+  for (int r = tid; r < rows; r += blockDim.x) {
+    float v = red[r];
+    for (int c = 1; c < p.cg; ++c) v += red[c * p.max_rows + r];
+    p.Y[r_begin + r] = v;
+  }
+}
+
 int align_up(int64_t v, int a) { return static_cast<int>((v + a - 1) / a * a); }
 
 template <int MODE, int MP, int RG>
@@ -562,10 +736,91 @@ qmm_status launch_stream(const DevInfo &dev, int M, int64_t N, int K, const void
   return cuda_check(e, MODE == kModeF32 ? "q8_gemv launch" : "q8q8_gemv launch");
 }
 
+
+// Resident variant when every CTA's weight slice fits (returns false if not).
+bool try_launch_resident(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, float *Y,
+                         cudaStream_t stream, uint32_t flags, qmm_status *out) {
+  const int KB = K / 32;
+  const int cg = (KB + 31) / 32;
+  if (K * 4 > kPanelBytes) return false;
+  const int grid = static_cast<int>(std::min<int64_t>(N, dev.sms));
+  const int64_t rows = (N + grid - 1) / grid;
+  const int64_t row_bytes = 34ll * KB;
+  // U rows per warp; max warps per CTA for each U (register budget)
+  const int maxw[3] = {16, 16, 11};
+  int U = 0, wpw = 0;
+  for (int ui = 0; ui < 3; ++ui) {
+    const int u = 1 << ui;
+    const int w = static_cast<int>((rows + u - 1) / u);
+    if (cg * w <= maxw[ui]) {
+      U = u;
+      wpw = w;
+      break;
+    }
+  }
+  if (U == 0) return false;
+  const int64_t slice = rows * row_bytes + 48;
+  if (slice > 48 * 1024) return false;
+  RParams p{};
+  p.W = static_cast<const uint8_t *>(W);
+  p.Y = Y;
+  p.N = N;
+  p.row_bytes = row_bytes;
+  p.total_bytes = N * row_bytes;
+  p.K = K;
+  p.KB = KB;
+  p.grid = grid;
+  p.cg = cg;
+  p.wpw = wpw;
+  p.max_rows = static_cast<int>(rows);
+  p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
+  p.xs_off = 1024;
+  p.red_off = align_up(p.xs_off + KB * 128, 128);
+  p.w_off = align_up(p.red_off + cg * rows * 4, 128);
+  const size_t smem = static_cast<size_t>(align_up(p.w_off + slice, 128)) + 1024;
+  const uint64_t dims[2] = {32, static_cast<uint64_t>(KB)};
+  const uint64_t strides[1] = {128};
+  const uint32_t box[2] = {32, static_cast<uint32_t>(KB)};
+  qmm_status st = encode_tiled(&p.xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, X, dims, strides, box,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QMM_OK) {
+    *out = st;
+    return true;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(cg * wpw * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto go = [&](auto kern) -> cudaError_t {
+    static bool configured[3][64] = {};
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    const int idx = U == 1 ? 0 : U == 2 ? 1 : 2;
+    if (dev_id >= 0 && dev_id < 64 && !configured[idx][dev_id]) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+      if (e != cudaSuccess) return e;
+      configured[idx][dev_id] = true;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, p);
+  };
+  cudaError_t e = U == 1 ? go(q8_gemv_resident_kernel<1>) : U == 2 ? go(q8_gemv_resident_kernel<2>)
+                                                                    : go(q8_gemv_resident_kernel<4>);
+  *out = cuda_check(e, "q8_gemv launch");
+  return true;
+}
+
 }  // namespace
 
 qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
                           cudaStream_t stream, uint32_t flags) {
+  qmm_status st;
+  if (M == 1 && try_launch_resident(dev, N, K, W, X, Y, stream, flags, &st)) return st;
   return launch_stream<kModeF32>(dev, M, N, K, W, X, nullptr, nullptr, Y, nullptr, stream, flags);
 }
 
