@@ -61,6 +61,8 @@ constexpr int kSmemBudget = 96 * 1024;   // two CTAs of consecutive launches fit
 constexpr int kBarBytes = 256;           // full[8] + empty[8] mbarriers
 constexpr int kMaxConsumerWarps = 16;
 constexpr int kPanelBytes = 32 * 1024;  // activation panel kept in shared memory up to this size (256 rows)
+constexpr int64_t kMmaMinSliceWeights = 16384;  // per-CTA weights above which M = 1 uses tensor cores
+constexpr int kMmaMaxK = 2048;  // longer rows: the per-CTA activation split costs more than it saves
 
 enum : int { kModeF32 = 0, kModeQ8 = 1, kModeQ8Dots = 2 };
 
@@ -631,6 +633,270 @@ q8_gemv_resident_kernel(const __grid_constant__ RParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core resident variant (M = 1) for weight slices whose fp32 register
+// form would fill the SM: the next launch in the stream could then not start
+// streaming its own weights before this one exits. Here the codes are held as
+// fp16 (exact for int8), half that footprint, so two consecutive launches
+// share an SM and the next one's weights land and are converted while this one
+// computes. Every CTA splits the whole activation vector once, so this only
+// pays for short rows (measured on B200 in a chain of dependent launches:
+// 896 -> 4864 at 2.80 us per GEMV against 3.19 us for the fp32 resident
+// kernel; 4864 -> 896 at 4.05 us against 3.38 us, so long rows stay there).
+//
+//  * mma.m16n8k16 with the weights as A: rows 0..7 of A are the eight rows of
+//    a row group at block b, rows 8..15 the same rows at block b + 1. Thread
+//    (g, t) holds codes 8t..8t+7 of row g at both blocks; inside a block the k
+//    order is free, so with c0 c1 c2 c3 = codes 8t+4s .. 8t+4s+3 (slice s) the
+//    register at k = 2t, 2t+1 holds (c0, c2) and the one at k = 2t+8, 2t+9
+//    holds (c1, c3). A masked xor puts each biased byte in the mantissa of
+//    1024 and one packed fp16 subtraction of 1152 leaves the code exactly.
+//  * Activations as B: column 0/1 = hi/lo parts of block b, column 2/3 = those
+//    of block b + 1 (columns 4..7 repeat 0..3). Each 32-block is scaled by
+//    2^(141 - E_b), E_b the biased exponent of its largest |x|, so its largest
+//    element lies in [2^14, 2^15), and split (Veltkamp) into hi with 11
+//    significant bits and lo = v - hi, both then rounded to fp16:
+//    |v - hi - lo| <= 2^-23 |v| + 2^-25. Products are exact in fp32. The parts
+//    are built once per CTA, in place over the activation vector in shared
+//    memory, laid out so that each lane reads its B registers with one 16-byte
+//    load.
+//  * C row g, columns 0 + 1 (thread (g, 0)) is row g's dot with block b;
+//    C row g + 8, columns 2 + 3 (thread (g, 1)) the dot with block b + 1. Each
+//    adds (dot * d) * 2^(E_b - 141) to its accumulator: dot * d is a normal
+//    number and the power-of-two factor costs one rounding, also where the
+//    result is subnormal. Threads (g, 0) and (g, 1) are summed and the warps
+//    (split-K) are added in warp order. Deterministic.
+
+struct alignas(64) MParams {
+  const uint8_t *W;
+  const float *X;
+  float *Y;
+  int64_t N;
+  int64_t row_bytes;
+  int64_t total_bytes;
+  int64_t ngroups;  // ceil(N / 8)
+  int K, KB, KBp;   // KBp = KB rounded up to even
+  int grid;
+  int np;           // block pairs per warp
+  int x_off, d_off, e_off, red_off, w_off;  // shared-memory offsets (bytes)
+  int prefetch_before_wait;
+};
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+
+// int8 codes in bytes 0 and 2 of w -> fp16x2 (exact).
+__device__ __forceinline__ uint32_t codes_even_h2(uint32_t w) {
+  const uint32_t biased = (w & 0x00ff00ffu) ^ 0x64806480u;  // 1024 + (code + 128) in each half
+  const __half2 k1152 = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+  return h2_bits(__hsub2(*reinterpret_cast<const __half2 *>(&biased), k1152));
+}
+
+// Veltkamp split of a pair: hi = the 11 leading bits, lo = v - hi (exact in fp32).
+__device__ __forceinline__ void split_pair(float2 v, uint32_t &hi, uint32_t &lo) {
+  const float2 c = __fmul2_rn(v, make_float2(8193.0f, 8193.0f));  // (rounded ops: never contracted)
+  const float hx = __fsub_rn(c.x, __fsub_rn(c.x, v.x)), hy = __fsub_rn(c.y, __fsub_rn(c.y, v.y));
+  hi = h2_bits(__floats2half2_rn(hx, hy));
+  lo = h2_bits(__floats2half2_rn(__fsub_rn(v.x, hx), __fsub_rn(v.y, hy)));
+}
+
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9},"
+      " {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int GM, int NPM>
+__global__ void __launch_bounds__(256, 2) q8_gemv_mma_kernel(const __grid_constant__ MParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw;  // 16-byte aligned, all the layout needs; kept un-cast so accesses stay LDS/STS
+  uint64_t *wbar = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *xbar = wbar + 1;
+  float *dtab = reinterpret_cast<float *>(smem + p.d_off);  // [group][block][8 rows] scales
+  float *ftab = reinterpret_cast<float *>(smem + p.e_off);  // block factors 2^(E_b - 141)
+  float *red = reinterpret_cast<float *>(smem + p.red_off); // [warp][group][8 rows] partials
+  uint8_t *xtab = smem + p.x_off;                           // activations, then their parts
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3, odd = t & 1;
+  const int64_t g_begin = static_cast<int64_t>(blockIdx.x) * p.ngroups / p.grid;
+  const int64_t g_end = static_cast<int64_t>(blockIdx.x + 1) * p.ngroups / p.grid;
+  const int groups = static_cast<int>(g_end - g_begin);
+  const int64_t r_begin = 8 * g_begin;
+  const int64_t r_end = min(p.N, 8 * g_end);
+  const int rows = static_cast<int>(r_end - r_begin);
+  const int64_t b0 = r_begin * p.row_bytes, b1 = r_end * p.row_bytes;
+  const int64_t a0 = b0 & ~int64_t(15);
+
+  pdl_launch_dependents();
+  if (tid == 0) {
+    mbar_init(wbar, 1);
+    mbar_init(xbar, 1);
+    fence_mbar_init();
+  }
+  if (p.KBp > p.KB) {  // padding block of an odd block count: zero parts, scales and exponent
+    for (int i = tid; i < 32 + 8 * GM; i += blockDim.x) {
+      if (i < 32) reinterpret_cast<float *>(xtab + 128 * p.KB)[i] = 0.f;
+      else dtab[((i - 32) / 8 * p.KBp + p.KB) * 8 + (i - 32) % 8] = 0.f;
+    }
+    if (tid == 0) ftab[p.KB] = 0.f;
+  }
+  __syncthreads();
+  auto issue_w = [&]() {
+    int64_t a1 = (b1 + 15) & ~int64_t(15);
+    const int64_t lim = p.total_bytes & ~int64_t(15);
+    uint8_t *dst = smem + p.w_off;
+    if (a1 > lim) {  // bytes past the last 16-byte boundary of W by hand
+      for (int64_t i = lim; i < b1; ++i) dst[i - a0] = p.W[i];
+      a1 = lim;
+    }
+    const uint32_t bytes = static_cast<uint32_t>(a1 - a0);
+    mbar_arrive_expect_tx(wbar, bytes);
+    const uint64_t pol = l2_evict_first_policy();
+    constexpr uint32_t kPiece = 8192;  // several copies in flight
+    for (uint32_t o = 0; o < bytes; o += kPiece)
+      bulk_g2s(dst + o, p.W + a0 + o, min(kPiece, bytes - o), wbar, pol);
+  };
+  auto issue_x = [&]() {
+    const uint32_t bytes = static_cast<uint32_t>(p.K) * 4u;
+    mbar_arrive_expect_tx(xbar, bytes);
+    bulk_g2s(xtab, p.X, bytes, xbar, l2_evict_last_policy());
+  };
+  if (tid == 0) {
+    if (!p.prefetch_before_wait) {
+      pdl_wait();
+      issue_x();
+    }
+    issue_w();
+  }
+
+  // ---- A fragments (fp16 codes of block pairs) and block scales; independent of X
+  const int P = p.KBp / 2;
+  const int kp0 = warp * p.np;
+  const uint32_t wbase = smem_u32(smem + p.w_off) + static_cast<uint32_t>(b0 - a0);
+  uint32_t Wr[NPM][GM][8];
+  bool ok = mbar_wait(wbar, 0);
+  if (!ok && lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+#pragma unroll
+  for (int j = 0; j < NPM; ++j) {
+    const int pp = kp0 + j;
+    const bool pair_ok = j < p.np && pp < P;
+#pragma unroll
+    for (int gi = 0; gi < GM; ++gi) {
+      const int rl = gi * 8 + g;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int blk = 2 * pp + h;
+        uint32_t w0 = 0u, w1 = 0u;
+        if (ok && pair_ok && blk < p.KB && rl < rows) {
+          const uint32_t blk_a = wbase + static_cast<uint32_t>(rl * p.row_bytes) + 34u * blk;
+          const uint32_t ca = blk_a + 2u + 8u * t;  // codes 8t..8t+7 (2-byte aligned)
+          const uint32_t mis = ca & 2u, wa = ca - mis, sh = mis << 3;
+          const uint32_t v0 = lds_u32(wa), v1 = lds_u32(wa + 4), v2 = lds_u32(wa + 8);
+          w0 = __funnelshift_r(v0, v1, sh);
+          w1 = __funnelshift_r(v1, v2, sh);
+          if (t == 0) dtab[(gi * p.KBp + blk) * 8 + g] = half_bits_to_float(lds_u16(blk_a));
+        } else if (pair_ok && blk < p.KB && t == 0) {
+          dtab[(gi * p.KBp + blk) * 8 + g] = 0.f;
+        }
+        Wr[j][gi][0 + h] = codes_even_h2(w0);       // slice 0, k = 2t, 2t+1: codes (0, 2)
+        Wr[j][gi][2 + h] = codes_even_h2(w0 >> 8);  // slice 0, k = 2t+8, 2t+9: codes (1, 3)
+        Wr[j][gi][4 + h] = codes_even_h2(w1);       // slice 1: codes (4, 6)
+        Wr[j][gi][6 + h] = codes_even_h2(w1 >> 8);  // slice 1: codes (5, 7)
+      }
+    }
+  }
+
+  // ---- activations (after the preceding grid): scaled hi/lo parts in place
+  pdl_wait();
+  if (tid == 0 && p.prefetch_before_wait) issue_x();
+  if (ok && !mbar_wait(xbar, 0)) {
+    ok = false;
+    if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+  }
+  const int slots = p.KB * 4;  // (block, t): eight activations 8t..8t+7 of a block
+#pragma unroll 2
+  for (int base = warp * 32; base < slots; base += blockDim.x) {
+    const int s = base + lane;
+    const bool have = ok && s < slots;
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f), w = u;
+    float4 *slot = reinterpret_cast<float4 *>(xtab + 32 * s);
+    if (have) {
+      u = slot[0];
+      w = slot[1];
+    }
+    uint32_t mb = max(max(max(__float_as_uint(u.x) & 0x7fffffffu, __float_as_uint(u.y) & 0x7fffffffu),
+                          max(__float_as_uint(u.z) & 0x7fffffffu, __float_as_uint(u.w) & 0x7fffffffu)),
+                      max(max(__float_as_uint(w.x) & 0x7fffffffu, __float_as_uint(w.y) & 0x7fffffffu),
+                          max(__float_as_uint(w.z) & 0x7fffffffu, __float_as_uint(w.w) & 0x7fffffffu)));
+    mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+    mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+    const int E = max(static_cast<int>(mb >> 23), 1);  // largest |x| of the block < 2^(E - 126)
+    const int sh = 141 - E, sh1 = min(sh, 127);
+    const float2 s1 = make_float2(__int_as_float((127 + sh1) << 23), __int_as_float((127 + sh1) << 23));
+    const float2 s2 = make_float2(__int_as_float((127 + sh - sh1) << 23), __int_as_float((127 + sh - sh1) << 23));
+    uint4 hi, lo;
+    split_pair(__fmul2_rn(__fmul2_rn(make_float2(u.x, u.z), s1), s2), hi.x, lo.x);  // elements 0, 2
+    split_pair(__fmul2_rn(__fmul2_rn(make_float2(u.y, u.w), s1), s2), hi.y, lo.y);  // 1, 3
+    split_pair(__fmul2_rn(__fmul2_rn(make_float2(w.x, w.z), s1), s2), hi.z, lo.z);  // 4, 6
+    split_pair(__fmul2_rn(__fmul2_rn(make_float2(w.y, w.w), s1), s2), hi.w, lo.w);  // 5, 7
+    if (have) {
+      uint4 *dst = reinterpret_cast<uint4 *>(xtab + 32 * s);
+      dst[0] = hi;
+      dst[1] = lo;
+      // 2^(E - 141), exact (a subnormal power of two below E = 15)
+      if (t == 0) ftab[s >> 2] = E >= 15 ? __int_as_float((E - 14) << 23) : __int_as_float(1 << (E + 8));
+    }
+  }
+  __syncthreads();
+
+  // ---- tensor-core block dots and the scale epilogue
+  float acc[GM];
+#pragma unroll
+  for (int gi = 0; gi < GM; ++gi) acc[gi] = 0.f;
+  if (ok) {
+#pragma unroll
+    for (int j = 0; j < NPM; ++j) {
+      const int pp = kp0 + j;
+      if (j < p.np && pp < P) {
+        // B registers: column g of the (hi b, lo b, hi b+1, lo b+1) pattern
+        const uint4 xb =
+            *reinterpret_cast<const uint4 *>(xtab + 128 * (2 * pp + ((g >> 1) & 1)) + 32 * t + 16 * (g & 1));
+        const int bo = 2 * pp + odd;  // the block whose dot this thread keeps
+        const float f = ftab[bo];
+#pragma unroll
+        for (int gi = 0; gi < GM; ++gi) {
+          if (gi < groups) {
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_f16_16816(c, Wr[j][gi][0], Wr[j][gi][1], Wr[j][gi][2], Wr[j][gi][3], xb.x, xb.y);
+            mma_f16_16816(c, Wr[j][gi][4], Wr[j][gi][5], Wr[j][gi][6], Wr[j][gi][7], xb.z, xb.w);
+            const float sv = odd ? c[2] + c[3] : c[0] + c[1];
+            // (dot * d) is a normal number; one rounding for the power-of-two factor
+            acc[gi] = fmaf(sv * dtab[(gi * p.KBp + bo) * 8 + g], f, acc[gi]);
+          }
+        }
+      }
+    }
+  }
+  if (!ok && tid == 0) {  // error path: give copies still in flight a bounded chance to land
+    if (!mbar_wait(wbar, 0) || !mbar_wait(xbar, 0)) atomicOr(&g_q8_gemv_status, kDevTimeoutDrain);
+  }
+#pragma unroll
+  for (int gi = 0; gi < GM; ++gi) {
+    const float v = acc[gi] + __shfl_xor_sync(0xffffffffu, acc[gi], 1);  // even + odd blocks
+    if (t == 0 && gi < groups) red[(warp * GM + gi) * 8 + g] = v;
+  }
+  __syncthreads();
+  const int nw = blockDim.x >> 5;
+  for (int r = tid; r < rows; r += blockDim.x) {
+    const int gi = r >> 3, rr = r & 7;
+    float v = 0.f;
+    for (int w = 0; w < nw; ++w) v += red[(w * GM + gi) * 8 + rr];
+    p.Y[r_begin + r] = v;
+  }
+}
+
 int align_up(int64_t v, int a) { return static_cast<int>((v + a - 1) / a * a); }
 
 template <int MODE, int MP, int RG>
@@ -815,12 +1081,101 @@ bool try_launch_resident(const DevInfo &dev, int64_t N, int K, const void *W, co
   return true;
 }
 
+// Tensor-core resident variant (returns false when the shape does not suit it).
+bool try_launch_mma(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, float *Y,
+                    cudaStream_t stream, uint32_t flags, qmm_status *out) {
+  constexpr int kMaxWarps = 8;
+  constexpr int kSmemMax = 110 * 1024;  // two CTAs per SM
+  const int KB = K / 32;
+  const int KBp = (KB + 1) & ~1;
+  const int P = KBp / 2;
+  if (static_cast<int64_t>(KBp) * 128 > kPanelBytes) return false;
+  const int64_t ngroups = (N + 7) / 8;
+  const int grid = static_cast<int>(std::min<int64_t>(ngroups, dev.sms));
+  const int gmax = static_cast<int>((ngroups + grid - 1) / grid);
+  // instances: row groups per CTA (GM) x block pairs per warp (NPM)
+  struct Inst {
+    int gm, npm;
+    void (*kern)(MParams);
+  };
+  static const Inst insts[] = {
+      {1, 2, q8_gemv_mma_kernel<1, 2>}, {1, 4, q8_gemv_mma_kernel<1, 4>}, {2, 5, q8_gemv_mma_kernel<2, 5>},
+      {3, 3, q8_gemv_mma_kernel<3, 3>}, {4, 2, q8_gemv_mma_kernel<4, 2>}, {5, 2, q8_gemv_mma_kernel<5, 2>},
+      {8, 1, q8_gemv_mma_kernel<8, 1>},
+  };
+  constexpr int kInsts = static_cast<int>(sizeof(insts) / sizeof(insts[0]));
+  int pick = -1, nw = 0;
+  for (int i = 0; i < kInsts; ++i) {
+    const int w = (P + insts[i].npm - 1) / insts[i].npm;
+    if (insts[i].gm >= gmax && w <= kMaxWarps) {
+      pick = i;
+      nw = w;
+      break;
+    }
+  }
+  if (pick < 0) return false;
+  const Inst &in = insts[pick];
+  const int64_t row_bytes = 34ll * KB;
+  MParams p{};
+  p.W = static_cast<const uint8_t *>(W);
+  p.X = X;
+  p.Y = Y;
+  p.N = N;
+  p.row_bytes = row_bytes;
+  p.total_bytes = N * row_bytes;
+  p.ngroups = ngroups;
+  p.K = K;
+  p.KB = KB;
+  p.KBp = KBp;
+  p.grid = grid;
+  p.np = (P + nw - 1) / nw;
+  p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
+  p.x_off = 128;
+  p.d_off = align_up(p.x_off + 128ll * KBp, 16);
+  p.e_off = align_up(p.d_off + 32ll * in.gm * KBp, 16);
+  p.red_off = align_up(p.e_off + 4ll * KBp, 16);
+  p.w_off = align_up(p.red_off + 32ll * nw * in.gm, 128);
+  const int64_t slice = 8ll * gmax * row_bytes + 48;
+  const size_t smem = static_cast<size_t>(align_up(p.w_off + slice, 128));
+  if (smem > static_cast<size_t>(kSmemMax)) return false;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(32 * nw);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static bool configured[kInsts][64] = {};
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  if (dev_id >= 0 && dev_id < 64 && !configured[pick][dev_id]) {
+    cudaError_t e = cudaFuncSetAttribute(in.kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
+    if (e != cudaSuccess) {
+      *out = cuda_check(e, "q8_gemv attribute");
+      return true;
+    }
+    configured[pick][dev_id] = true;
+  }
+  *out = cuda_check(cudaLaunchKernelEx(&cfg, in.kern, p), "q8_gemv launch");
+  return true;
+}
+
 }  // namespace
 
 qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
                           cudaStream_t stream, uint32_t flags) {
   qmm_status st;
-  if (M == 1 && try_launch_resident(dev, N, K, W, X, Y, stream, flags, &st)) return st;
+  if (M == 1) {
+    // Slices whose fp32 register form would fill the SM go to the tensor-core
+    // variant (two launches per SM); smaller ones to the fp32 resident kernel.
+    const int64_t rows_per_cta = (N + dev.sms - 1) / dev.sms;
+    if (rows_per_cta * K >= kMmaMinSliceWeights && K <= kMmaMaxK && try_launch_mma(dev, N, K, W, X, Y, stream, flags, &st))
+      return st;
+    if (try_launch_resident(dev, N, K, W, X, Y, stream, flags, &st)) return st;
+  }
   return launch_stream<kModeF32>(dev, M, N, K, W, X, nullptr, nullptr, Y, nullptr, stream, flags);
 }
 

@@ -110,3 +110,104 @@ def test_empty_and_k0():
     assert qmm.lib.qmm_q8_gemv(0, 5, 64, 32, 0, 0, 0, 0) == 0
     assert qmm.lib.qmm_q8_gemv(1, 0, 64, 32, 0, 0, 0, 0) == 0
     assert qmm.device_status() == 0
+
+
+@pytest.mark.parametrize("n,k", [(37, 256), (2000, 2048)])
+def test_extreme_codes_and_scales_single_row(n, k):
+    # the M = 1 kernels on the same extremes: (37, 256) takes the fp32 register-resident
+    # kernel, (2000, 2048) the tensor-core resident one
+    g = syn.rng(13)
+    q = g.integers(-128, 128, size=(n, k)).astype(np.int8)
+    q[0, :] = -128
+    q[1, :] = 127
+    d = syn.fp16_bits(np.abs(g.standard_normal((n, k // 32))) * 0.02)
+    d[2, :] = 0x0000
+    d[3, :] = 0x8000
+    d[4, :] = 0x0001
+    d[5, :] = 0x03FF
+    d[6, :] = 0x7BFF
+    d[7, :] = 0xBC00
+    W = syn.pack_q8_0(q, d)
+    x = syn.act_f32(g, 1, k)
+    y = run(W, x, n)
+    ref, S = oracle.gemv(syn.Q8_0, W, x, n)
+    assert_within(y, ref, S, TOL_FP32, "extreme codes/scales, M=1")
+    assert y[0, 2] == 0 and y[0, 3] == 0
+
+
+def _dynamic_range_inputs(g, k):
+    x = syn.act_f32(g, 1, k)
+    mixed = (x * 10.0 ** g.uniform(-4, 4, size=x.shape)).astype(np.float32)
+    blocks = x.copy()
+    blocks[0, 32:64] = 0.0                       # an all-zero block
+    blocks[0, 64] = 2.0 ** 12                    # one element far above the rest of its block
+    blocks[0, 96:128] = 2.0 ** np.arange(-15, 17, dtype=np.float64)  # exact powers of two
+    blocks[0, 128] = -1.0                        # block max exactly a power of two
+    blocks[0, 129:160] = 0.5
+    return {
+        "mixed_1e-4_1e4": mixed,
+        "tiny_1e-33": (x * 1e-33).astype(np.float32),
+        "subnormal": (x * 1e-40).astype(np.float32),
+        "huge_1e30": (x * 1e30).astype(np.float32),
+        "structured_blocks": blocks.astype(np.float32),
+    }
+
+
+@pytest.mark.parametrize("n,k", [(1152, 896), (896, 4864), (45, 160)])
+def test_single_row_activation_dynamic_range(n, k):
+    g = syn.rng(21 + n + k)
+    W, _, _ = syn.q8_0_weights(g, n, k)
+    for name, x in _dynamic_range_inputs(g, k).items():
+        y = run(W, x, n)
+        ref, S = oracle.gemv(syn.Q8_0, W, x, n)
+        assert_within(y, ref, S, TOL_FP32, f"M=1 N={n} K={k} x={name}")
+
+
+def test_single_row_zero_activation_gives_exact_zero():
+    g = syn.rng(22)
+    n, k = 4864, 896
+    W, _, _ = syn.q8_0_weights(g, n, k)
+    y = run(W, np.zeros((1, k), np.float32), n)
+    assert np.all(y == 0)
+
+
+@pytest.mark.parametrize("n,k", [
+    (4869, 896),   # ragged last row group, five groups per CTA
+    (4864, 864),   # odd block count (a zero padding block), five groups per CTA
+    (2000, 2048),  # two groups per CTA
+    (1200, 2048),  # one or two groups per CTA, seven warps of five block pairs
+    (3000, 1024),  # three groups per CTA
+    (9000, 512),   # eight groups per CTA
+    (600, 5120),   # long rows: fp32 resident kernel
+    (893, 4864),   # long rows, ragged N: fp32 resident kernel
+])
+def test_single_row_large_slices(n, k):
+    # M = 1 slices large enough for the tensor-core resident kernel (short rows)
+    check(1, n, k, seed=31 + n + k)
+
+
+def test_single_row_tensor_core_chained_calls():
+    # consecutive launches in one stream (programmatic dependent launch, early weights):
+    # each call reads the previous call's output as its activation vector
+    g = syn.rng(41)
+    k = 896
+    Ws = [syn.q8_0_weights(g, k, k)[0] for _ in range(3)] + [syn.q8_0_weights(g, 4864, k)[0]]
+    x = syn.act_f32(g, 1, k)
+    Wd = [dev(w) for w in Ws]
+    bufs = [dev(x)] + [torch.empty((1, k), dtype=torch.float32, device="cuda") for _ in range(3)]
+    out = torch.empty((1, 4864), dtype=torch.float32, device="cuda")
+    ys = bufs[1:] + [out]
+    for i, w in enumerate(Wd):
+        n = ys[i].shape[1]
+        st = qmm.lib.qmm_q8_gemv_ex(1, n, k, 32, w.data_ptr(), bufs[i].data_ptr(), ys[i].data_ptr(),
+                                    qmm.QMM_FLAG_EARLY_WEIGHTS, 0)
+        assert st == 0
+    torch.cuda.synchronize()
+    assert qmm.device_status() == 0
+    xin = x
+    for i, w in enumerate(Ws):
+        n = ys[i].shape[1]
+        ref, S = oracle.gemv(syn.Q8_0, w, xin, n)
+        got = host(ys[i])
+        assert_within(got, ref, S, TOL_FP32, f"chained call {i}")
+        xin = got.astype(np.float32)
