@@ -8,23 +8,34 @@
 // round-to-nearest-even to bf16) and the products accumulate in fp32 in
 // tensor memory.
 //
-// B200 design (one CTA per 128 x MT output tile, MT <= 256 tokens):
+// B200 design (one CTA per 128 x MT output tile and K range, MT <= 256 tokens):
 //  * MMA shape M = 128 weight rows, N = MT tokens, K = 16 (kind::f16, bf16
 //    inputs, fp32 accumulator in TMEM, one thread issues, cta_group::1). The
 //    accumulator D[n][m] lives in MT TMEM columns x 128 lanes.
-//  * A (weights, 128 x 64 per stage) is written by four "dequant" warps in
+//  * A (weights, 128 x 64 per stage) is written by eight "dequant" warps in
 //    the canonical K-major 128-byte-swizzled layout (8-row atoms of 1 KB,
 //    16-byte chunk c of row r at c ^ (r % 8)); B (X, MT x 64 per stage) comes
 //    straight from a 2-D TMA load with the same 128-byte swizzle.
-//  * Raw weight blocks arrive in 8-block (256 k) chunks per 128-row tile:
-//    by 2-D TMA (W viewed as uint16 rows; needs 16-byte row pitch, i.e.
-//    K % 256 == 0) or, otherwise, by the dequant warps' own global loads.
+//  * Raw weight blocks arrive in 8-block (256 k) chunks per 128-row tile by
+//    2-D TMA. A Q8_0 row is 34 * K/32 bytes, in general not a multiple of 16
+//    (a TMA row pitch must be), so W is viewed as super-rows of rs = 1, 2, 4
+//    or 8 rows whose pitch is; one box per row position of a super-row, each
+//    started at the 16-byte boundary below the chunk, and the dequant warps
+//    index from the row's offset. The < rs rows at the end of W that do not
+//    fill a super-row are read by the dequant warps directly.
+//  * Split K: when the output tiles alone leave SMs idle, the K range is split
+//    across the CTAs of a thread-block cluster (gridDim.z = cluster size).
+//    After every CTA's accumulator is complete, each CTA scatters its partial
+//    tile through distributed shared memory so that rank r receives all
+//    partials of its 128/S weight rows, then sums them in rank order and
+//    writes Y: deterministic, and no global scratch memory.
 //  * Pipelines: producer -> (X tile, raw chunk) -> dequant -> A tile -> MMA
 //    -> tcgen05.commit frees the stage. After the last MMA a commit signals
-//    the four dequant warps, which become the epilogue: tcgen05.ld 32 columns
-//    at a time (lane = weight row) and coalesced stores of Y.
+//    the eight dequant warps, which become the epilogue: tcgen05.ld 32 columns
+//    at a time (lane = weight row) and coalesced stores of Y (or the scatter).
 //  * Every mbarrier wait is bounded; on a timeout the kernel records a status
-//    bit, finishes without waiting further and still frees its TMEM.
+//    bit, finishes without waiting further (still meeting both cluster
+//    barriers) and frees its TMEM.
 #include <algorithm>
 
 #include "qmm_common.cuh"
@@ -36,27 +47,33 @@ namespace {
 
 static __device__ uint32_t g_prefill_status;
 
-constexpr int kThreads = 192;          // warp 0 producer, warp 1 MMA, warps 2-5 dequant + epilogue
+constexpr int kDqWarps = 8;            // dequant (then epilogue) warps: thread = (weight row, block of the stage, part)
+constexpr int kParts = kDqWarps / 8;    // parts of a block per thread: 32 / kParts weights each
+constexpr int kThreads = 64 + 32 * kDqWarps;  // warp 0 producer, warp 1 MMA, warps 2.. dequant + epilogue
 constexpr int kRawBlocks = 8;          // blocks per raw weight chunk
 constexpr int kStageK = 64;            // k per MMA stage (one 128-byte swizzle row of bf16)
 constexpr int kATileBytes = 128 * 128; // 128 rows x 64 bf16
 constexpr int kRawStages = 2;
+constexpr int kMaxSplit = 8;           // portable cluster size
 
 struct alignas(64) Params {
   CUtensorMap tm_x;    // X: dims {K, M} bf16, box {64, MT}, 128-byte swizzle
-  CUtensorMap tm_w;    // W: dims {row_bytes / 2, N} uint16, box {raw_box_elems, 128}
+  CUtensorMap tm_w;    // W as super-rows of rs rows: dims {rs * row_bytes / 2, N / rs} uint16, box {raw_pitch / 2, 128 / rs}
   const uint8_t *W;
   float *Y;
   int M, K, KB;
   int64_t N;
   int64_t row_bytes;
+  int64_t tma_rows;    // rows loaded by TMA (whole super-rows); the rest by the dequant warps
+  int rs;              // rows per super-row: the smallest of 1, 2, 4, 8 whose pitch is a multiple of 16
   int MT;              // tokens per tile (multiple of 16, <= 256)
   int tmem_cols;
   int stages;          // MMA stages in flight
-  int raw_pitch;       // bytes per row of a raw chunk in shared memory
+  int raw_pitch;       // bytes per row of a raw chunk in shared memory (a chunk + up to 15 bytes in front)
   int x_stage_bytes;
   int off_x, off_a, off_raw;  // shared-memory offsets (1024-aligned)
-  int tma_w;           // raw weights by TMA (1) or by the dequant warps' loads (0)
+  int split;           // K ranges per output tile (cluster size along z)
+  int red_pitch;       // floats per row of the split-K exchange buffer (MT + 4)
 };
 
 // ---------------------------------------------------------------- tcgen05 PTX
@@ -109,6 +126,28 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
 // kind::f16 instruction descriptor: D f32, A = B = bf16, both K-major, M = 128, N = n.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- cluster PTX
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of all CTAs of the cluster; orders shared-memory accesses across it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared-memory address of this CTA's `saddr` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
 }
 
 // ------------------------------------------------------------- block decode
@@ -167,8 +206,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = p.stages;
-  const int nstages = (p.K + kStageK - 1) / kStageK;
-  const int nraw = (p.KB + kRawBlocks - 1) / kRawBlocks;
+  const int nst_all = (p.KB + 1) / 2;  // stages of two blocks over the whole K
+  const int split = p.split;
+  const int zr = split > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int j_lo = zr * nst_all / split, j_hi = (zr + 1) * nst_all / split;
+  const int nst = j_hi - j_lo;                              // this CTA's stages
+  const int nraw = (nst + kRawBlocks / 2 - 1) / (kRawBlocks / 2);  // raw chunks (four stages each)
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;
   const int m0 = blockIdx.y * p.MT;
   constexpr int kBlockBytes = (WT == QMM_Q8_0) ? 34 : 18;
@@ -177,12 +220,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&x_full[s], 1);
-      mbar_init(&a_full[s], 4);
+      mbar_init(&a_full[s], kDqWarps);
       mbar_init(&st_empty[s], 1);
     }
     for (int r = 0; r < kRawStages; ++r) {
       mbar_init(&raw_full[r], 1);
-      mbar_init(&raw_empty[r], 4);
+      mbar_init(&raw_empty[r], kDqWarps);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -193,9 +236,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the preceding grid's writes (X, and any reader of Y) are done
 
   // Bounded wait shared by all roles: after any timeout every later wait
-  // returns at once, so the CTA always reaches the TMEM release below.
+  // returns at once, so the CTA always reaches the cluster barriers and the
+  // TMEM release below.
   auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
     if (*abort_flag) return false;
     if (mbar_wait(bar, parity)) return true;
@@ -207,35 +252,48 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   const uint32_t sbase = smem_u32(smem);
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      pdl_wait();
-      int raw_issued = 0;
-      auto issue_raw = [&](int r) {
-        const int slot = r % kRawStages;
-        if (r >= kRawStages) wait(&raw_empty[slot], static_cast<uint32_t>(r / kRawStages - 1) & 1u);
+    // raw chunk c: blocks from kb of the tile's 128 rows; one TMA box per row
+    // position j of a super-row, started at the 16-byte boundary below the
+    // chunk (the dequant warps index from the offset); out-of-range bytes read 0
+    auto issue_raw = [&](int c) {
+      const int slot = c % kRawStages;
+      if (c >= kRawStages) wait(&raw_empty[slot], static_cast<uint32_t>(c / kRawStages - 1) & 1u);
+      if (*abort_flag) return;  // after a timeout nothing more is copied
+      const int kb = 2 * (j_lo + c * (kRawBlocks / 2));
+      if (n0 < p.tma_rows) {
         mbar_arrive_expect_tx(&raw_full[slot], static_cast<uint32_t>(128 * p.raw_pitch));
-        tma_load_2d(smem + p.off_raw + slot * 128 * p.raw_pitch, &p.tm_w, r * kRawBlocks * kBlockBytes / 2,
-                    static_cast<int>(n0), &raw_full[slot]);
-      };
-      for (int j = 0; j < nstages; ++j) {
-        const int s = j % S;
-        if (p.tma_w) {  // keep the raw chunk feeding this stage (and the next) in flight
-          const int need = min(nraw, (j * kStageK) / (kRawBlocks * 32) + 2);
-          while (raw_issued < need) issue_raw(raw_issued++);
+        const int sub = 128 / p.rs;
+        for (int j = 0; j < p.rs; ++j) {
+          const int64_t off = j * p.row_bytes + static_cast<int64_t>(kb) * kBlockBytes;
+          tma_load_2d(smem + p.off_raw + (slot * 128 + j * sub) * p.raw_pitch, &p.tm_w,
+                      static_cast<int>((off & ~int64_t(15)) / 2), static_cast<int>(n0 / p.rs), &raw_full[slot]);
         }
-        if (j >= S) wait(&st_empty[s], static_cast<uint32_t>(j / S - 1) & 1u);
-        mbar_arrive_expect_tx(&x_full[s], static_cast<uint32_t>(p.x_stage_bytes));
-        tma_load_2d(smem + p.off_x + s * p.x_stage_bytes, &p.tm_x, j * kStageK, m0, &x_full[s]);
+      } else {
+        mbar_arrive(&raw_full[slot]);  // every row of this tile is read directly
+      }
+    };
+    if (lane == 0) {
+      int raw_issued = 0;
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % S;
+        // keep the raw chunk feeding this stage and the next one in flight
+        const int need = min(nraw, i / (kRawBlocks / 2) + 2);
+        while (raw_issued < need) issue_raw(raw_issued++);
+        if (i >= S) wait(&st_empty[s], static_cast<uint32_t>(i / S - 1) & 1u);
+        if (!*abort_flag) {
+          mbar_arrive_expect_tx(&x_full[s], static_cast<uint32_t>(p.x_stage_bytes));
+          tma_load_2d(smem + p.off_x + s * p.x_stage_bytes, &p.tm_x, (j_lo + i) * kStageK, m0, &x_full[s]);
+        }
       }
     }
-    __syncwarp();  // no early exit: every warp meets at the final barrier
+    __syncwarp();
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(p.MT);
-      for (int j = 0; j < nstages; ++j) {
-        const int s = j % S;
-        const uint32_t ph = static_cast<uint32_t>(j / S) & 1u;
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % S;
+        const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
         wait(&x_full[s], ph);
         wait(&a_full[s], ph);
         tc_fence_after();
@@ -245,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 #pragma unroll
           for (int kk = 0; kk < kStageK / 16; ++kk)
             umma_f16(tmem, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc,
-                     j > 0 || kk > 0);
+                     i > 0 || kk > 0);
         }
         umma_commit(&st_empty[s]);  // frees this stage's A and X buffers when the MMAs finish
       }
@@ -254,90 +312,86 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------------ dequant warps
-    pdl_wait();
-    const int r = tid - 64;  // A-tile row = weight row n0 + r
+    // thread (r, h, pt): weight row n0 + r, block h of each stage's two blocks, part pt of the block
+    const int r = (tid - 64) & 127, h = ((tid - 64) >> 7) & 1, pt = (tid - 64) >> 8;
     const int64_t n = n0 + r;
     const bool row_ok = n < p.N;
     const uint32_t a_base0 = sbase + p.off_a;
-    for (int j = 0; j < nstages; ++j) {
-      const int s = j % S;
-      const int kb0 = j * 2;  // first of this stage's two blocks
-      const int raw = kb0 / kRawBlocks, q = (kb0 % kRawBlocks) / 2;
-      if (p.tma_w && q == 0) wait(&raw_full[raw % kRawStages], static_cast<uint32_t>(raw / kRawStages) & 1u);
-      if (j >= S) wait(&st_empty[s], static_cast<uint32_t>(j / S - 1) & 1u);
+    constexpr int kWords = (kBlockBytes + 2 + 3) / 4;  // the block as words, plus the 16-bit shift (Q8: 9, Q4: 5)
+    for (int i = 0; i < nst; ++i) {
+      const int s = i % S;
+      const int c = i / (kRawBlocks / 2), q = i % (kRawBlocks / 2);
+      const int kb = 2 * (j_lo + i) + h;  // this thread's block
+      if (q == 0) wait(&raw_full[c % kRawStages], static_cast<uint32_t>(c / kRawStages) & 1u);
+      if (i >= S) wait(&st_empty[s], static_cast<uint32_t>(i / S - 1) & 1u);
       const uint32_t a_base = a_base0 + s * kATileBytes;
-      // the two blocks' bytes as aligned 32-bit words (Q8: 68 bytes = 17 words, Q4: 36 bytes = 9 words)
-      constexpr int kWords = (2 * kBlockBytes + 3) / 4;
+      const bool have = row_ok && kb < p.KB;
+      // w: the block's bytes from its fp16 scale on, as little-endian words
       uint32_t w[kWords];
-      const bool have2 = kb0 + 1 < p.KB;
-      if (p.tma_w) {
-        const uint32_t ra = sbase + p.off_raw + (raw % kRawStages) * 128 * p.raw_pitch + r * p.raw_pitch +
-                            q * 2 * kBlockBytes;  // 4-byte aligned: 68q / 36q
+      if (n < p.tma_rows) {
+        // row r sits at position j = r % rs of super-row r / rs; its chunk starts
+        // at the source offset modulo 16 inside the box
+        const int j = r % p.rs, sub = 128 / p.rs;
+        const int64_t off = j * p.row_bytes + static_cast<int64_t>(2 * (j_lo + c * (kRawBlocks / 2))) * kBlockBytes;
+        const uint32_t ra = sbase + p.off_raw + ((c % kRawStages) * 128 + j * sub + r / p.rs) * p.raw_pitch +
+                            static_cast<uint32_t>(off & 15) + (2 * q + h) * kBlockBytes;
+        const uint32_t mis = ra & 3u, wa = ra - mis;  // 2-byte aligned
+        if (mis == 0) {
 #pragma unroll
-        for (int i = 0; i < kWords; ++i) w[i] = lds_u32(ra + 4 * i);
-      } else if (row_ok) {
-        const uint8_t *src = p.W + n * p.row_bytes + static_cast<int64_t>(kb0) * kBlockBytes;
-        if (have2 && (reinterpret_cast<uintptr_t>(src) & 3) == 0) {
+          for (int k = 0; k < kWords; ++k) w[k] = lds_u32(wa + 4 * k);
+        } else {
+          uint32_t prev = lds_u32(wa);
 #pragma unroll
-          for (int i = 0; i < kWords; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t *>(src) + i);
-        } else {  // 2-byte aligned, or a lone final block: never read past the block
-          const uint16_t *h = reinterpret_cast<const uint16_t *>(src);
-#pragma unroll
-          for (int i = 0; i < kWords; ++i) {
-            const bool in0 = have2 || 4 * i + 2 <= kBlockBytes, in1 = have2 || 4 * i + 4 <= kBlockBytes;
-            w[i] = (in0 ? static_cast<uint32_t>(__ldg(h + 2 * i)) : 0u) |
-                   (in1 ? static_cast<uint32_t>(__ldg(h + 2 * i + 1)) << 16 : 0u);
+          for (int k = 0; k < kWords; ++k) {
+            const uint32_t next = lds_u32(wa + 4 * (k + 1));
+            w[k] = __funnelshift_r(prev, next, 16);
+            prev = next;
           }
         }
+      } else if (have) {  // the last rows of W, short of a whole super-row: global loads
+        const uint16_t *hp = reinterpret_cast<const uint16_t *>(p.W + n * p.row_bytes + static_cast<int64_t>(kb) * kBlockBytes);
+#pragma unroll
+        for (int k = 0; k < kWords; ++k) {
+          const bool in0 = 4 * k + 2 <= kBlockBytes, in1 = 4 * k + 4 <= kBlockBytes;  // never past the block
+          w[k] = (in0 ? static_cast<uint32_t>(__ldg(hp + 2 * k)) : 0u) |
+                 (in1 ? static_cast<uint32_t>(__ldg(hp + 2 * k + 1)) << 16 : 0u);
+        }
       } else {
 #pragma unroll
-        for (int i = 0; i < kWords; ++i) w[i] = 0u;
+        for (int k = 0; k < kWords; ++k) w[k] = 0u;
       }
+      float d = half_bits_to_float(w[0]);
+      if (!have || *abort_flag) d = 0.f;
       if constexpr (WT == QMM_Q8_0) {
-        // block 0: d = bytes 0-1, qs at bytes 2..33; block 1: d = bytes 34-35, qs at 36..67
-        float d0 = half_bits_to_float(w[0]), d1 = half_bits_to_float(w[8] >> 16);
-        if (!row_ok) d0 = d1 = 0.f;
-        if (!have2) d1 = 0.f;
+        // codes at bytes 2..33 -> chunks 4h .. 4h+3 (this part: 4 / kParts of them); the
+        // words are picked by selects, never by a runtime register index
+        constexpr int kCw = 8 / kParts + 1;
+        uint32_t cw[kCw];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {  // block 0 -> chunks 0..3 (qs words unaligned by 2 bytes)
-          uint32_t o[4];
-          q8_word_bf16(__funnelshift_r(w[2 * c], w[2 * c + 1], 16), d0, o[0], o[1]);
-          q8_word_bf16(__funnelshift_r(w[2 * c + 1], w[2 * c + 2], 16), d0, o[2], o[3]);
-          st_a_chunk(a_base, r, c, o[0], o[1], o[2], o[3]);
-        }
+        for (int k = 0; k < kCw; ++k) cw[k] = (kParts == 2 && pt) ? w[4 + k] : w[k];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {  // block 1 -> chunks 4..7 (qs words aligned)
+        for (int c2 = 0; c2 < 4 / kParts; ++c2) {
           uint32_t o[4];
-          q8_word_bf16(w[9 + 2 * c], d1, o[0], o[1]);
-          q8_word_bf16(w[10 + 2 * c], d1, o[2], o[3]);
-          st_a_chunk(a_base, r, 4 + c, o[0], o[1], o[2], o[3]);
+          q8_word_bf16(__funnelshift_r(cw[2 * c2], cw[2 * c2 + 1], 16), d, o[0], o[1]);
+          q8_word_bf16(__funnelshift_r(cw[2 * c2 + 1], cw[2 * c2 + 2], 16), d, o[2], o[3]);
+          st_a_chunk(a_base, r, 4 * h + pt * (4 / kParts) + c2, o[0], o[1], o[2], o[3]);
         }
       } else {
-        // block 0: d = bytes 0-1, qs at 2..17; block 1: d = bytes 18-19, qs at 20..35
-        float d0 = half_bits_to_float(w[0]), d1 = half_bits_to_float(w[4] >> 16);
-        if (!row_ok) d0 = d1 = 0.f;
-        if (!have2) d1 = 0.f;
-        uint32_t qs0[4], qs1[4];
+        // nibbles at bytes 2..17: low nibbles = elements 0..15, high = 16..31 (this part: one or both)
+        uint32_t qs[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          qs0[i] = __funnelshift_r(w[i], w[i + 1], 16);
-          qs1[i] = w[5 + i];
-        }
+        for (int k = 0; k < 4; ++k) qs[k] = __funnelshift_r(w[k], w[k + 1], 16);
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          const uint32_t *qs = b ? qs1 : qs0;
-          const float d = b ? d1 : d0;
+        for (int h2 = 0; h2 < 2 / kParts; ++h2) {
+          const int half = pt * (2 / kParts) + h2;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {  // low nibbles: elements 0..15, high: 16..31
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const uint32_t v0 = half ? (qs[2 * c] >> 4) & 0x0F0F0F0Fu : qs[2 * c] & 0x0F0F0F0Fu;
-              const uint32_t v1 = half ? (qs[2 * c + 1] >> 4) & 0x0F0F0F0Fu : qs[2 * c + 1] & 0x0F0F0F0Fu;
-              uint32_t o[4];
-              q4_nib_bf16(v0, d, o[0], o[1]);
-              q4_nib_bf16(v1, d, o[2], o[3]);
-              st_a_chunk(a_base, r, b * 4 + half * 2 + c, o[0], o[1], o[2], o[3]);
-            }
+          for (int cc = 0; cc < 2; ++cc) {
+            const uint32_t v0 = half ? (qs[2 * cc] >> 4) & 0x0F0F0F0Fu : qs[2 * cc] & 0x0F0F0F0Fu;
+            const uint32_t v1 = half ? (qs[2 * cc + 1] >> 4) & 0x0F0F0F0Fu : qs[2 * cc + 1] & 0x0F0F0F0Fu;
+            uint32_t o[4];
+            q4_nib_bf16(v0, d, o[0], o[1]);
+            q4_nib_bf16(v1, d, o[2], o[3]);
+            st_a_chunk(a_base, r, 4 * h + 2 * half + cc, o[0], o[1], o[2], o[3]);
           }
         }
       }
@@ -345,24 +399,65 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&a_full[s]);
-        if (p.tma_w && (q == kRawBlocks / 2 - 1 || kb0 + 2 >= p.KB)) mbar_arrive(&raw_empty[raw % kRawStages]);
+        if (q == kRawBlocks / 2 - 1 || i == nst - 1) mbar_arrive(&raw_empty[c % kRawStages]);
       }
     }
+    wait(acc_full, 0);  // accumulator complete: every MMA (and so every stage buffer) is done
+  }
 
-    // ------------------------------------------------------------ epilogue
-    wait(acc_full, 0);
-    tc_fence_after();
-    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 belong to this warp
-    const int64_t row = n0 + 32 * quarter + lane;
-    for (int c0 = 0; c0 < p.MT; c0 += 32) {
-      uint32_t v[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(c0), v);
-      if (!*abort_flag && row < p.N) {
+  // ------------------------------------------------------------ epilogue
+  const bool epi = warp >= 2;
+  const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 belong to this warp
+  const int col0 = warp >= 2 ? 32 * ((warp - 2) >> 2) : 0;  // the warps of a quarter take turns at 32 columns
+  if (split == 1) {
+    if (epi) {
+      tc_fence_after();
+      const int64_t row = n0 + 32 * quarter + lane;
+      for (int c0 = col0; c0 < p.MT; c0 += 32 * (kDqWarps / 4)) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(c0), v);
+        if (!*abort_flag && row < p.N) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int m = m0 + c0 + c;
-          if (m < p.M) p.Y[static_cast<int64_t>(m) * p.N + row] = __uint_as_float(v[c]);
+          for (int c = 0; c < 32; ++c) {
+            const int m = m0 + c0 + c;
+            if (m < p.M) p.Y[static_cast<int64_t>(m) * p.N + row] = __uint_as_float(v[c]);
+          }
         }
+      }
+    }
+  } else {
+    // Split K: rank r owns weight rows [r*128/split, (r+1)*128/split) of the
+    // tile and receives every rank's partial of them in its stage buffers
+    // (free once all ranks' accumulators are complete: first cluster barrier).
+    const int rmax = (128 + split - 1) / split;
+    const uint32_t xbuf = sbase + p.off_x;  // [src rank][rmax rows][red_pitch floats]
+    cluster_sync_all();
+    if (epi) {
+      tc_fence_after();
+      const int row = 32 * quarter + lane;
+      const int dst = (row * split + split - 1) / 128;  // owner rank of this row
+      const int lr = row - dst * 128 / split;
+      const uint32_t raddr =
+          map_rank(xbuf + static_cast<uint32_t>(((zr * rmax + lr) * p.red_pitch) * 4), static_cast<uint32_t>(dst));
+      for (int c0 = col0; c0 < p.MT; c0 += 32 * (kDqWarps / 4)) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(c0), v);
+#pragma unroll
+        for (int c = 0; c < 32; c += 4)  // MT is a multiple of 16: the last load may hold 16 columns
+          if (c0 + c < p.MT) st_cluster_v4(raddr + 4u * (c0 + c), v[c], v[c + 1], v[c + 2], v[c + 3]);
+      }
+    }
+    cluster_sync_all();  // every partial has landed
+    const int rbase = zr * 128 / split, rown = (zr + 1) * 128 / split - rbase;
+    const float *buf = reinterpret_cast<const float *>(smem + p.off_x);
+    if (!*abort_flag) {
+      for (int e = tid; e < rown * p.MT; e += kThreads) {
+        const int col = e / rown, lr = e - col * rown;
+        const int m = m0 + col;
+        const int64_t row = n0 + rbase + lr;
+        float acc = 0.f;
+        for (int src = 0; src < split; ++src) acc += buf[(src * rmax + lr) * p.red_pitch + col];
+        if (m < p.M && row < p.N) p.Y[static_cast<int64_t>(m) * p.N + row] = acc;
       }
     }
   }
@@ -377,18 +472,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 }
 
 template <int WT>
-cudaError_t launch(const cudaLaunchConfig_t &cfg, const Params &p) {
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    int optin = 0;
-    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
-  return cudaLaunchKernelEx(&cfg, prefill_kernel<WT>, p);
+void *kernel_ptr() {
+  return reinterpret_cast<void *>(prefill_kernel<WT>);
 }
 
 int round_up(int v, int a) { return (v + a - 1) / a * a; }
@@ -406,12 +491,16 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
   p.N = N;
   const int bb = wtype == QMM_Q8_0 ? 34 : 18;
   p.row_bytes = static_cast<int64_t>(bb) * p.KB;
+  p.rs = 1;
+  while ((p.rs * p.row_bytes) % 16 != 0) p.rs *= 2;  // at most 8: 8 * 34 = 16 * 17, 8 * 18 = 16 * 9
+  p.tma_rows = N / p.rs * p.rs;
   p.MT = static_cast<int>(std::min<int64_t>(256, round_up(static_cast<int>(std::min<int64_t>(M, 256)), 16)));
   p.tmem_cols = p.MT <= 32 ? 32 : p.MT <= 64 ? 64 : p.MT <= 128 ? 128 : 256;
   p.x_stage_bytes = p.MT * 128;
-  p.tma_w = (p.row_bytes % 16 == 0) ? 1 : 0;
-  p.raw_pitch = kRawBlocks * bb;  // 272 (Q8) or 144 (Q4): box rows are dense
-  const int raw_bytes = p.tma_w ? kRawStages * 128 * p.raw_pitch : 0;
+  // a row's chunk plus up to 15 bytes of alignment in front, rounded to 16
+  // and then to 16 mod 32 (rows spread over eight 4-byte bank groups)
+  p.raw_pitch = wtype == QMM_Q8_0 ? 304 : 176;
+  const int raw_bytes = kRawStages * 128 * p.raw_pitch;
   const int per_stage = p.x_stage_bytes + kATileBytes;
   const int budget = dev.smem_optin - 1024 /*align*/ - 1024 /*barriers*/ - round_up(raw_bytes, 1024);
   p.stages = std::max(2, std::min(8, budget / per_stage));
@@ -427,27 +516,65 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
   const uint32_t xb[2] = {64, static_cast<uint32_t>(p.MT)};
   qmm_status st = encode_tiled(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, xd, xs, xb, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != QMM_OK) return st;
-  if (p.tma_w) {
-    const uint64_t wd[2] = {static_cast<uint64_t>(p.row_bytes / 2), static_cast<uint64_t>(N)};
-    const uint64_t ws[1] = {static_cast<uint64_t>(p.row_bytes)};
-    const uint32_t wb[2] = {static_cast<uint32_t>(p.raw_pitch / 2), 128};
-    st = encode_tiled(&p.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (st != QMM_OK) return st;
-  }
 
   const int64_t ntiles = (N + 127) / 128, mtiles = (M + p.MT - 1) / p.MT;
   if (ntiles > 0x7fffffff || mtiles > 65535) return set_error(QMM_ERR_SHAPE, "prefill: grid too large");
+  void *kern = wtype == QMM_Q8_0 ? kernel_ptr<QMM_Q8_0>() : kernel_ptr<QMM_Q4_0>();
+  static bool configured[2][64] = {};
+  if (dev.device >= 0 && dev.device < 64 && !configured[wtype][dev.device]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
+    if (e != cudaSuccess) return cuda_check(e, "prefill attribute");
+    configured[wtype][dev.device] = true;
+  }
+
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(ntiles), static_cast<unsigned>(mtiles));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cuda_check(wtype == QMM_Q8_0 ? launch<QMM_Q8_0>(cfg, p) : launch<QMM_Q4_0>(cfg, p), "prefill launch");
+
+  // Split K over a cluster when the output tiles leave SMs idle: as many
+  // ranks as fit one wave, each with at least one stage, the exchange buffer
+  // inside the stage buffers, and every cluster resident at once.
+  const int64_t base = ntiles * mtiles;
+  const int nst_all = (p.KB + 1) / 2;
+  int split = 1;
+  if (base < dev.sms) {
+    split = static_cast<int>(std::min<int64_t>({kMaxSplit, nst_all, dev.sms / base}));
+    for (; split > 1; --split) {
+      const int rmax = (128 + split - 1) / split;
+      if (static_cast<int64_t>(split) * rmax * (p.MT + 4) * 4 > static_cast<int64_t>(p.stages) * per_stage) continue;
+      cfg.gridDim = dim3(static_cast<unsigned>(ntiles), static_cast<unsigned>(mtiles), static_cast<unsigned>(split));
+      attr[1].val.clusterDim.x = 1;
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = static_cast<unsigned>(split);
+      cfg.numAttrs = 2;
+      int active = 0;
+      if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active >= base) break;
+      cudaGetLastError();  // a refused query is not an error of this call
+    }
+  }
+  p.split = split;
+  p.red_pitch = p.MT + 4;
+  if (p.rs == 1 && split == 1) p.raw_pitch = kRawBlocks * bb;  // chunks start on 16-byte boundaries: 272 / 144
+  if (p.tma_rows > 0) {
+    const uint64_t wd[2] = {static_cast<uint64_t>(p.rs * p.row_bytes / 2), static_cast<uint64_t>(N / p.rs)};
+    const uint64_t ws[1] = {static_cast<uint64_t>(p.rs * p.row_bytes)};
+    const uint32_t wb[2] = {static_cast<uint32_t>(p.raw_pitch / 2), static_cast<uint32_t>(128 / p.rs)};
+    st = encode_tiled(&p.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != QMM_OK) return st;
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(ntiles), static_cast<unsigned>(mtiles), static_cast<unsigned>(split));
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = static_cast<unsigned>(split);
+  cfg.numAttrs = split > 1 ? 2 : 1;
+  void *args[] = {&p};
+  return cuda_check(cudaLaunchKernelExC(&cfg, kern, args), "prefill launch");
 }
 
 cudaError_t prefill_status(uint32_t *bits) {

@@ -22,6 +22,7 @@ def run(wtype, m, n, k, seed, window_rows=None):
     xb = syn.act_bf16_bits(g, m, k)
     Y = qmm.qmm_quant_matmul_prefill(wtype, dev(W), dev(xb), n)
     torch.cuda.synchronize()
+    assert qmm.device_status() == 0
     y = host(Y)
     return W, xb, y
 
@@ -38,13 +39,15 @@ def check_full(wtype, m, n, k, seed):
 @pytest.mark.parametrize("wtype", [syn.Q8_0, syn.Q4_0])
 @pytest.mark.parametrize("m,n,k", [(16, 128, 256), (32, 256, 512), (7, 130, 256), (100, 200, 1024), (1, 1, 256),
                                    (300, 129, 768)])
-def test_prefill_tma_weight_path(wtype, m, n, k):
+def test_prefill_rows_16_byte_multiple(wtype, m, n, k):
+    # row pitch a multiple of 16 bytes (K % 256 == 0); small shapes split K over a cluster
     check_full(wtype, m, n, k, seed=m + n + k)
 
 
 @pytest.mark.parametrize("wtype", [syn.Q8_0, syn.Q4_0])
 @pytest.mark.parametrize("m,n,k", [(32, 128, 896), (16, 77, 96), (5, 3, 32), (64, 257, 160)])
-def test_prefill_direct_weight_path(wtype, m, n, k):
+def test_prefill_rows_not_16_byte_multiple(wtype, m, n, k):
+    # widened per-row bulk copies; (64, 257, 160) splits three stages over three ranks
     check_full(wtype, m, n, k, seed=3 * m + n + k)
 
 
@@ -74,3 +77,22 @@ def test_prefill_q8_panels_full_size(m, n, k):
 
 def test_prefill_q4_m1024_k5120_n17408():
     check_sampled(syn.Q4_0, 1024, 17408, 5120, seed=11, n_samples=64)
+
+
+@pytest.mark.parametrize("wtype", [syn.Q8_0, syn.Q4_0])
+@pytest.mark.parametrize("m,n,k", [(48, 300, 4864), (40, 1000, 2048), (200, 129, 1312), (17, 5, 7200)])
+def test_prefill_split_k(wtype, m, n, k):
+    # few output tiles, long K: the K range is split across a thread-block cluster
+    check_full(wtype, m, n, k, seed=5 * m + n + k)
+
+
+def test_prefill_split_k_deterministic():
+    g = syn.rng(9)
+    n, k, m = 896, 4864, 32
+    W = dev(syn.weights(g, syn.Q8_0, n, k))
+    xb = dev(syn.act_bf16_bits(g, m, k))
+    a = qmm.qmm_quant_matmul_prefill(syn.Q8_0, W, xb, n)
+    b = qmm.qmm_quant_matmul_prefill(syn.Q8_0, W, xb, n)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert qmm.device_status() == 0
