@@ -12,10 +12,15 @@
 //  * MMA shape M = 128 weight rows, N = MT tokens, K = 16 (kind::f16, bf16
 //    inputs, fp32 accumulator in TMEM, one thread issues, cta_group::1). The
 //    accumulator D[n][m] lives in MT TMEM columns x 128 lanes.
-//  * A (weights, 128 x 64 per stage) is written by eight "dequant" warps in
-//    the canonical K-major 128-byte-swizzled layout (8-row atoms of 1 KB,
-//    16-byte chunk c of row r at c ^ (r % 8)); B (X, MT x 64 per stage) comes
-//    straight from a 2-D TMA load with the same 128-byte swizzle.
+//  * A (weights, 128 x 64 per stage) never touches shared memory: eight
+//    "dequant" warps write each decoded row into tensor memory (tcgen05.st,
+//    lane = weight row, two bf16 per 32-bit column; a ring of 32-column stages
+//    beside the accumulator) and the MMA takes A from there. Shared memory
+//    then carries only X and the raw blocks, which is what let the pipeline
+//    keep up: with A in shared memory the operand reads, TMA writes and
+//    dequant stores of one stage exceeded the SM's shared-memory bandwidth.
+//    B (X, MT x 64 per stage) comes from a 2-D TMA load with the 128-byte
+//    swizzle.
 //  * Raw weight blocks arrive in 8-block (256 k) chunks per 128-row tile by
 //    2-D TMA. A Q8_0 row is 34 * K/32 bytes, in general not a multiple of 16
 //    (a TMA row pitch must be), so W is viewed as super-rows of rs = 1, 2, 4
@@ -47,12 +52,12 @@ namespace {
 
 static __device__ uint32_t g_prefill_status;
 
-constexpr int kDqWarps = 8;            // dequant (then epilogue) warps: thread = (weight row, block of the stage, part)
-constexpr int kParts = kDqWarps / 8;    // parts of a block per thread: 32 / kParts weights each
+constexpr int kDqWarps = 8;            // dequant (then epilogue) warps: thread = (weight row, block of the stage)
 constexpr int kThreads = 64 + 32 * kDqWarps;  // warp 0 producer, warp 1 MMA, warps 2.. dequant + epilogue
 constexpr int kRawBlocks = 8;          // blocks per raw weight chunk
 constexpr int kStageK = 64;            // k per MMA stage (one 128-byte swizzle row of bf16)
-constexpr int kATileBytes = 128 * 128; // 128 rows x 64 bf16
+constexpr int kAccCols = 256;          // TMEM columns 0..255: the fp32 accumulator (MT <= 256)
+constexpr int kACols = 32;             // TMEM columns per A stage: 128 rows x 64 bf16 (two per 32-bit cell)
 constexpr int kRawStages = 2;
 constexpr int kMaxSplit = 8;           // portable cluster size
 
@@ -71,7 +76,7 @@ struct alignas(64) Params {
   int stages;          // MMA stages in flight
   int raw_pitch;       // bytes per row of a raw chunk in shared memory (a chunk + up to 15 bytes in front)
   int x_stage_bytes;
-  int off_x, off_a, off_raw;  // shared-memory offsets (1024-aligned)
+  int off_x, off_raw;  // shared-memory offsets (1024-aligned)
   int split;           // K ranges per output tile (cluster size along z)
   int red_pitch;       // floats per row of the split-K exchange buffer (MT + 4)
 };
@@ -99,6 +104,26 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc ? 1u : 0u)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem]^T: A is 128 lanes (rows) x K packed two
+// bf16 per 32-bit column, B K-major in shared memory.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, bool acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc ? 1u : 0u)
+      : "memory");
+}
+// Each thread of the warp writes 16 consecutive 32-bit columns of its own lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // Arrive once on `bar` when all previously issued tcgen05.mma of this thread complete.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -180,14 +205,6 @@ __device__ __forceinline__ void q4_nib_bf16(uint32_t v, float d, uint32_t &o01, 
   f23 = __fmul2_rn(__fadd2_rn(f23, nb), dd);
   o01 = bf16x2(f01.x, f01.y);
   o23 = bf16x2(f23.x, f23.y);
-}
-
-// Store 16-byte chunk c (bf16 elements 8c..8c+7) of A-tile row r, swizzled.
-__device__ __forceinline__ void st_a_chunk(uint32_t a_base, int r, int c, uint32_t w0, uint32_t w1, uint32_t w2,
-                                           uint32_t w3) {
-  const uint32_t addr = a_base + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4);
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1), "r"(w2), "r"(w3)
-               : "memory");
 }
 
 template <int WT>
@@ -272,19 +289,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         mbar_arrive(&raw_full[slot]);  // every row of this tile is read directly
       }
     };
+    // Two independent streams, so that neither waits behind the other's ring:
+    // lane 0 feeds the X stages, lane 1 the raw chunks.
     if (lane == 0) {
-      int raw_issued = 0;
       for (int i = 0; i < nst; ++i) {
         const int s = i % S;
-        // keep the raw chunk feeding this stage and the next one in flight
-        const int need = min(nraw, i / (kRawBlocks / 2) + 2);
-        while (raw_issued < need) issue_raw(raw_issued++);
         if (i >= S) wait(&st_empty[s], static_cast<uint32_t>(i / S - 1) & 1u);
         if (!*abort_flag) {
           mbar_arrive_expect_tx(&x_full[s], static_cast<uint32_t>(p.x_stage_bytes));
           tma_load_2d(smem + p.off_x + s * p.x_stage_bytes, &p.tm_x, (j_lo + i) * kStageK, m0, &x_full[s]);
         }
       }
+    } else if (lane == 1) {
+      for (int c = 0; c < nraw; ++c) issue_raw(c);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -298,12 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         wait(&a_full[s], ph);
         tc_fence_after();
         if (!*abort_flag) {
-          const uint32_t a_addr = sbase + p.off_a + s * kATileBytes;
+          const uint32_t a_tmem = tmem + static_cast<uint32_t>(kAccCols + s * kACols);
           const uint32_t b_addr = sbase + p.off_x + s * p.x_stage_bytes;
 #pragma unroll
           for (int kk = 0; kk < kStageK / 16; ++kk)
-            umma_f16(tmem, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk), idesc,
-                     i > 0 || kk > 0);
+            umma_f16_ts(tmem, a_tmem + 8 * kk, sw128_kmajor_desc(b_addr + 32 * kk), idesc, i > 0 || kk > 0);
         }
         umma_commit(&st_empty[s]);  // frees this stage's A and X buffers when the MMAs finish
       }
@@ -312,11 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------------ dequant warps
-    // thread (r, h, pt): weight row n0 + r, block h of each stage's two blocks, part pt of the block
-    const int r = (tid - 64) & 127, h = ((tid - 64) >> 7) & 1, pt = (tid - 64) >> 8;
+    // thread (r, h): weight row n0 + r, block h of each stage's two blocks. A
+    // warp may only reach its own quarter of the TMEM lanes, so warp w takes
+    // rows 32 (w % 4) .. +31; lane = row.
+    const int quarter = warp & 3;
+    const int r = 32 * quarter + lane, h = (warp - 2) >> 2;
     const int64_t n = n0 + r;
     const bool row_ok = n < p.N;
-    const uint32_t a_base0 = sbase + p.off_a;
+    const uint32_t a_lane = tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(kAccCols + 16 * h);
     constexpr int kWords = (kBlockBytes + 2 + 3) / 4;  // the block as words, plus the 16-bit shift (Q8: 9, Q4: 5)
     for (int i = 0; i < nst; ++i) {
       const int s = i % S;
@@ -324,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       const int kb = 2 * (j_lo + i) + h;  // this thread's block
       if (q == 0) wait(&raw_full[c % kRawStages], static_cast<uint32_t>(c / kRawStages) & 1u);
       if (i >= S) wait(&st_empty[s], static_cast<uint32_t>(i / S - 1) & 1u);
-      const uint32_t a_base = a_base0 + s * kATileBytes;
+      tc_fence_after();  // the MMAs that read this stage's A columns are complete
       const bool have = row_ok && kb < p.KB;
       // w: the block's bytes from its fp16 scale on, as little-endian words
       uint32_t w[kWords];
@@ -362,40 +381,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       }
       float d = half_bits_to_float(w[0]);
       if (!have || *abort_flag) d = 0.f;
+      uint32_t o[16];  // bf16 pairs of the block's 32 weights, in k order
       if constexpr (WT == QMM_Q8_0) {
-        // codes at bytes 2..33 -> chunks 4h .. 4h+3 (this part: 4 / kParts of them); the
-        // words are picked by selects, never by a runtime register index
-        constexpr int kCw = 8 / kParts + 1;
-        uint32_t cw[kCw];
 #pragma unroll
-        for (int k = 0; k < kCw; ++k) cw[k] = (kParts == 2 && pt) ? w[4 + k] : w[k];
-#pragma unroll
-        for (int c2 = 0; c2 < 4 / kParts; ++c2) {
-          uint32_t o[4];
-          q8_word_bf16(__funnelshift_r(cw[2 * c2], cw[2 * c2 + 1], 16), d, o[0], o[1]);
-          q8_word_bf16(__funnelshift_r(cw[2 * c2 + 1], cw[2 * c2 + 2], 16), d, o[2], o[3]);
-          st_a_chunk(a_base, r, 4 * h + pt * (4 / kParts) + c2, o[0], o[1], o[2], o[3]);
-        }
+        for (int cc = 0; cc < 8; ++cc)  // codes at bytes 2..33
+          q8_word_bf16(__funnelshift_r(w[cc], w[cc + 1], 16), d, o[2 * cc], o[2 * cc + 1]);
       } else {
-        // nibbles at bytes 2..17: low nibbles = elements 0..15, high = 16..31 (this part: one or both)
-        uint32_t qs[4];
+        // nibbles at bytes 2..17: low nibbles = elements 0..15, high = 16..31
 #pragma unroll
-        for (int k = 0; k < 4; ++k) qs[k] = __funnelshift_r(w[k], w[k + 1], 16);
-#pragma unroll
-        for (int h2 = 0; h2 < 2 / kParts; ++h2) {
-          const int half = pt * (2 / kParts) + h2;
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const uint32_t v0 = half ? (qs[2 * cc] >> 4) & 0x0F0F0F0Fu : qs[2 * cc] & 0x0F0F0F0Fu;
-            const uint32_t v1 = half ? (qs[2 * cc + 1] >> 4) & 0x0F0F0F0Fu : qs[2 * cc + 1] & 0x0F0F0F0Fu;
-            uint32_t o[4];
-            q4_nib_bf16(v0, d, o[0], o[1]);
-            q4_nib_bf16(v1, d, o[2], o[3]);
-            st_a_chunk(a_base, r, 4 * h + 2 * half + cc, o[0], o[1], o[2], o[3]);
-          }
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t qs = __funnelshift_r(w[k], w[k + 1], 16);
+          q4_nib_bf16(qs & 0x0F0F0F0Fu, d, o[2 * k], o[2 * k + 1]);
+          q4_nib_bf16((qs >> 4) & 0x0F0F0F0Fu, d, o[8 + 2 * k], o[9 + 2 * k]);
         }
       }
-      fence_proxy_async_smem();
+      tmem_st16(a_lane + static_cast<uint32_t>(s * kACols), o);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&a_full[s]);
@@ -427,8 +429,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     }
   } else {
     // Split K: rank r owns weight rows [r*128/split, (r+1)*128/split) of the
-    // tile and receives every rank's partial of them in its stage buffers
-    // (free once all ranks' accumulators are complete: first cluster barrier).
+    // tile and receives every rank's partial of them in its X stage and raw
+    // chunk buffers (free once all ranks' accumulators are complete: first
+    // cluster barrier).
     const int rmax = (128 + split - 1) / split;
     const uint32_t xbuf = sbase + p.off_x;  // [src rank][rmax rows][red_pitch floats]
     cluster_sync_all();
@@ -495,19 +498,22 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
   while ((p.rs * p.row_bytes) % 16 != 0) p.rs *= 2;  // at most 8: 8 * 34 = 16 * 17, 8 * 18 = 16 * 9
   p.tma_rows = N / p.rs * p.rs;
   p.MT = static_cast<int>(std::min<int64_t>(256, round_up(static_cast<int>(std::min<int64_t>(M, 256)), 16)));
-  p.tmem_cols = p.MT <= 32 ? 32 : p.MT <= 64 ? 64 : p.MT <= 128 ? 128 : 256;
+  p.tmem_cols = 512;  // accumulator in columns 0..MT-1, A stage s at 256 + 32 s
   p.x_stage_bytes = p.MT * 128;
   // a row's chunk plus up to 15 bytes of alignment in front, rounded to 16
   // and then to 16 mod 32 (rows spread over eight 4-byte bank groups)
   p.raw_pitch = wtype == QMM_Q8_0 ? 304 : 176;
   const int raw_bytes = kRawStages * 128 * p.raw_pitch;
-  const int per_stage = p.x_stage_bytes + kATileBytes;
+  const int per_stage = p.x_stage_bytes;  // A lives in tensor memory
   const int budget = dev.smem_optin - 1024 /*align*/ - 1024 /*barriers*/ - round_up(raw_bytes, 1024);
   p.stages = std::max(2, std::min(8, budget / per_stage));
   p.off_x = 1024;
-  p.off_a = p.off_x + p.stages * p.x_stage_bytes;
-  p.off_raw = p.off_a + p.stages * kATileBytes;
-  const size_t smem = static_cast<size_t>(p.off_raw) + raw_bytes + 1024;
+  p.off_raw = p.off_x + p.stages * p.x_stage_bytes;
+  // Every CTA allocates all 512 TMEM columns, so never two CTAs on one SM (a
+  // second one would wait in tcgen05.alloc, and across clusters that wait
+  // could close a cycle): ask for more than half of the shared memory.
+  const size_t smem = std::max<size_t>(static_cast<size_t>(p.off_raw) + raw_bytes + 1024,
+                                       static_cast<size_t>(dev.smem_optin / 2 + 1024));
   if (smem > static_cast<size_t>(dev.smem_optin))
     return set_error(QMM_ERR_SHAPE, "prefill: tile needs %zu bytes of shared memory", smem);
 
@@ -547,7 +553,8 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
     split = static_cast<int>(std::min<int64_t>({kMaxSplit, nst_all, dev.sms / base}));
     for (; split > 1; --split) {
       const int rmax = (128 + split - 1) / split;
-      if (static_cast<int64_t>(split) * rmax * (p.MT + 4) * 4 > static_cast<int64_t>(p.stages) * per_stage) continue;
+      // the exchange buffer reuses the X stages and the raw chunks (all consumed by then)
+      if (static_cast<int64_t>(split) * rmax * (p.MT + 4) * 4 > p.off_raw + raw_bytes - p.off_x) continue;
       cfg.gridDim = dim3(static_cast<unsigned>(ntiles), static_cast<unsigned>(mtiles), static_cast<unsigned>(split));
       attr[1].val.clusterDim.x = 1;
       attr[1].val.clusterDim.y = 1;
