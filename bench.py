@@ -319,6 +319,61 @@ def component_gateup(qmm, dev_peak_gbs, m=8, n=17408, k=5120, reps=10):
     return out
 
 
+def component_q8q8(qmm, dev_peak_gbs, reps_graph=4):
+    """Q8xQ8 decode GEMV (M=1) at K=896/N=4864 and K=4864/N=896: the GEMV on
+    quantized activations alone, activation quantization + GEMV, and the fp32
+    activation GEMV of the same shape for comparison; rotating weight copies
+    (> 2x L2) in one CUDA graph."""
+    import torch
+
+    props = torch.cuda.get_device_properties(0)
+    l2 = getattr(props, "L2_cache_size", 126 * 2**20)
+    out = {}
+    for n, k in ((4864, 896), (896, 4864)):
+        wbytes = n * (k // 32) * 34
+        copies = max(8, int(2.2 * l2 // wbytes) + 1)
+        g = syn.rng(2)
+        W0 = torch.from_numpy(syn.q8_0_weights(g, n, k)[0]).cuda()
+        Ws = [W0.clone() for _ in range(copies)]
+        x = torch.from_numpy(syn.act_f32(g, 1, k)).cuda()
+        qx = torch.empty(k, dtype=torch.int8, device="cuda")
+        dx = torch.empty(k // 32, device="cuda")
+        Y = torch.empty(n, device="cuda")
+        s = torch.cuda.Stream()
+        lib = qmm.lib
+        fl = qmm.QMM_FLAG_EARLY_WEIGHTS
+
+        def gemv_q8(h):
+            for w in Ws:
+                assert lib.qmm_q8q8_gemv_ex(1, n, k, 32, w.data_ptr(), qx.data_ptr(), dx.data_ptr(), Y.data_ptr(), fl, h) == 0
+
+        def quant_gemv(h):
+            for w in Ws:
+                assert lib.qmm_quantize_act_q8(1, k, 32, x.data_ptr(), qx.data_ptr(), dx.data_ptr(), h) == 0
+                assert lib.qmm_q8q8_gemv_ex(1, n, k, 32, w.data_ptr(), qx.data_ptr(), dx.data_ptr(), Y.data_ptr(), fl, h) == 0
+
+        def gemv_f32(h):
+            for w in Ws:
+                assert lib.qmm_q8_gemv_ex(1, n, k, 32, w.data_ptr(), x.data_ptr(), Y.data_ptr(), fl, h) == 0
+
+        res = {}
+        for name, fn, extra in (("q8q8_gemv", gemv_q8, k + (k // 32) * 4),
+                                ("quantize_plus_q8q8_gemv", quant_gemv, k * 4),
+                                ("f32_gemv_same_shape", gemv_f32, k * 4)):
+            fn(s.cuda_stream)
+            torch.cuda.synchronize()
+            gr = capture(fn, s)
+            time_graph(gr, s, 2)
+            ms = time_graph(gr, s, reps_graph) / copies
+            bytes_ = wbytes + extra + n * 4
+            res[name] = {"us": round(ms * 1e3, 3), "GB_s": round(bytes_ / ms / 1e6, 1),
+                         "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4)}
+            del gr
+        res["note"] = f"{copies} rotating weight copies; per-call times in a chain of stream-ordered launches"
+        out[f"k{k}_n{n}"] = res
+    return out
+
+
 def component_prefill(qmm, pk, reps=10):
     """Prefill panels on the tensor cores: TFLOP/s per shape (rotating weight copies
     > L2 where the weights are small; activations bf16 N(0,1))."""
@@ -633,6 +688,7 @@ def main(argv=None):
         components = {"lm_head_896x151936": component_lm_head(qmm, step, pk["hbm_gbs"]),
                       "single_gemv_896x1152": component_single_gemv(qmm, pk["hbm_gbs"]),
                       "q4_gateup_m8_k5120_n17408": component_gateup(qmm, pk["hbm_gbs"]),
+                      "q8q8_gemv": component_q8q8(qmm, pk["hbm_gbs"]),
                       "prefill": component_prefill(qmm, pk)}
 
     cpu = None
