@@ -58,7 +58,7 @@ constexpr int kRawBlocks = 8;          // blocks per raw weight chunk
 constexpr int kStageK = 64;            // k per MMA stage (one 128-byte swizzle row of bf16)
 constexpr int kAccCols = 256;          // TMEM columns 0..255: the fp32 accumulator (MT <= 256)
 constexpr int kACols = 32;             // TMEM columns per A stage: 128 rows x 64 bf16 (two per 32-bit cell)
-constexpr int kRawStages = 2;
+constexpr int kRawStages = 4;          // raw chunks in flight: three chunks (12 stages) of lead
 constexpr int kMaxSplit = 8;           // portable cluster size
 
 struct alignas(64) Params {
@@ -211,13 +211,13 @@ template <int WT>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // barriers: x_full[8], a_full[8], st_empty[8], raw_full[2], raw_empty[2], acc_full, tmem slot
+  // barriers: x_full[8], a_full[8], st_empty[8], raw_full[kRawStages], raw_empty[kRawStages], acc_full, tmem slot
   uint64_t *x_full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *a_full = x_full + 8;
   uint64_t *st_empty = a_full + 8;
   uint64_t *raw_full = st_empty + 8;
-  uint64_t *raw_empty = raw_full + 2;
-  uint64_t *acc_full = raw_empty + 2;
+  uint64_t *raw_empty = raw_full + kRawStages;
+  uint64_t *acc_full = raw_empty + kRawStages;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
   volatile uint32_t *abort_flag = tmem_slot + 1;
 
@@ -229,8 +229,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   const int j_lo = zr * nst_all / split, j_hi = (zr + 1) * nst_all / split;
   const int nst = j_hi - j_lo;                              // this CTA's stages
   const int nraw = (nst + kRawBlocks / 2 - 1) / (kRawBlocks / 2);  // raw chunks (four stages each)
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;
-  const int m0 = blockIdx.y * p.MT;
+  // token tiles vary fastest, so the CTAs sharing a weight tile run together
+  // and all but the first read its blocks from L2
+  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 128;
+  const int m0 = blockIdx.x * p.MT;
   constexpr int kBlockBytes = (WT == QMM_Q8_0) ? 34 : 18;
 
   pdl_launch_dependents();
@@ -292,12 +294,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // Two independent streams, so that neither waits behind the other's ring:
     // lane 0 feeds the X stages, lane 1 the raw chunks.
     if (lane == 0) {
-      for (int i = 0; i < nst; ++i) {
-        const int s = i % S;
-        if (i >= S) wait(&st_empty[s], static_cast<uint32_t>(i / S - 1) & 1u);
+      // stage slot and ring pass kept incrementally: a runtime division per
+      // stage costs the serial issuers hundreds of cycles
+      for (int i = 0, s = 0, pass = 0; i < nst; ++i) {
+        if (pass > 0) wait(&st_empty[s], static_cast<uint32_t>(pass - 1) & 1u);
         if (!*abort_flag) {
           mbar_arrive_expect_tx(&x_full[s], static_cast<uint32_t>(p.x_stage_bytes));
           tma_load_2d(smem + p.off_x + s * p.x_stage_bytes, &p.tm_x, (j_lo + i) * kStageK, m0, &x_full[s]);
+        }
+        if (++s == S) {
+          s = 0;
+          ++pass;
         }
       }
     } else if (lane == 1) {
@@ -308,9 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(p.MT);
-      for (int i = 0; i < nst; ++i) {
-        const int s = i % S;
-        const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
+      for (int i = 0, s = 0, pass = 0; i < nst; ++i) {
+        const uint32_t ph = static_cast<uint32_t>(pass) & 1u;
         wait(&x_full[s], ph);
         wait(&a_full[s], ph);
         tc_fence_after();
@@ -322,6 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             umma_f16_ts(tmem, a_tmem + 8 * kk, sw128_kmajor_desc(b_addr + 32 * kk), idesc, i > 0 || kk > 0);
         }
         umma_commit(&st_empty[s]);  // frees this stage's A and X buffers when the MMAs finish
+        if (++s == S) {
+          s = 0;
+          ++pass;
+        }
       }
       umma_commit(acc_full);        // accumulator complete
     }
@@ -337,12 +347,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const bool row_ok = n < p.N;
     const uint32_t a_lane = tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(kAccCols + 16 * h);
     constexpr int kWords = (kBlockBytes + 2 + 3) / 4;  // the block as words, plus the 16-bit shift (Q8: 9, Q4: 5)
-    for (int i = 0; i < nst; ++i) {
-      const int s = i % S;
+    for (int i = 0, s = 0, pass = 0; i < nst; ++i, (++s == S) ? (s = 0, ++pass) : 0) {
       const int c = i / (kRawBlocks / 2), q = i % (kRawBlocks / 2);
       const int kb = 2 * (j_lo + i) + h;  // this thread's block
       if (q == 0) wait(&raw_full[c % kRawStages], static_cast<uint32_t>(c / kRawStages) & 1u);
-      if (i >= S) wait(&st_empty[s], static_cast<uint32_t>(i / S - 1) & 1u);
+      if (pass > 0) wait(&st_empty[s], static_cast<uint32_t>(pass - 1) & 1u);
       tc_fence_after();  // the MMAs that read this stage's A columns are complete
       const bool have = row_ok && kb < p.KB;
       // w: the block's bytes from its fp16 scale on, as little-endian words
@@ -524,7 +533,7 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
   if (st != QMM_OK) return st;
 
   const int64_t ntiles = (N + 127) / 128, mtiles = (M + p.MT - 1) / p.MT;
-  if (ntiles > 0x7fffffff || mtiles > 65535) return set_error(QMM_ERR_SHAPE, "prefill: grid too large");
+  if (ntiles > 65535 || mtiles > 0x7fffffff) return set_error(QMM_ERR_SHAPE, "prefill: grid too large");
   void *kern = wtype == QMM_Q8_0 ? kernel_ptr<QMM_Q8_0>() : kernel_ptr<QMM_Q4_0>();
   static bool configured[2][64] = {};
   if (dev.device >= 0 && dev.device < 64 && !configured[wtype][dev.device]) {
@@ -555,7 +564,7 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
       const int rmax = (128 + split - 1) / split;
       // the exchange buffer reuses the X stages and the raw chunks (all consumed by then)
       if (static_cast<int64_t>(split) * rmax * (p.MT + 4) * 4 > p.off_raw + raw_bytes - p.off_x) continue;
-      cfg.gridDim = dim3(static_cast<unsigned>(ntiles), static_cast<unsigned>(mtiles), static_cast<unsigned>(split));
+      cfg.gridDim = dim3(static_cast<unsigned>(mtiles), static_cast<unsigned>(ntiles), static_cast<unsigned>(split));
       attr[1].val.clusterDim.x = 1;
       attr[1].val.clusterDim.y = 1;
       attr[1].val.clusterDim.z = static_cast<unsigned>(split);
@@ -575,7 +584,7 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
     st = encode_tiled(&p.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != QMM_OK) return st;
   }
-  cfg.gridDim = dim3(static_cast<unsigned>(ntiles), static_cast<unsigned>(mtiles), static_cast<unsigned>(split));
+  cfg.gridDim = dim3(static_cast<unsigned>(mtiles), static_cast<unsigned>(ntiles), static_cast<unsigned>(split));
   attr[1].val.clusterDim.x = 1;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = static_cast<unsigned>(split);
