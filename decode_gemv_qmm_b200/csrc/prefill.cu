@@ -12,8 +12,10 @@
 //  * MMA shape M = 128 weight rows, N = MT tokens, K = 16 (kind::f16, bf16
 //    inputs, fp32 accumulator in TMEM, one thread issues, cta_group::1). The
 //    accumulator D[n][m] lives in MT TMEM columns x 128 lanes.
-//  * A (weights, 128 x 64 per stage) never touches shared memory: eight
-//    "dequant" warps write each decoded row into tensor memory (tcgen05.st,
+//  * A (weights, 128 x 64 per stage) never touches shared memory: sixteen
+//    "dequant" warps in two groups that take alternate stages (each warp has
+//    two stages of MMA time per stage it converts) write each decoded row
+//    into tensor memory (tcgen05.st,
 //    lane = weight row, two bf16 per 32-bit column; a ring of 32-column stages
 //    beside the accumulator) and the MMA takes A from there. Shared memory
 //    then carries only X and the raw blocks, which is what let the pipeline
@@ -35,8 +37,12 @@
 //    partials of its 128/S weight rows, then sums them in rank order and
 //    writes Y: deterministic, and no global scratch memory.
 //  * Pipelines: producer -> (X tile, raw chunk) -> dequant -> A tile -> MMA
-//    -> tcgen05.commit frees the stage. After the last MMA a commit signals
-//    the eight dequant warps, which become the epilogue: tcgen05.ld 32 columns
+//    -> tcgen05.commit frees the stage. One barrier per stage tells the MMA
+//    issuer that both its X tile and its A columns are ready; the issuer
+//    keeps slots and ring passes incrementally and offsets precomputed
+//    descriptors (it is a single thread: every cycle there shows up as an
+//    idle tensor pipe). After the last MMA a commit signals the dequant
+//    warps, which become the epilogue: tcgen05.ld 32 columns
 //    at a time (lane = weight row) and coalesced stores of Y (or the scatter).
 //  * Every mbarrier wait is bounded; on a timeout the kernel records a status
 //    bit, finishes without waiting further (still meeting both cluster
@@ -52,7 +58,8 @@ namespace {
 
 static __device__ uint32_t g_prefill_status;
 
-constexpr int kDqWarps = 8;            // dequant (then epilogue) warps: thread = (weight row, block of the stage)
+constexpr int kDqGroups = 2;           // dequant groups; group g converts the stages i = g (mod kDqGroups)
+constexpr int kDqWarps = 8 * kDqGroups; // dequant (then epilogue) warps: thread = (weight row, block of the stage)
 constexpr int kThreads = 64 + 32 * kDqWarps;  // warp 0 producer, warp 1 MMA, warps 2.. dequant + epilogue
 constexpr int kRawBlocks = 8;          // blocks per raw weight chunk
 constexpr int kStageK = 64;            // k per MMA stage (one 128-byte swizzle row of bf16)
@@ -211,10 +218,11 @@ template <int WT>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // barriers: x_full[8], a_full[8], st_empty[8], raw_full[kRawStages], raw_empty[kRawStages], acc_full, tmem slot
-  uint64_t *x_full = reinterpret_cast<uint64_t *>(smem);
-  uint64_t *a_full = x_full + 8;
-  uint64_t *st_empty = a_full + 8;
+  // barriers: full[8], st_empty[8], raw_full[kRawStages], raw_empty[kRawStages], acc_full, tmem slot.
+  // full[s]: the stage's X tile has landed (producer arrival + TMA bytes) and
+  // all dequant warps have written its A columns -- one wait for the issuer.
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *st_empty = full + 8;
   uint64_t *raw_full = st_empty + 8;
   uint64_t *raw_empty = raw_full + kRawStages;
   uint64_t *acc_full = raw_empty + kRawStages;
@@ -238,13 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   pdl_launch_dependents();
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&x_full[s], 1);
-      mbar_init(&a_full[s], kDqWarps);
+      mbar_init(&full[s], 1 + 8);  // the producer, and the eight warps of the group that converts stage s
       mbar_init(&st_empty[s], 1);
     }
     for (int r = 0; r < kRawStages; ++r) {
       mbar_init(&raw_full[r], 1);
-      mbar_init(&raw_empty[r], kDqWarps);
+      mbar_init(&raw_empty[r], kDqWarps);  // every dequant warp, after its last stage of the chunk
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -299,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       for (int i = 0, s = 0, pass = 0; i < nst; ++i) {
         if (pass > 0) wait(&st_empty[s], static_cast<uint32_t>(pass - 1) & 1u);
         if (!*abort_flag) {
-          mbar_arrive_expect_tx(&x_full[s], static_cast<uint32_t>(p.x_stage_bytes));
-          tma_load_2d(smem + p.off_x + s * p.x_stage_bytes, &p.tm_x, (j_lo + i) * kStageK, m0, &x_full[s]);
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.x_stage_bytes));
+          tma_load_2d(smem + p.off_x + s * p.x_stage_bytes, &p.tm_x, (j_lo + i) * kStageK, m0, &full[s]);
         }
         if (++s == S) {
           s = 0;
@@ -315,18 +322,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(p.MT);
+      // descriptors of stage 0; a stage / k step is an offset in 16-byte units
+      // of the descriptor's address field (shared-memory addresses < 256 KB)
+      const uint64_t bdesc0 = sw128_kmajor_desc(sbase + p.off_x);
+      const uint32_t xs16 = static_cast<uint32_t>(p.x_stage_bytes) >> 4;
       for (int i = 0, s = 0, pass = 0; i < nst; ++i) {
-        const uint32_t ph = static_cast<uint32_t>(pass) & 1u;
-        wait(&x_full[s], ph);
-        wait(&a_full[s], ph);
+        wait(&full[s], static_cast<uint32_t>(pass) & 1u);  // after a timeout: garbage in, discarded
         tc_fence_after();
-        if (!*abort_flag) {
-          const uint32_t a_tmem = tmem + static_cast<uint32_t>(kAccCols + s * kACols);
-          const uint32_t b_addr = sbase + p.off_x + s * p.x_stage_bytes;
-#pragma unroll
-          for (int kk = 0; kk < kStageK / 16; ++kk)
-            umma_f16_ts(tmem, a_tmem + 8 * kk, sw128_kmajor_desc(b_addr + 32 * kk), idesc, i > 0 || kk > 0);
-        }
+        const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * xs16);
+        const uint32_t at = tmem + static_cast<uint32_t>(kAccCols + s * kACols);
+        umma_f16_ts(tmem, at, bd, idesc, i > 0);
+        umma_f16_ts(tmem, at + 8, bd + 2, idesc, true);
+        umma_f16_ts(tmem, at + 16, bd + 4, idesc, true);
+        umma_f16_ts(tmem, at + 24, bd + 6, idesc, true);
         umma_commit(&st_empty[s]);  // frees this stage's A and X buffers when the MMAs finish
         if (++s == S) {
           s = 0;
@@ -340,17 +348,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // ------------------------------------------------------ dequant warps
     // thread (r, h): weight row n0 + r, block h of each stage's two blocks. A
     // warp may only reach its own quarter of the TMEM lanes, so warp w takes
-    // rows 32 (w % 4) .. +31; lane = row.
+    // rows 32 (w % 4) .. +31; lane = row. Group dg takes every kDqGroups-th
+    // stage, so each warp has kDqGroups stages of MMA time per stage it converts.
     const int quarter = warp & 3;
-    const int r = 32 * quarter + lane, h = (warp - 2) >> 2;
+    const int dw = warp - 2, dg = dw >> 3;
+    const int r = 32 * quarter + lane, h = (dw >> 2) & 1;
     const int64_t n = n0 + r;
     const bool row_ok = n < p.N;
     const uint32_t a_lane = tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(kAccCols + 16 * h);
     constexpr int kWords = (kBlockBytes + 2 + 3) / 4;  // the block as words, plus the 16-bit shift (Q8: 9, Q4: 5)
-    for (int i = 0, s = 0, pass = 0; i < nst; ++i, (++s == S) ? (s = 0, ++pass) : 0) {
+    int s0 = dg, pass0 = 0;  // the slot and ring pass of stage dg (S >= kDqGroups)
+    for (int i = dg, s = s0, pass = pass0; i < nst;
+         i += kDqGroups, (s += kDqGroups) >= S ? (s -= S, ++pass) : 0) {
       const int c = i / (kRawBlocks / 2), q = i % (kRawBlocks / 2);
       const int kb = 2 * (j_lo + i) + h;  // this thread's block
-      if (q == 0) wait(&raw_full[c % kRawStages], static_cast<uint32_t>(c / kRawStages) & 1u);
+      if (q < kDqGroups) wait(&raw_full[c % kRawStages], static_cast<uint32_t>(c / kRawStages) & 1u);
       if (pass > 0) wait(&st_empty[s], static_cast<uint32_t>(pass - 1) & 1u);
       tc_fence_after();  // the MMAs that read this stage's A columns are complete
       const bool have = row_ok && kb < p.KB;
@@ -409,8 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&a_full[s]);
-        if (q == kRawBlocks / 2 - 1 || i == nst - 1) mbar_arrive(&raw_empty[c % kRawStages]);
+        mbar_arrive(&full[s]);
+        // this warp's last stage of the chunk (a chunk's slot is reused only after a whole chunk)
+        if (q + kDqGroups >= kRawBlocks / 2 || i + kDqGroups >= nst) mbar_arrive(&raw_empty[c % kRawStages]);
       }
     }
     wait(acc_full, 0);  // accumulator complete: every MMA (and so every stage buffer) is done
