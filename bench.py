@@ -677,7 +677,8 @@ def main(argv=None):
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved_gbs / pk["hbm_gbs"], 4),
                 "traffic": (round(traffic / launches) if traffic else None),
-                "kernel": "q8_gemv_kernel<1>",
+                "kernel": "q8_gemv (121 launches per step: fp32 register-resident, tensor-core resident and "
+                          "streaming variants)",
                 "per_launch": {"algorithmic_bytes": round(bytes_step / launches),
                                "avg_duration_us": round(ms_step * 1e3 / launches, 3)},
                 "peak_source": pk["source"], "vs_8TBs_spec": round(achieved_gbs / 8000.0, 4)}
