@@ -897,6 +897,265 @@ __global__ void __launch_bounds__(256, 2) q8_gemv_mma_kernel(const __grid_consta
   }
 }
 
+// ---------------------------------------------------------------------------
+// Integer tensor-core streaming variant (M = 1, K <= 2048, many rows per CTA:
+// lm_head-like shapes). The fp32 streaming kernel is ALU-bound in the int8 ->
+// fp32 conversion (~2.9 instructions per weight); here the raw int8 codes are
+// the A operand of mma.m16n8k32.s8 as they sit in shared memory, so a weight
+// costs only its share of the loads.
+//
+//  * Activations, once per CTA: x_j = M_j 2^(E_j - 150) (24-bit significand)
+//    becomes the integer x_int = M_j 2^(E_j - E_b + 38) (rounded to nearest
+//    for elements 2^38 below the block's largest exponent E_b), |x_int| <
+//    2^62, written as eight balanced base-256 digits in [-128, 127]: the
+//    bytes of (x_int + 0x8080..80) xor 0x8080..80. Digit k of the eight
+//    activations of a lane's k slots forms B column k.
+//  * C column k = sum_j q_j digit_k(x_j): exact int32 (|C| < 2^20). Thread
+//    (g, t) holds digits 2t, 2t+1 for rows g and g + 8 and adds
+//    (C_2t 2^16t + C_2t+1 2^(16t+8)) * d * 2^(E_b - E) in fp32 (E the largest
+//    E_b of the vector); the four digit lanes are summed at the end and the
+//    row total is scaled by 2^(E - 188). The only rounding is fp32's: the
+//    activation representation is exact for every element within 2^38 of its
+//    block maximum.
+//  * Rows come in 16-row tiles; 32 rows (two tiles) per stage for K <= 1024,
+//    16 otherwise. Eight consumer warps split a stage as (tile, K slice); the
+//    producer warp sums the K slices of each row in slice order when the
+//    stage is released and writes Y. Deterministic.
+
+struct alignas(64) DParams {
+  const uint8_t *W;
+  const float *X;
+  float *Y;
+  int64_t N;
+  int64_t row_bytes;
+  int64_t total_bytes;
+  int K, KB;
+  int grid;
+  int tps;        // 16-row tiles per stage (1 or 2)
+  int stages;
+  int stage_bytes;
+  int tab_off, ftab_off, eb_off, red_off, stage_off;  // shared-memory offsets
+  int prefetch_before_wait;
+};
+
+constexpr int kDigitWarps = 8;
+
+__device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9},"
+      " {%10, %10, %10, %10};"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+
+// x * 2^(38 - E_b) as a signed 64-bit integer (x = M 2^(E - 150)).
+__device__ __forceinline__ long long x_fixed(float x, int Eb) {
+  const uint32_t b = __float_as_uint(x);
+  int E = static_cast<int>((b >> 23) & 0xffu);
+  uint64_t M = b & 0x7fffffu;
+  if (E == 0) E = 1;
+  else M |= 0x800000u;
+  const int s = E - Eb + 38;
+  uint64_t v;
+  if (s >= 0) v = M << s;
+  else if (s > -26) v = (M + (uint64_t(1) << (-s - 1))) >> (-s);
+  else v = 0;
+  return (b >> 31) ? -static_cast<long long>(v) : static_cast<long long>(v);
+}
+
+__device__ __forceinline__ float int_exact_f(int v) {  // |v| < 2^22
+  return __int_as_float(v + 0x4B400000) - 12582912.0f;
+}
+
+template <int TPS>
+__global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(const __grid_constant__ DParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *empty = full + kMaxStages;
+  int *emax = reinterpret_cast<int *>(empty + kMaxStages);
+  uint2 *tab = reinterpret_cast<uint2 *>(smem + p.tab_off);     // [KB][32 lanes] B registers
+  float *ftab = reinterpret_cast<float *>(smem + p.ftab_off);   // [KB] 2^(E_b - E)
+  int *ebt = reinterpret_cast<int *>(smem + p.eb_off);          // [KB] E_b
+  float *red = reinterpret_cast<float *>(smem + p.red_off);     // [stage][kSlices][16 TPS rows]
+  uint8_t *stage_mem = smem + p.stage_off;
+  constexpr int kRows = 16 * TPS;
+  constexpr int kSlices = kDigitWarps / TPS;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * p.N / p.grid;
+  const int64_t r_end = static_cast<int64_t>(blockIdx.x + 1) * p.N / p.grid;
+  const int nchunks = static_cast<int>((r_end - r_begin + kRows - 1) / kRows);
+  const int S = p.stages;
+
+  pdl_launch_dependents();
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDigitWarps);
+    }
+    *emax = 1;
+    fence_mbar_init();
+  }
+  for (int b = tid; b < p.KB; b += blockDim.x) ebt[b] = 1;
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint64_t policy = 0;
+    auto issue = [&](int c) {
+      const int s = c % S;
+      const int64_t r0 = r_begin + static_cast<int64_t>(c) * kRows;
+      const int64_t r1 = min(r0 + kRows, r_end);
+      const int64_t b0 = r0 * p.row_bytes, b1 = r1 * p.row_bytes;
+      const int64_t a0 = b0 & ~int64_t(15);
+      int64_t a1 = (b1 + 15) & ~int64_t(15);
+      const int64_t lim = p.total_bytes & ~int64_t(15);
+      uint8_t *dst = stage_mem + static_cast<int64_t>(s) * p.stage_bytes;
+      if (a1 > lim) {  // last chunk of W: bytes past the last 16-byte boundary by hand
+        for (int64_t t = max(lim, a0); t < b1; ++t) dst[t - a0] = p.W[t];
+        a1 = max(lim, a0);
+      }
+      const uint32_t bytes = static_cast<uint32_t>(a1 - a0);
+      mbar_arrive_expect_tx(&full[s], bytes);
+      if (bytes) bulk_g2s(dst, p.W + a0, bytes, &full[s], policy);
+    };
+    const int prologue = min(S, nchunks);
+    if (lane == 0) {
+      policy = l2_evict_first_policy();
+      if (!p.prefetch_before_wait) pdl_wait();
+      for (int c = 0; c < prologue; ++c) issue(c);
+    }
+    pdl_wait();
+    bool ok = true;
+    int issued = prologue;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      ok = mbar_wait(&empty[c % S], static_cast<uint32_t>(c / S) & 1u);
+      if (!ok) break;
+      // rows of chunk c: sum the K slices in order, scale by 2^(E - 188) (two exact steps)
+      const int s = c % S;
+      const int64_t r0 = r_begin + static_cast<int64_t>(c) * kRows;
+      const int rows = static_cast<int>(min(static_cast<int64_t>(kRows), r_end - r0));
+      const int e = *emax - 188, e1 = max(e, -120);
+      const float f1 = __int_as_float((127 + e1) << 23), f2 = __int_as_float((127 + e - e1) << 23);
+      const float *rb = red + s * kSlices * kRows;
+      for (int r = lane; r < rows; r += 32) {
+        float v = rb[r];
+        for (int k = 1; k < kSlices; ++k) v += rb[k * kRows + r];
+        p.Y[r0 + r] = (v * f1) * f2;
+      }
+      __syncwarp();
+      if (lane == 0 && issued < nchunks) {
+        issue(issued);
+        ++issued;
+      }
+    }
+    if (!ok && lane == 0) {  // error path: record, then drain copies still in flight
+      atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+      for (int c = max(0, issued - S); c < issued; ++c)
+        if (!mbar_wait(&full[c % S], static_cast<uint32_t>(c / S) & 1u)) atomicOr(&g_q8_gemv_status, kDevTimeoutDrain);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  pdl_wait();
+  const int ctid = tid - 32;  // 0 .. 255
+  const int units = p.KB * 8;  // (block, t, half): four activations each
+  // pass 1: block exponents and the vector's largest
+  for (int u = ctid; u < units; u += 32 * kDigitWarps) {
+    const int b = u >> 3;
+    const float4 v = __ldg(reinterpret_cast<const float4 *>(p.X) + u);
+    const uint32_t m = max(max(__float_as_uint(v.x) & 0x7fffffffu, __float_as_uint(v.y) & 0x7fffffffu),
+                           max(__float_as_uint(v.z) & 0x7fffffffu, __float_as_uint(v.w) & 0x7fffffffu));
+    const int E = max(static_cast<int>(m >> 23), 1);
+    atomicMax(&ebt[b], E);
+    atomicMax(emax, E);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kDigitWarps) : "memory");
+  // pass 2: the digits, transposed into B registers: lane (k, t) of block b
+  // holds digit k of activations 8t..8t+3 (word 0) and 8t+4..8t+7 (word 1)
+  const int Emax = *emax;
+  for (int u = ctid; u < units; u += 32 * kDigitWarps) {
+    const int b = u >> 3, t = (u >> 1) & 3, h = u & 1;
+    const int Eb = ebt[b];
+    const float4 v = __ldg(reinterpret_cast<const float4 *>(p.X) + u);
+    const uint64_t bias = 0x8080808080808080ull;
+    const uint64_t d0 = (static_cast<uint64_t>(x_fixed(v.x, Eb)) + bias) ^ bias;
+    const uint64_t d1 = (static_cast<uint64_t>(x_fixed(v.y, Eb)) + bias) ^ bias;
+    const uint64_t d2 = (static_cast<uint64_t>(x_fixed(v.z, Eb)) + bias) ^ bias;
+    const uint64_t d3 = (static_cast<uint64_t>(x_fixed(v.w, Eb)) + bias) ^ bias;
+    uint32_t *tb = reinterpret_cast<uint32_t *>(tab + b * 32);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {  // digits 0..3, then 4..7
+      const uint32_t w0 = static_cast<uint32_t>(d0 >> (32 * half)), w1 = static_cast<uint32_t>(d1 >> (32 * half));
+      const uint32_t w2 = static_cast<uint32_t>(d2 >> (32 * half)), w3 = static_cast<uint32_t>(d3 >> (32 * half));
+      const uint32_t l01 = __byte_perm(w0, w1, 0x5140u), h01 = __byte_perm(w0, w1, 0x7362u);
+      const uint32_t l23 = __byte_perm(w2, w3, 0x5140u), h23 = __byte_perm(w2, w3, 0x7362u);
+      const uint32_t dig[4] = {__byte_perm(l01, l23, 0x5410u), __byte_perm(l01, l23, 0x7632u),
+                               __byte_perm(h01, h23, 0x5410u), __byte_perm(h01, h23, 0x7632u)};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) tb[2 * ((4 * half + k) * 4 + t) + h] = dig[k];  // lane 4k' + t, word h
+    }
+    if (t == 0 && h == 0) ftab[b] = Eb - Emax >= -126 ? __int_as_float((127 + Eb - Emax) << 23) : 0.f;
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kDigitWarps) : "memory");
+
+  const int cw = warp - 1;
+  const int tl = cw % TPS, ks = cw / TPS;  // this warp's tile of the stage and K slice
+  const int kb0 = ks * p.KB / kSlices, kb1 = (ks + 1) * p.KB / kSlices;
+  const int g = lane >> 2, t = lane & 3;
+  const float w0 = __int_as_float((127 + 16 * t) << 23), w1 = __int_as_float((127 + 16 * t + 8) << 23);
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = c % S;
+    if (!mbar_wait(&full[s], static_cast<uint32_t>(c / S) & 1u)) {
+      if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+      return;  // the producer times out on this warp's missing arrival and drains
+    }
+    const int64_t r0 = r_begin + static_cast<int64_t>(c) * kRows;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(kRows), r_end - r0));
+    const uint32_t base = smem_u32(stage_mem) + s * p.stage_bytes + static_cast<uint32_t>((r0 * p.row_bytes) & 15);
+    const int ra = tl * 16 + g, rb = ra + 8;  // rows of this lane
+    const bool oka = ra < rows, okb = rb < rows;
+    const uint32_t pa = base + static_cast<uint32_t>(min(ra, rows - 1) * p.row_bytes);
+    const uint32_t pb = base + static_cast<uint32_t>(min(rb, rows - 1) * p.row_bytes);
+    float2 acc = make_float2(0.f, 0.f);  // rows ra, rb
+#pragma unroll 4
+    for (int b = kb0; b < kb1; ++b) {
+      // codes 8t..8t+7 of both rows (2-byte aligned) and their block scales
+      const uint32_t ca = pa + 34u * b, cb = pb + 34u * b;
+      const uint32_t ma = (ca + 2u + 8u * t) & 2u, mb = (cb + 2u + 8u * t) & 2u;
+      const uint32_t xa = ca + 2u + 8u * t - ma, xb = cb + 2u + 8u * t - mb;
+      const uint32_t a0 = lds_u32(xa), a1w = lds_u32(xa + 4), a2 = lds_u32(xa + 8);
+      const uint32_t b0w = lds_u32(xb), b1w = lds_u32(xb + 4), b2w = lds_u32(xb + 8);
+      const uint32_t A0 = oka ? __funnelshift_r(a0, a1w, ma << 3) : 0u, A2 = oka ? __funnelshift_r(a1w, a2, ma << 3) : 0u;
+      const uint32_t A1 = okb ? __funnelshift_r(b0w, b1w, mb << 3) : 0u, A3 = okb ? __funnelshift_r(b1w, b2w, mb << 3) : 0u;
+      const float2 dd = make_float2(half_bits_to_float(lds_u16(ca)), half_bits_to_float(lds_u16(cb)));
+      const uint2 B = tab[b * 32 + lane];
+      int cc[4];
+      imma_16832(cc, A0, A1, A2, A3, B.x, B.y);
+      // this lane's two digits of both rows, then the block scale
+      const float2 lo = make_float2(int_exact_f(cc[0]), int_exact_f(cc[2]));
+      const float2 hi = make_float2(int_exact_f(cc[1]), int_exact_f(cc[3]));
+      const float2 v = __ffma2_rn(hi, make_float2(w1, w1), __fmul2_rn(lo, make_float2(w0, w0)));
+      const float f = ftab[b];
+      acc = __ffma2_rn(v, __fmul2_rn(dd, make_float2(f, f)), acc);
+    }
+    // the four digit lanes of each row
+    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
+    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
+    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 2);
+    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 2);
+    if (t == 0) {
+      float *rbuf = red + (s * kSlices + ks) * kRows;
+      rbuf[ra] = acc.x;
+      rbuf[rb] = acc.y;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
 int align_up(int64_t v, int a) { return static_cast<int>((v + a - 1) / a * a); }
 
 template <int MODE, int MP, int RG>
@@ -1163,6 +1422,64 @@ bool try_launch_mma(const DevInfo &dev, int64_t N, int K, const void *W, const f
   return true;
 }
 
+
+// Integer tensor-core streaming variant for M = 1, K <= 2048 and enough rows
+// for two CTAs per SM (returns false when the shape does not suit it).
+bool try_launch_digits(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, float *Y,
+                       cudaStream_t stream, uint32_t flags, qmm_status *out) {
+  if (K > 2048) return false;
+  const int grid = 2 * dev.sms;
+  if (N < static_cast<int64_t>(grid) * 32) return false;
+  const int KB = K / 32;
+  const int tps = K <= 1024 ? 2 : 1;
+  DParams p{};
+  p.W = static_cast<const uint8_t *>(W);
+  p.X = X;
+  p.Y = Y;
+  p.N = N;
+  p.K = K;
+  p.KB = KB;
+  p.row_bytes = 34ll * KB;
+  p.total_bytes = N * p.row_bytes;
+  p.grid = grid;
+  p.tps = tps;
+  p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
+  p.stage_bytes = align_up(16ll * tps * p.row_bytes + 64, 128);
+  p.tab_off = 1024;
+  p.ftab_off = p.tab_off + 256 * KB;
+  p.eb_off = p.ftab_off + 4 * KB;
+  p.red_off = align_up(p.eb_off + 4ll * KB, 16);
+  p.stage_off = align_up(p.red_off + 4ll * kMaxStages * 16 * kDigitWarps, 128);  // K-slice partials
+  constexpr int kBudget = 113 * 1024;  // two CTAs per SM
+  p.stages = std::min(kMaxStages, (kBudget - p.stage_off) / p.stage_bytes);
+  if (p.stages < 2) return false;
+  const size_t smem = static_cast<size_t>(p.stage_off) + static_cast<size_t>(p.stages) * p.stage_bytes;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3((kDigitWarps + 1) * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void (*kern)(DParams) = tps == 2 ? q8_gemv_digits_kernel<2> : q8_gemv_digits_kernel<1>;
+  static bool configured[2][64] = {};
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  if (dev_id >= 0 && dev_id < 64 && !configured[tps - 1][dev_id]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBudget);
+    if (e != cudaSuccess) {
+      *out = cuda_check(e, "q8_gemv attribute");
+      return true;
+    }
+    configured[tps - 1][dev_id] = true;
+  }
+  *out = cuda_check(cudaLaunchKernelEx(&cfg, kern, p), "q8_gemv launch");
+  return true;
+}
+
 }  // namespace
 
 qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
@@ -1175,6 +1492,7 @@ qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
     if (rows_per_cta * K >= kMmaMinSliceWeights && K <= kMmaMaxK && try_launch_mma(dev, N, K, W, X, Y, stream, flags, &st))
       return st;
     if (try_launch_resident(dev, N, K, W, X, Y, stream, flags, &st)) return st;
+    if (try_launch_digits(dev, N, K, W, X, Y, stream, flags, &st)) return st;
   }
   return launch_stream<kModeF32>(dev, M, N, K, W, X, nullptr, nullptr, Y, nullptr, stream, flags);
 }

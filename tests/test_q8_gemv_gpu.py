@@ -112,10 +112,11 @@ def test_empty_and_k0():
     assert qmm.device_status() == 0
 
 
-@pytest.mark.parametrize("n,k", [(37, 256), (2000, 2048)])
+@pytest.mark.parametrize("n,k", [(37, 256), (2000, 2048), (10000, 896)])
 def test_extreme_codes_and_scales_single_row(n, k):
     # the M = 1 kernels on the same extremes: (37, 256) takes the fp32 register-resident
-    # kernel, (2000, 2048) the tensor-core resident one
+    # kernel, (2000, 2048) the tensor-core resident one, (10000, 896) the integer
+    # tensor-core streaming one
     g = syn.rng(13)
     q = g.integers(-128, 128, size=(n, k)).astype(np.int8)
     q[0, :] = -128
@@ -153,7 +154,7 @@ def _dynamic_range_inputs(g, k):
     }
 
 
-@pytest.mark.parametrize("n,k", [(1152, 896), (896, 4864), (45, 160)])
+@pytest.mark.parametrize("n,k", [(1152, 896), (896, 4864), (45, 160), (12000, 896), (9472, 2048)])
 def test_single_row_activation_dynamic_range(n, k):
     g = syn.rng(21 + n + k)
     W, _, _ = syn.q8_0_weights(g, n, k)
@@ -211,3 +212,16 @@ def test_single_row_tensor_core_chained_calls():
         got = host(ys[i])
         assert_within(got, ref, S, TOL_FP32, f"chained call {i}")
         xin = got.astype(np.float32)
+
+
+@pytest.mark.parametrize("n,k", [
+    (10000, 896),   # two 16-row tiles per stage, ragged rows per CTA
+    (9472, 2048),   # one tile per stage (K > 1024)
+    (20011, 32),    # one block per row: most K slices empty
+    (30000, 864),   # odd block count
+    (40000, 1024),
+])
+def test_single_row_integer_streaming_shapes(n, k):
+    # M = 1 with many rows per CTA and K <= 2048: raw codes x 8-digit activations on the
+    # integer tensor cores
+    check(1, n, k, seed=61 + n + k)
