@@ -27,10 +27,14 @@
 // Data movement: a producer warp streams 8-block (256 k) stages with 2-D TMA
 // loads -- one 16-row x 144-byte box per weight tile and matrix, one
 // 8-token x 32-float box (128-byte swizzle) per block of X. Consumer warp w
-// owns block w of every stage for all of the CTA's row tiles, so its B
-// fragments are built once and reused 2 x tiles times. At the end the 8
-// warps' partial sums are added in warp order through shared memory and the
-// SwiGLU epilogue writes Y. Rows of W must be 16-byte multiples for the
+// owns block w % 8 of every stage for half of the CTA's row tiles (tiles i
+// with i % 2 == w / 8): sixteen consumer warps, four per scheduler, so the
+// chains of dependent mma / conversion instructions overlap (with eight the
+// kernel was latency-bound: ncu showed issue 46% active, tensor pipe 22%).
+// The hi and lo parts of each block accumulate in two independent chains.
+// Its B fragments are built once and reused for its tiles. At the end the
+// partial sums of the eight warps holding a tile are added in block order
+// through shared memory and the SwiGLU epilogue writes Y. Rows of W must be 16-byte multiples for the
 // tensor maps (K % 256 == 0); other K use the same code reading global memory
 // directly.
 //
@@ -48,7 +52,8 @@ namespace {
 
 static __device__ uint32_t g_q4_status;
 
-constexpr int kWarps = 8;            // consumer warps; warp w owns block w of each stage
+constexpr int kWarps = 16;           // consumer warps; warp w owns block w % 8 of each stage
+constexpr int kHalves = kWarps / 8;  // ... and the row tiles i with i % kHalves == w / 8
 constexpr int kBlocksPerStage = 8;   // 8 Q4_0 blocks = 256 k = 144 bytes per row
 constexpr int kTilesMax = 8;         // 16-row tiles per CTA
 constexpr int kStages = 4;
@@ -153,16 +158,17 @@ __device__ __forceinline__ BFrag make_bfrag(float4 x0, float4 x1) {
 __device__ __forceinline__ void tile_block(float (&acc)[4], uint32_t vg, uint32_t vh, float dg, float dh,
                                            const BFrag &b) {
   const Nib4 ng = q4_word_to_half2(vg), nh = q4_word_to_half2(vh);
-  float c[4] = {0.f, 0.f, 0.f, 0.f};
+  // the hi and lo parts in two independent chains, joined once: shorter latency
+  float c[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
   mma_16816(c, ng.lo01, nh.lo01, ng.lo23, nh.lo23, b.hi0, b.hi1);  // k-step 0 (low nibbles)
+  mma_16816(e, ng.lo01, nh.lo01, ng.lo23, nh.lo23, b.lo0, b.lo1);
   mma_16816(c, ng.hi01, nh.hi01, ng.hi23, nh.hi23, b.hi2, b.hi3);  // k-step 1 (high nibbles)
-  mma_16816(c, ng.lo01, nh.lo01, ng.lo23, nh.lo23, b.lo0, b.lo1);
-  mma_16816(c, ng.hi01, nh.hi01, ng.hi23, nh.hi23, b.lo2, b.lo3);
+  mma_16816(e, ng.hi01, nh.hi01, ng.hi23, nh.hi23, b.lo2, b.lo3);
   const float sg = __fmul_rn(dg, b.inv_scale), sh = __fmul_rn(dh, b.inv_scale);
-  acc[0] = __fmaf_rn(sg, c[0], acc[0]);
-  acc[1] = __fmaf_rn(sg, c[1], acc[1]);
-  acc[2] = __fmaf_rn(sh, c[2], acc[2]);
-  acc[3] = __fmaf_rn(sh, c[3], acc[3]);
+  acc[0] = __fmaf_rn(sg, __fadd_rn(c[0], e[0]), acc[0]);
+  acc[1] = __fmaf_rn(sg, __fadd_rn(c[1], e[1]), acc[1]);
+  acc[2] = __fmaf_rn(sh, __fadd_rn(c[2], e[2]), acc[2]);
+  acc[3] = __fmaf_rn(sh, __fadd_rn(c[3], e[3]), acc[3]);
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) {
@@ -249,9 +255,10 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
   // ---------------------------------------------------------------- consumers
   pdl_wait();
   const int g = lane >> 2, t = lane & 3;
-  float acc[kTilesMax][2][4];
+  const int wb = warp & 7, th = warp >> 3;  // this warp's block of the stage and tile parity
+  float acc[kTilesMax / kHalves][2][4];
 #pragma unroll
-  for (int i = 0; i < kTilesMax; ++i)
+  for (int i = 0; i < kTilesMax / kHalves; ++i)
 #pragma unroll
     for (int mat = 0; mat < 2; ++mat)
 #pragma unroll
@@ -264,12 +271,12 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
       if (lane == 0) atomicOr(&g_q4_status, kDevTimeoutFull);
       return;  // the producer gives up on this warp's missing arrival and drains
     }
-    const int kb = j * kBlocksPerStage + warp;  // this warp's block
+    const int kb = j * kBlocksPerStage + wb;  // this warp's block
     if (kb < p.KB) {
       // activations of block kb for token g
       float4 x0, x1;
       if (!DIRECT) {
-        const uint32_t xa = smem_u32(stages + s * kStageBytes + warp * 1024) + g * 128;
+        const uint32_t xa = smem_u32(stages + s * kStageBytes + wb * 1024) + g * 128;
         x0 = lds_f4(xa + 16u * (t ^ g));
         x1 = lds_f4(xa + 16u * ((4 + t) ^ g));
       } else if (g < p.M) {
@@ -284,15 +291,16 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
       for (int mat = 0; mat < 2; ++mat) {
         if (mat >= p.nmat) break;
 #pragma unroll
-        for (int i = 0; i < kTilesMax; ++i) {
+        for (int ii = 0; ii < kTilesMax / kHalves; ++ii) {
+          const int i = ii * kHalves + th;  // this warp's share of the row tiles
           if (i >= ntiles) break;
           uint32_t vg, vh;
           float dg, dh;
           if (!DIRECT) {
-            // row r of the tile at r * 144 bytes; block `warp` at 18 * warp
+            // row r of the tile at r * 144 bytes; block `wb` at 18 * wb
             const uint32_t tb = smem_u32(stages + s * kStageBytes + kXStageBytes + (mat * kTilesMax + i) * kTileBytes);
-            const uint32_t ag = tb + g * kRowStageBytes + 18 * warp, ah = ag + 8 * kRowStageBytes;
-            if (warp & 1) {  // block starts 2 bytes past a 4-byte boundary: qs word aligned
+            const uint32_t ag = tb + g * kRowStageBytes + 18 * wb, ah = ag + 8 * kRowStageBytes;
+            if (wb & 1) {  // block starts 2 bytes past a 4-byte boundary: qs word aligned
               vg = lds_u32(ag + 2 + 4 * t);
               vh = lds_u32(ah + 2 + 4 * t);
             } else {
@@ -316,7 +324,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
             vg = word(rg, dg);
             vh = word(rh, dh);
           }
-          tile_block(acc[i][mat], vg, vh, dg, dh, bf);
+          tile_block(acc[ii][mat], vg, vh, dg, dh, bf);
         }
       }
     }
@@ -329,15 +337,15 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
   // ------------------------------------------ cross-warp sum, SwiGLU epilogue
   // Every consumer has passed its last stage, so the stage memory is free.
   asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
-  float4 *red = reinterpret_cast<float4 *>(stages);  // [warp][tile][mat][lane]
+  float4 *red = reinterpret_cast<float4 *>(stages);  // [warp][tile of the warp][mat][lane]
 #pragma unroll
-  for (int i = 0; i < kTilesMax; ++i) {
-    if (i >= ntiles) break;
+  for (int ii = 0; ii < kTilesMax / kHalves; ++ii) {
+    if (ii * kHalves + th >= ntiles) break;
 #pragma unroll
     for (int mat = 0; mat < 2; ++mat) {
       if (mat >= p.nmat) break;
-      red[((warp * kTilesMax + i) * 2 + mat) * 32 + lane] =
-          make_float4(acc[i][mat][0], acc[i][mat][1], acc[i][mat][2], acc[i][mat][3]);
+      red[((warp * (kTilesMax / kHalves) + ii) * 2 + mat) * 32 + lane] =
+          make_float4(acc[ii][mat][0], acc[ii][mat][1], acc[ii][mat][2], acc[ii][mat][3]);
     }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
@@ -350,8 +358,11 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
     float v[2] = {0.f, 0.f};
     for (int mat = 0; mat < p.nmat; ++mat) {
       float sum = 0.f;
+      // the eight block warps that hold tile i, in block order
+      const int wbase = 8 * (i % kHalves), ii = i / kHalves;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) sum = __fadd_rn(sum, redf[(((w * kTilesMax + i) * 2 + mat) * 32 + src_lane) * 4 + idx]);
+      for (int b = 0; b < 8; ++b)
+        sum = __fadd_rn(sum, redf[((((wbase + b) * (kTilesMax / kHalves) + ii) * 2 + mat) * 32 + src_lane) * 4 + idx]);
       v[mat] = sum;
     }
     const int64_t n = 16ll * tile0 + rl;
@@ -419,7 +430,7 @@ qmm_status launch_proj(const DevInfo &dev, int M, int64_t N, int K, const void *
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(p.grid);
   cfg.blockDim = dim3((kWarps + 1) * 32);
-  cfg.dynamicSmemBytes = direct ? static_cast<size_t>(kWarps * kTilesMax * 2 * 32 * 16 + 2048)
+  cfg.dynamicSmemBytes = direct ? static_cast<size_t>(kWarps * (kTilesMax / kHalves) * 2 * 32 * 16 + 2048)
                                 : static_cast<size_t>(kBarBytes + kStages * kStageBytes + 1024);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
