@@ -321,7 +321,8 @@ def component_gateup(qmm, dev_peak_gbs, m=8, n=17408, k=5120, reps=10):
 
 def component_q8q8(qmm, dev_peak_gbs, reps_graph=4):
     """Q8xQ8 decode GEMV (M=1) at K=896/N=4864 and K=4864/N=896: the GEMV on
-    quantized activations alone, activation quantization + GEMV, and the fp32
+    quantized activations alone, activation quantization + GEMV as two launches
+    and as one fused launch, and the fp32
     activation GEMV of the same shape for comparison; rotating weight copies
     (> 2x L2) in one CUDA graph."""
     import torch
@@ -356,9 +357,15 @@ def component_q8q8(qmm, dev_peak_gbs, reps_graph=4):
             for w in Ws:
                 assert lib.qmm_q8_gemv_ex(1, n, k, 32, w.data_ptr(), x.data_ptr(), Y.data_ptr(), fl, h) == 0
 
+        def fused(h):
+            for w in Ws:
+                assert lib.qmm_q8q8_gemv_fused(1, n, k, 32, w.data_ptr(), x.data_ptr(), qx.data_ptr(), dx.data_ptr(),
+                                               Y.data_ptr(), fl, h) == 0
+
         res = {}
         for name, fn, extra in (("q8q8_gemv", gemv_q8, k + (k // 32) * 4),
                                 ("quantize_plus_q8q8_gemv", quant_gemv, k * 4),
+                                ("q8q8_gemv_fused", fused, k * 4 + k + (k // 32) * 4),
                                 ("f32_gemv_same_shape", gemv_f32, k * 4)):
             fn(s.cuda_stream)
             torch.cuda.synchronize()
@@ -515,6 +522,7 @@ def run_case(spec: str, reps: int, seed: int):
 
     gemv:N:K            qmm_q8_gemv, M=1
     q8q8:N:K            qmm_quantize_act_q8 + qmm_q8q8_gemv, M=1
+    q8q8f:N:K           qmm_q8q8_gemv_fused, M=1
     gateup:M:N:K        qmm_q4_swiglu_gateup
     prefill:q8|q4:M:N:K qmm_quant_matmul_prefill
     decode_step         the 121 GEMVs of one decode step
@@ -541,6 +549,14 @@ def run_case(spec: str, reps: int, seed: int):
         dx = torch.empty(1, k // 32, device="cuda")
         y = torch.empty(1, n, device="cuda")
         launches.append(lambda: (qmm.qmm_quantize_act_q8(x, qx, dx), qmm.qmm_q8q8_gemv(W, qx, dx, n, y)))
+    elif parts[0] == "q8q8f":
+        n, k = int(parts[1]), int(parts[2])
+        W = torch.from_numpy(syn.q8_0_weights(g, n, k)[0]).cuda()
+        x = torch.from_numpy(syn.act_f32(g, 1, k)).cuda()
+        qx = torch.empty(1, k, dtype=torch.int8, device="cuda")
+        dx = torch.empty(1, k // 32, device="cuda")
+        y = torch.empty(1, n, device="cuda")
+        launches.append(lambda: qmm.qmm_q8q8_gemv_fused(W, x, n, y, qx, dx))
     elif parts[0] == "gateup":
         m, n, k = int(parts[1]), int(parts[2]), int(parts[3])
         Wg = torch.from_numpy(syn.q4_0_weights(g, n, k)[0]).cuda()

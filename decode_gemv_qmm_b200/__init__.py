@@ -39,6 +39,7 @@ _SIGS = {
     "qmm_quantize_act_q8": [_i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q8q8_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_q8q8_gemv_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
+    "qmm_q8q8_gemv_fused": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _u32, _p],
     "qmm_q4_swiglu_gateup": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_q4_swiglu_gateup_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
     "qmm_quant_matmul_prefill": [_int, _i64, _i64, _i64, _int, _p, _p, _p, _p],
@@ -138,6 +139,19 @@ def qmm_q8q8_gemv(W: torch.Tensor, QX: torch.Tensor, DX: torch.Tensor, N: int, Y
         st = lib.qmm_q8q8_gemv(M, N, K, block, _ptr(W), _ptr(QX), _ptr(DX), _ptr(Y), _stream(stream))
     _check(st, "qmm_q8q8_gemv")
     return Y
+
+
+def qmm_q8q8_gemv_fused(W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None = None,
+                        QX: torch.Tensor | None = None, DX: torch.Tensor | None = None, *, block: int = BLOCK,
+                        flags: int = 0, stream=None):
+    """(Y, QX, DX): the Q8xQ8 GEMV of X with its own activation quantisation in the same call."""
+    M, K = X.shape
+    Y = _out(Y, (M, N), X.device)
+    QX = _out(QX, (M, K), X.device, torch.int8)
+    DX = _out(DX, (M, K // BLOCK), X.device)
+    _check(lib.qmm_q8q8_gemv_fused(M, N, K, block, _ptr(W), _ptr(X), _ptr(QX), _ptr(DX), _ptr(Y), flags,
+                                   _stream(stream)), "qmm_q8q8_gemv_fused")
+    return Y, QX, DX
 
 
 def qmm_q8q8_block_dots(W: torch.Tensor, QX: torch.Tensor, N: int, isum: torch.Tensor | None = None, *,

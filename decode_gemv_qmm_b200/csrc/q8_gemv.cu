@@ -488,6 +488,10 @@ struct alignas(64) RParams {
   int w_off;       // raw weight slice
   int max_rows;    // rows per CTA upper bound
   int prefetch_before_wait;
+  // fused Q8xQ8 only: the CTA's quantised activations, and where CTA 0 also writes them
+  int qx_off, dx_off;
+  int8_t *QXo;
+  float *DXo;
 };
 
 template <int U>
@@ -613,6 +617,187 @@ q8_gemv_resident_kernel(const __grid_constant__ RParams p) {
     for (int i = 4; i < 16; ++i) a[i & 3] = __ffma2_rn(wq[u][i], x2[i], a[i & 3]);
     const float2 t = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
     part[u] = wd[u] * (t.x + t.y);
+  }
+  if (!ok && tid == 0) {  // error path: give copies still in flight a bounded chance to land
+    if (!mbar_wait(wbar, 0) || !mbar_wait(xbar, 0)) atomicOr(&g_q8_gemv_status, kDevTimeoutDrain);
+  }
+  const float tot = warp_reduce_scatter<U>(part, lane);
+  const int ui = scatter_index<U>(lane);
+  const int rl = k + ui * p.wpw;
+  if (p.cg == 1) {
+    if (scatter_writer<U>(lane) && rl < rows) p.Y[r_begin + rl] = tot;
+    return;
+  }
+  if (scatter_writer<U>(lane) && rl < rows) red[cw * p.max_rows + rl] = tot;
+  __syncthreads();
+  for (int r = tid; r < rows; r += blockDim.x) {
+    float v = red[r];
+    for (int c = 1; c < p.cg; ++c) v += red[c * p.max_rows + r];
+    p.Y[r_begin + r] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fused Q8xQ8 resident variant (M = 1): the activation quantisation of
+// qmm_quantize_act_q8 done by every CTA into shared memory (same binary32
+// operations, so the same codes), then the exact int32 block dots on raw code
+// words held in registers. Q8 codes are one byte per weight, so a CTA keeps
+// its whole slice as raw words (8 registers per block and row) -- a quarter of
+// the fp32 resident form -- loaded and unpacked before the dependency wait; the
+// work left after it is the quantisation of X, eight dp4a per block and row,
+// one multiply by d_w * d_x, the reductions and the store.
+//
+//   isum[n][b] = sum_j q[n][b][j] * qx[32b + j]      (exact int32)
+//   Y[n]       = sum_b (d[n][b] * dx[b]) * isum[n][b]
+//
+// Quantisation: eight lanes per 32-block (four activations each, read from
+// the 128-byte-swizzled panel), the block maximum by a three-step shuffle max
+// over |x| bit patterns, then q8_act_scale / q8_act_code. CTA 0 also writes the
+// codes and scales to QX / DX.
+
+template <int U>
+__global__ void __launch_bounds__(512, 1) q8q8_resident_kernel(const __grid_constant__ RParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *wbar = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *xbar = wbar + 1;
+  float *red = reinterpret_cast<float *>(smem + p.red_off);
+  uint8_t *qx = smem + p.qx_off;
+  float *dx = reinterpret_cast<float *>(smem + p.dx_off);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * p.N / p.grid;
+  const int64_t r_end = static_cast<int64_t>(blockIdx.x + 1) * p.N / p.grid;
+  const int rows = static_cast<int>(r_end - r_begin);
+  const int64_t b0 = r_begin * p.row_bytes, b1 = r_end * p.row_bytes;
+  const int64_t a0 = b0 & ~int64_t(15);
+
+  pdl_launch_dependents();
+  if (tid == 0) {
+    mbar_init(wbar, 1);
+    mbar_init(xbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue_w = [&]() {
+    int64_t a1 = (b1 + 15) & ~int64_t(15);
+    const int64_t lim = p.total_bytes & ~int64_t(15);
+    uint8_t *dst = smem + p.w_off;
+    if (a1 > lim) {  // bytes past the last 16-byte boundary of W by hand
+      for (int64_t t = lim; t < b1; ++t) dst[t - a0] = p.W[t];
+      a1 = lim;
+    }
+    const uint32_t bytes = static_cast<uint32_t>(a1 - a0);
+    mbar_arrive_expect_tx(wbar, bytes);
+    const uint64_t pol = l2_evict_first_policy();
+    constexpr uint32_t kPiece = 8192;  // several copies in flight
+    for (uint32_t o = 0; o < bytes; o += kPiece)
+      bulk_g2s(dst + o, p.W + a0 + o, min(kPiece, bytes - o), wbar, pol);
+  };
+  auto issue_x = [&]() {
+    mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(p.KB) * 128u);
+    tma_load_2d(smem + p.xs_off, &p.xmap, 0, 0, xbar);
+  };
+  if (tid == 0) {
+    if (p.prefetch_before_wait) {
+      issue_w();
+      pdl_wait();
+      issue_x();
+    } else {
+      pdl_wait();
+      issue_x();
+      issue_w();
+    }
+  }
+
+  // ---- raw code words and block scales into registers (does not need X)
+  const int cw = warp % p.cg, k = warp / p.cg;
+  const int col = cw * 32 + lane;
+  const bool act = col < p.KB;
+  const uint32_t wbase = smem_u32(smem + p.w_off) + static_cast<uint32_t>(b0 - a0);
+  uint32_t wc[U][8];
+  float wd[U];
+  bool ok = mbar_wait(wbar, 0);
+  if (!ok && lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int rl = k + u * p.wpw;
+    if (ok && act && rl < rows) {
+      const uint32_t sa = wbase + static_cast<uint32_t>(rl * p.row_bytes) + 34u * col;
+      const uint32_t mis = sa & 2u, wa = sa - mis;
+      uint32_t w[9];
+#pragma unroll
+      for (int i = 0; i < 9; ++i) w[i] = lds_u32(wa + 4 * i);
+      const uint32_t r8 = mis << 3, sh = 16u + r8;
+      wd[u] = half_bits_to_float(__funnelshift_rc(w[0], w[1], r8));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wc[u][i] = __funnelshift_rc(w[i], w[i + 1], sh);
+    } else {
+      wd[u] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wc[u][i] = 0u;
+    }
+  }
+
+  // ---- activations (after the preceding grid has finished), quantised by the CTA
+  pdl_wait();
+  if (ok && !mbar_wait(xbar, 0)) {
+    ok = false;
+    if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
+  }
+  const uint32_t xa = smem_u32(smem + p.xs_off);
+  const int units = p.KB * 8;  // (block, unit of four activations)
+#pragma unroll 1
+  for (int base = warp * 32; base < units; base += blockDim.x) {  // uniform per warp: it shuffles
+    const int it = base + lane;
+    const int c = it >> 3, u = it & 7;
+    const bool have = ok && it < units;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (have) v = lds_f4(xa + 16u * (c * 8 + (u ^ (c & 7))));
+    uint32_t m = max(max(__float_as_uint(fabsf(v.x)), __float_as_uint(fabsf(v.y))),
+                     max(__float_as_uint(fabsf(v.z)), __float_as_uint(fabsf(v.w))));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    const float d = q8_act_scale(__uint_as_float(m));
+    const uint32_t word = (static_cast<uint32_t>(q8_act_code(v.x, d)) & 0xffu) |
+                          ((static_cast<uint32_t>(q8_act_code(v.y, d)) & 0xffu) << 8) |
+                          ((static_cast<uint32_t>(q8_act_code(v.z, d)) & 0xffu) << 16) |
+                          (static_cast<uint32_t>(q8_act_code(v.w, d)) << 24);
+    if (have) {
+      *reinterpret_cast<uint32_t *>(qx + 32 * c + 4 * u) = word;
+      if (u == 0) dx[c] = d;
+      if (blockIdx.x == 0) {  // the codes and scales for the caller
+        *reinterpret_cast<uint32_t *>(p.QXo + 32 * c + 4 * u) = word;
+        if (u == 0) p.DXo[c] = d;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- exact int32 block dots, then (d_w * d_x) * isum
+  uint32_t qa[8];
+  float dxv = 0.f;
+  if (ok && act) {
+    const uint4 lo = *reinterpret_cast<const uint4 *>(qx + 32 * col);
+    const uint4 hi = *reinterpret_cast<const uint4 *>(qx + 32 * col + 16);
+    qa[0] = lo.x; qa[1] = lo.y; qa[2] = lo.z; qa[3] = lo.w;
+    qa[4] = hi.x; qa[5] = hi.y; qa[6] = hi.z; qa[7] = hi.w;
+    dxv = dx[col];
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qa[i] = 0u;
+  }
+  float part[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    int s0 = 0, s1 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      s0 = __dp4a(static_cast<int>(wc[u][i]), static_cast<int>(qa[i]), s0);
+      s1 = __dp4a(static_cast<int>(wc[u][i + 1]), static_cast<int>(qa[i + 1]), s1);
+    }
+    part[u] = (wd[u] * dxv) * static_cast<float>(s0 + s1);  // |isum| <= 2^19: exact in fp32
   }
   if (!ok && tid == 0) {  // error path: give copies still in flight a bounded chance to land
     if (!mbar_wait(wbar, 0) || !mbar_wait(xbar, 0)) atomicOr(&g_q8_gemv_status, kDevTimeoutDrain);
@@ -1340,6 +1525,96 @@ bool try_launch_resident(const DevInfo &dev, int64_t N, int K, const void *W, co
   return true;
 }
 
+// Fused Q8xQ8 resident variant (returns false when the slice does not fit).
+bool try_launch_q8q8_resident(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, int8_t *QX,
+                              float *DX, float *Y, cudaStream_t stream, uint32_t flags, qmm_status *out) {
+  constexpr int kMaxWarps = 16;
+  constexpr int64_t kMaxSlice = 96 * 1024;
+  const int KB = K / 32;
+  const int cg = (KB + 31) / 32;
+  if (K * 4 > kPanelBytes) return false;
+  const int grid = static_cast<int>(std::min<int64_t>(N, dev.sms));
+  const int64_t rows = (N + grid - 1) / grid;
+  const int64_t row_bytes = 34ll * KB;
+  // U rows per warp; max warps per CTA for each U such that two CTAs' registers
+  // fit one SM (about 48, 56 and 72 registers a thread for U = 1, 2, 4)
+  const int maxw[3] = {kMaxWarps, kMaxWarps, 14};
+  int U = 0, wpw = 0;
+  for (int ui = 0; ui < 3; ++ui) {
+    const int u = 1 << ui;
+    const int w = static_cast<int>((rows + u - 1) / u);
+    if (cg * w <= maxw[ui]) {
+      U = u;
+      wpw = w;
+      break;
+    }
+  }
+  if (U == 0) return false;
+  const int64_t slice = rows * row_bytes + 48;
+  if (slice > kMaxSlice) return false;
+  RParams p{};
+  p.W = static_cast<const uint8_t *>(W);
+  p.Y = Y;
+  p.N = N;
+  p.row_bytes = row_bytes;
+  p.total_bytes = N * row_bytes;
+  p.K = K;
+  p.KB = KB;
+  p.grid = grid;
+  p.cg = cg;
+  p.wpw = wpw;
+  p.max_rows = static_cast<int>(rows);
+  p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
+  p.QXo = QX;
+  p.DXo = DX;
+  p.xs_off = 1024;
+  p.qx_off = align_up(p.xs_off + KB * 128, 128);
+  p.dx_off = align_up(p.qx_off + KB * 32, 128);
+  p.red_off = align_up(p.dx_off + KB * 4, 128);
+  p.w_off = align_up(p.red_off + cg * rows * 4, 128);
+  const size_t smem = static_cast<size_t>(align_up(p.w_off + slice, 128)) + 1024;
+  constexpr size_t kSmemAttr = 160 * 1024;
+  if (smem > kSmemAttr) return false;
+  const uint64_t dims[2] = {32, static_cast<uint64_t>(KB)};
+  const uint64_t strides[1] = {128};
+  const uint32_t box[2] = {32, static_cast<uint32_t>(KB)};
+  qmm_status st = encode_tiled(&p.xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, X, dims, strides, box,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QMM_OK) {
+    *out = st;
+    return true;
+  }
+  cudaLaunchConfig_t cfg{};
+  // Only the dot-product warps: a CTA must stay small enough (threads x
+  // registers) for two to share an SM, so that a launch can start while its
+  // predecessor in the stream still runs.
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(cg * wpw * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto go = [&](auto kern) -> cudaError_t {
+    static bool configured[3][64] = {};
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    const int idx = U == 1 ? 0 : U == 2 ? 1 : 2;
+    if (dev_id >= 0 && dev_id < 64 && !configured[idx][dev_id]) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemAttr));
+      if (e != cudaSuccess) return e;
+      configured[idx][dev_id] = true;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, p);
+  };
+  cudaError_t e = U == 1 ? go(q8q8_resident_kernel<1>) : U == 2 ? go(q8q8_resident_kernel<2>)
+                                                                : go(q8q8_resident_kernel<4>);
+  *out = cuda_check(e, "q8q8_gemv_fused launch");
+  return true;
+}
+
 // Tensor-core resident variant (returns false when the shape does not suit it).
 bool try_launch_mma(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, float *Y,
                     cudaStream_t stream, uint32_t flags, qmm_status *out) {
@@ -1499,6 +1774,17 @@ qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
 
 qmm_status launch_q8q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,
                             const float *DX, float *Y, cudaStream_t stream, uint32_t flags) {
+  return launch_stream<kModeQ8>(dev, M, N, K, W, nullptr, QX, DX, Y, nullptr, stream, flags);
+}
+
+qmm_status launch_q8q8_gemv_fused(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
+                                  int8_t *QX, float *DX, float *Y, cudaStream_t stream, uint32_t flags) {
+  qmm_status st;
+  if (M == 1 && try_launch_q8q8_resident(dev, N, K, W, X, QX, DX, Y, stream, flags, &st)) return st;
+  // Other shapes: the same quantisation as its own launch into the caller's
+  // QX / DX, then the streaming Q8xQ8 kernel.
+  st = launch_quantize_act_q8(dev, M, K, X, QX, DX, stream, kLaunchPdl);
+  if (st != QMM_OK) return st;
   return launch_stream<kModeQ8>(dev, M, N, K, W, nullptr, QX, DX, Y, nullptr, stream, flags);
 }
 

@@ -159,6 +159,27 @@ static qmm_status q8q8_impl(int64_t M, int64_t N, int64_t K, int block, const vo
   return launch_q8q8_gemv(dev, static_cast<int>(M), N, static_cast<int>(K), W, QX, DX, Y, s, flags);
 }
 
+static qmm_status q8q8_fused_impl(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
+                                  int8_t *QX, float *DX, float *Y, qmm_stream_t stream, uint32_t user_flags) {
+  const char *fn = "qmm_q8q8_gemv_fused";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, N, K, block, QMM_MAX_DECODE_M));
+  if (user_flags & ~uint32_t(QMM_FLAG_EARLY_WEIGHTS))
+    return set_error(QMM_ERR_SHAPE, "%s: unknown flags 0x%x", fn, user_flags);
+  if (M == 0 || N == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "W", W, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "X", X, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "QX", QX, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "DX", DX, K > 0, 4));
+  QMM_TRY(check_ptr(fn, "Y", Y, true, 4));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return zero_fill(Y, M * N, s);
+  uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
+  return launch_q8q8_gemv_fused(dev, static_cast<int>(M), N, static_cast<int>(K), W, X, QX, DX, Y, s, flags);
+}
+
 static qmm_status gateup_impl(int64_t M, int64_t N, int64_t K, int block, const void *Wg, const void *Wu,
                               const float *X, float *G, float *U, float *Y, qmm_stream_t stream, bool unfused,
                               uint32_t user_flags) {
@@ -239,6 +260,11 @@ QMM_API qmm_status qmm_q8q8_gemv(int64_t M, int64_t N, int64_t K, int block, con
 QMM_API qmm_status qmm_q8q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, const void *W, const int8_t *QX,
                                     const float *DX, float *Y, uint32_t flags, qmm_stream_t stream) {
   return q8q8_impl(M, N, K, block, W, QX, DX, Y, nullptr, stream, flags);
+}
+
+QMM_API qmm_status qmm_q8q8_gemv_fused(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
+                                       int8_t *QX, float *DX, float *Y, uint32_t flags, qmm_stream_t stream) {
+  return q8q8_fused_impl(M, N, K, block, W, X, QX, DX, Y, stream, flags);
 }
 
 QMM_API qmm_status qmm_q8q8_block_dots(int64_t M, int64_t N, int64_t K, int block, const void *W, const int8_t *QX,

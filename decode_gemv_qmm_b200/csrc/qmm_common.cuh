@@ -131,6 +131,19 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
   return v;
 }
 
+// Q8 activation quantisation of one element ("Lumen v0.4.0", section "Phase
+// 7.M -- Q8xQ8 AVX2 int dot"): with the block scale d = amax / 127 (IEEE
+// binary32 division), q = round-half-away-from-zero(x / d) (binary32 division)
+// clamped to [-127, 127]; d == 0 gives 0. Every kernel that quantises
+// activations calls these two functions, so their codes agree bit for bit.
+__device__ __forceinline__ float q8_act_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
+__device__ __forceinline__ int q8_act_code(float x, float d) {
+  if (d == 0.0f) return 0;
+  float r = roundf(__fdiv_rn(x, d));
+  r = fminf(fmaxf(r, -127.0f), 127.0f);
+  return static_cast<int>(r);
+}
+
 // fp16 bits -> float (exact).
 __device__ __forceinline__ float half_bits_to_float(uint32_t bits16) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(bits16 & 0xffffu)));

@@ -28,14 +28,8 @@ __global__ void __launch_bounds__(256) quantize_act_q8_kernel(const float *__res
   for (int64_t b = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; b < nblocks; b += nwarps) {
     const float x = __ldg(X + b * 32 + lane);
     const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(x))));
-    const float d = __fdiv_rn(amax, 127.0f);
-    int q = 0;
-    if (d != 0.0f) {
-      float r = roundf(__fdiv_rn(x, d));
-      r = fminf(fmaxf(r, -127.0f), 127.0f);
-      q = static_cast<int>(r);
-    }
-    QX[b * 32 + lane] = static_cast<int8_t>(q);
+    const float d = q8_act_scale(amax);
+    QX[b * 32 + lane] = static_cast<int8_t>(q8_act_code(x, d));
     if (lane == 0) DX[b] = d;
   }
 }

@@ -171,6 +171,27 @@ QMM_API qmm_status qmm_q8q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, 
                                     qmm_stream_t stream);
 
 /*
+ * qmm_q8q8_gemv_fused -- qmm_quantize_act_q8 followed by qmm_q8q8_gemv as one
+ * call: the per-block activation quantisation of "Lumen v0.4.0", section
+ * "Phase 7.M -- Q8xQ8 AVX2 int dot", done inside the GEMV (at M = 1, when each
+ * CTA's weight slice fits on chip, every CTA quantises X itself; otherwise a
+ * quantisation launch precedes the streaming Q8xQ8 launch).
+ *
+ *   M       1 .. QMM_MAX_DECODE_M (0 = empty call)
+ *   W       N * K/32 Q8_0 blocks (16-byte aligned)
+ *   X       M x K fp32 (16-byte aligned, read only)
+ *   QX, DX  M x K int8 (16-byte aligned) and M x K/32 fp32, written with the
+ *           codes and scales qmm_quantize_act_q8 writes for X (bit for bit),
+ *           so other Q8xQ8 calls on the same X can reuse them; caller-owned,
+ *           the call allocates nothing
+ *   Y       M x N fp32 (written), the qmm_q8q8_gemv formula
+ *   flags   0 or QMM_FLAG_EARLY_WEIGHTS
+ */
+QMM_API qmm_status qmm_q8q8_gemv_fused(int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                       const float *X, int8_t *QX, float *DX, float *Y, uint32_t flags,
+                                       qmm_stream_t stream);
+
+/*
  * qmm_q4_swiglu_gateup -- fused gate/up projection with SwiGLU on Q4_0 weights.
  *
  * "LSE v0.4.16", section "Combined M8 Q4 gate/up execution": one launch reads

@@ -19,7 +19,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     names = declared_symbols()
-    assert len(names) >= 13
+    assert len(names) >= 14
     for name in names:
         assert hasattr(lib, name), f"{name} declared in include/qmm.h but not exported"
 
@@ -53,6 +53,11 @@ def st_name(st):
     (lambda: lib.qmm_q8q8_gemv(1, 8, 64, 32, P16, 0, P16, P16, 0), "QMM_ERR_NULL"),
     (lambda: lib.qmm_q8q8_gemv(1, 8, 64, 32, P16, P16, 0, P16, 0), "QMM_ERR_NULL"),
     (lambda: lib.qmm_q8q8_block_dots(1, 8, 64, 32, P16, P16, 0, 0), "QMM_ERR_NULL"),
+    (lambda: lib.qmm_q8q8_gemv_fused(1, 8, 64, 32, P16, P16, 0, P16, P16, 0, 0), "QMM_ERR_NULL"),
+    (lambda: lib.qmm_q8q8_gemv_fused(1, 8, 64, 32, P16, P16, P16, 0, P16, 0, 0), "QMM_ERR_NULL"),
+    (lambda: lib.qmm_q8q8_gemv_fused(1, 8, 64, 32, P16, P16, P_ODD, P16, P16, 0, 0), "QMM_ERR_ALIGN"),
+    (lambda: lib.qmm_q8q8_gemv_fused(9, 8, 64, 32, P16, P16, P16, P16, P16, 0, 0), "QMM_ERR_SHAPE"),
+    (lambda: lib.qmm_q8q8_gemv_fused(1, 8, 64, 32, P16, P16, P16, P16, P16, 2, 0), "QMM_ERR_SHAPE"),
     (lambda: lib.qmm_q4_swiglu_gateup(9, 8, 64, 32, P16, P16, P16, P16, 0), "QMM_ERR_SHAPE"),
     (lambda: lib.qmm_q4_swiglu_gateup(8, 8, 64, 32, P16, P_ODD, P16, P16, 0), "QMM_ERR_ALIGN"),
     (lambda: lib.qmm_q4_gateup_unfused(8, 8, 64, 32, P16, P16, P16, 0, P16, P16, 0), "QMM_ERR_NULL"),
@@ -72,6 +77,7 @@ def test_empty_calls_are_ok_without_touching_cuda():
     assert lib.qmm_quantize_act_q8(0, 64, 32, 0, 0, 0, 0) == 0
     assert lib.qmm_quantize_act_q8(3, 0, 32, 0, 0, 0, 0) == 0
     assert lib.qmm_q4_swiglu_gateup(0, 5, 64, 32, 0, 0, 0, 0, 0) == 0
+    assert lib.qmm_q8q8_gemv_fused(0, 5, 64, 32, 0, 0, 0, 0, 0, 0, 0) == 0
     assert lib.qmm_quant_matmul_prefill(1, 5, 0, 64, 32, 0, 0, 0, 0) == 0
 
 
