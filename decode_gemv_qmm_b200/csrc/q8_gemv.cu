@@ -1525,10 +1525,11 @@ bool try_launch_resident(const DevInfo &dev, int64_t N, int K, const void *W, co
   return true;
 }
 
-// Fused Q8xQ8 resident variant (returns false when the slice does not fit).
+// Fused Q8xQ8 resident variant: false when the slice does not fit. Warps per
+// CTA are capped so that two CTAs' registers fit one SM (the next launch in the
+// stream can then start, and prefetch its weights, while this one runs).
 bool try_launch_q8q8_resident(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, int8_t *QX,
                               float *DX, float *Y, cudaStream_t stream, uint32_t flags, qmm_status *out) {
-  constexpr int kMaxWarps = 16;
   constexpr int64_t kMaxSlice = 96 * 1024;
   const int KB = K / 32;
   const int cg = (KB + 31) / 32;
@@ -1536,9 +1537,9 @@ bool try_launch_q8q8_resident(const DevInfo &dev, int64_t N, int K, const void *
   const int grid = static_cast<int>(std::min<int64_t>(N, dev.sms));
   const int64_t rows = (N + grid - 1) / grid;
   const int64_t row_bytes = 34ll * KB;
-  // U rows per warp; max warps per CTA for each U such that two CTAs' registers
-  // fit one SM (about 48, 56 and 72 registers a thread for U = 1, 2, 4)
-  const int maxw[3] = {kMaxWarps, kMaxWarps, 14};
+  // U rows per warp; at about 48 / 56 / 72 registers a thread for U = 1, 2, 4
+  // these warp counts leave room for two CTAs per SM
+  const int maxw[3] = {16, 16, 14};
   int U = 0, wpw = 0;
   for (int ui = 0; ui < 3; ++ui) {
     const int u = 1 << ui;
@@ -1585,9 +1586,6 @@ bool try_launch_q8q8_resident(const DevInfo &dev, int64_t N, int K, const void *
     return true;
   }
   cudaLaunchConfig_t cfg{};
-  // Only the dot-product warps: a CTA must stay small enough (threads x
-  // registers) for two to share an SM, so that a launch can start while its
-  // predecessor in the stream still runs.
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(cg * wpw * 32);
   cfg.dynamicSmemBytes = smem;
