@@ -65,7 +65,11 @@ constexpr int kRawBlocks = 8;          // blocks per raw weight chunk
 constexpr int kStageK = 64;            // k per MMA stage (one 128-byte swizzle row of bf16)
 constexpr int kAccCols = 256;          // TMEM columns 0..255: the fp32 accumulator (MT <= 256)
 constexpr int kACols = 32;             // TMEM columns per A stage: 128 rows x 64 bf16 (two per 32-bit cell)
-constexpr int kRawStages = 4;          // raw chunks in flight: three chunks (12 stages) of lead
+// Raw chunks in flight. Q8 chunks are twice the size of Q4 ones; two in flight
+// (eight stages of lead) leave room for four X stages instead of two, which
+// measured 8-15% faster on the Q8 panels.
+template <int WT>
+constexpr int raw_stages() { return WT == QMM_Q8_0 ? 2 : 4; }
 constexpr int kMaxSplit = 8;           // portable cluster size
 
 struct alignas(64) Params {
@@ -85,7 +89,7 @@ struct alignas(64) Params {
   int x_stage_bytes;
   int off_x, off_raw;  // shared-memory offsets (1024-aligned)
   int split;           // K ranges per output tile (cluster size along z)
-  int red_pitch;       // floats per row of the split-K exchange buffer (MT + 4)
+  int red_pitch;       // floats per token column of the split-K exchange buffer (rows of one rank)
 };
 
 // ---------------------------------------------------------------- tcgen05 PTX
@@ -177,9 +181,8 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
+__device__ __forceinline__ void st_cluster_b32(uint32_t addr, uint32_t a) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
 }
 
 // ------------------------------------------------------------- block decode
@@ -218,6 +221,7 @@ template <int WT>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kRawStages = raw_stages<WT>();
   // barriers: full[8], st_empty[8], raw_full[kRawStages], raw_empty[kRawStages], acc_full, tmem slot.
   // full[s]: the stage's X tile has landed (producer arrival + TMA bytes) and
   // all dequant warps have written its A columns -- one wait for the issuer.
@@ -453,23 +457,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // Split K: rank r owns weight rows [r*128/split, (r+1)*128/split) of the
     // tile and receives every rank's partial of them in its X stage and raw
     // chunk buffers (free once all ranks' accumulators are complete: first
-    // cluster barrier).
-    const int rmax = (128 + split - 1) / split;
-    const uint32_t xbuf = sbase + p.off_x;  // [src rank][rmax rows][red_pitch floats]
+    // cluster barrier). The buffer is [source rank][token column][row of the
+    // owner], rows contiguous: a warp holds 32 consecutive rows of one column
+    // after each TMEM load, so every remote store is one contiguous 128-byte
+    // segment (storing each row's columns instead scattered a warp's store
+    // over 32 rows and made the exchange several times slower).
+    const uint32_t xbuf = sbase + p.off_x;
     cluster_sync_all();
     if (epi) {
       tc_fence_after();
       const int row = 32 * quarter + lane;
       const int dst = (row * split + split - 1) / 128;  // owner rank of this row
       const int lr = row - dst * 128 / split;
-      const uint32_t raddr =
-          map_rank(xbuf + static_cast<uint32_t>(((zr * rmax + lr) * p.red_pitch) * 4), static_cast<uint32_t>(dst));
+      const uint32_t raddr = map_rank(xbuf + static_cast<uint32_t>((zr * p.MT * p.red_pitch + lr) * 4),
+                                      static_cast<uint32_t>(dst));
+      const uint32_t cstride = static_cast<uint32_t>(p.red_pitch) * 4u;
       for (int c0 = col0; c0 < p.MT; c0 += 32 * (kDqWarps / 4)) {
         uint32_t v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(c0), v);
 #pragma unroll
-        for (int c = 0; c < 32; c += 4)  // MT is a multiple of 16: the last load may hold 16 columns
-          if (c0 + c < p.MT) st_cluster_v4(raddr + 4u * (c0 + c), v[c], v[c + 1], v[c + 2], v[c + 3]);
+        for (int c = 0; c < 32; ++c)  // MT is a multiple of 16: the last load may hold 16 columns
+          if (c0 + c < p.MT) st_cluster_b32(raddr + static_cast<uint32_t>(c0 + c) * cstride, v[c]);
       }
     }
     cluster_sync_all();  // every partial has landed
@@ -481,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const int m = m0 + col;
         const int64_t row = n0 + rbase + lr;
         float acc = 0.f;
-        for (int src = 0; src < split; ++src) acc += buf[(src * rmax + lr) * p.red_pitch + col];
+        for (int src = 0; src < split; ++src) acc += buf[(src * p.MT + col) * p.red_pitch + lr];
         if (m < p.M && row < p.N) p.Y[static_cast<int64_t>(m) * p.N + row] = acc;
       }
     }
@@ -525,7 +533,7 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
   // a row's chunk plus up to 15 bytes of alignment in front, rounded to 16
   // and then to 16 mod 32 (rows spread over eight 4-byte bank groups)
   p.raw_pitch = wtype == QMM_Q8_0 ? 304 : 176;
-  const int raw_bytes = kRawStages * 128 * p.raw_pitch;
+  const int raw_bytes = (wtype == QMM_Q8_0 ? raw_stages<QMM_Q8_0>() : raw_stages<QMM_Q4_0>()) * 128 * p.raw_pitch;
   const int per_stage = p.x_stage_bytes;  // A lives in tensor memory
   const int budget = dev.smem_optin - 1024 /*align*/ - 1024 /*barriers*/ - round_up(raw_bytes, 1024);
   p.stages = std::max(2, std::min(8, budget / per_stage));
@@ -576,7 +584,7 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
     for (; split > 1; --split) {
       const int rmax = (128 + split - 1) / split;
       // the exchange buffer reuses the X stages and the raw chunks (all consumed by then)
-      if (static_cast<int64_t>(split) * rmax * (p.MT + 4) * 4 > p.off_raw + raw_bytes - p.off_x) continue;
+      if (static_cast<int64_t>(split) * p.MT * rmax * 4 > p.off_raw + raw_bytes - p.off_x) continue;
       cfg.gridDim = dim3(static_cast<unsigned>(mtiles), static_cast<unsigned>(ntiles), static_cast<unsigned>(split));
       attr[1].val.clusterDim.x = 1;
       attr[1].val.clusterDim.y = 1;
@@ -588,7 +596,7 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
     }
   }
   p.split = split;
-  p.red_pitch = p.MT + 4;
+  p.red_pitch = (128 + split - 1) / split;  // rows of the largest rank share
   if (p.rs == 1 && split == 1) p.raw_pitch = kRawBlocks * bb;  // chunks start on 16-byte boundaries: 272 / 144
   if (p.tma_rows > 0) {
     const uint64_t wd[2] = {static_cast<uint64_t>(p.rs * p.row_bytes / 2), static_cast<uint64_t>(N / p.rs)};
