@@ -1168,9 +1168,15 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   constexpr int kSlices = kDigitWarps / TPS;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * p.N / p.grid;
-  const int64_t r_end = static_cast<int64_t>(blockIdx.x + 1) * p.N / p.grid;
-  const int nchunks = static_cast<int>((r_end - r_begin + kRows - 1) / kRows);
+  // whole chunks per CTA: a chunk costs the same however few of its rows are
+  // valid, so an even split of rows (every CTA ending in a one-row chunk)
+  // costs a chunk per CTA more than an even split of chunks
+  const int64_t tchunks = (p.N + kRows - 1) / kRows;
+  const int64_t c_begin = static_cast<int64_t>(blockIdx.x) * tchunks / p.grid;
+  const int64_t c_end = static_cast<int64_t>(blockIdx.x + 1) * tchunks / p.grid;
+  const int64_t r_begin = c_begin * kRows;
+  const int64_t r_end = min(p.N, c_end * kRows);
+  const int nchunks = static_cast<int>(c_end - c_begin);
   const int S = p.stages;
 
   pdl_launch_dependents();
