@@ -259,7 +259,10 @@ def component_single_gemv(qmm, dev_peak_gbs, n=1152, k=896, reps_graph=4):
 
 
 def component_lm_head(qmm, step: DecodeStep, dev_peak_gbs, reps=20):
-    """The largest GEMV of the step alone (lm_head 896->151936, 145 MB of blocks)."""
+    """The largest GEMV of the step (lm_head 896->151936, 145 MB of blocks): one
+    launch alone per graph replay, and per launch in a chain of dependent
+    launches over three weight copies (as in the step: programmatic dependent
+    launch, weights streamed ahead of the dependency)."""
     import torch
 
     n, k = step.shapes[-1][1], step.shapes[-1][2]
@@ -267,6 +270,7 @@ def component_lm_head(qmm, step: DecodeStep, dev_peak_gbs, reps=20):
     W = step.W[-1]
     xp = step.X.data_ptr() + 4 * int(step.x_offsets[-2])
     yp = step.Y.data_ptr() + 4 * int(step.y_offsets[-2])
+    bytes_ = n * (k // 32) * 34 + k * 4 + n * 4
 
     def fn(h):
         assert qmm.lib.qmm_q8_gemv_ex(1, n, k, 32, W.data_ptr(), xp, yp, 0, h) == 0
@@ -274,9 +278,22 @@ def component_lm_head(qmm, step: DecodeStep, dev_peak_gbs, reps=20):
     gr = capture(fn, s)
     time_graph(gr, s, 3)
     ms = time_graph(gr, s, reps)
-    bytes_ = n * (k // 32) * 34 + k * 4 + n * 4
-    return {"us": round(ms * 1e3, 2), "GB_s": round(bytes_ / ms / 1e6, 1),
-            "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4), "bytes": bytes_}
+    out = {"us": round(ms * 1e3, 2), "GB_s": round(bytes_ / ms / 1e6, 1),
+           "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4), "bytes": bytes_}
+    Ws = [W] + [W.clone() for _ in range(2)]
+
+    def chain(h):
+        for w in Ws:
+            assert qmm.lib.qmm_q8_gemv_ex(1, n, k, 32, w.data_ptr(), xp, yp, qmm.QMM_FLAG_EARLY_WEIGHTS, h) == 0
+    chain(s.cuda_stream)
+    torch.cuda.synchronize()
+    gr2 = capture(chain, s)
+    time_graph(gr2, s, 3)
+    ms2 = time_graph(gr2, s, reps) / len(Ws)
+    out["chain"] = {"us": round(ms2 * 1e3, 2), "GB_s": round(bytes_ / ms2 / 1e6, 1),
+                    "frac_hbm": round(bytes_ / ms2 / 1e6 / dev_peak_gbs, 4)}
+    del gr2, Ws
+    return out
 
 
 def component_gateup(qmm, dev_peak_gbs, m=8, n=17408, k=5120, reps=10):
