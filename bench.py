@@ -192,6 +192,32 @@ class DecodeStep:
             if st != 0:
                 raise qmm.QmmError(st, "qmm_q8_gemv_ex")
 
+    def launch_multi(self, qmm, stream_handle: int, flags: int):
+        """The same matmul set with each layer's gate and up projections as one
+        qmm_q8_gemv_multi launch over the gate's activation vector (97 launches)."""
+        import ctypes
+
+        lib = qmm.lib
+        xp, yp = self.X.data_ptr(), self.Y.data_ptr()
+        i = 0
+        while i < len(self.shapes):
+            name, n, k = self.shapes[i]
+            if name.endswith(".gate") and i + 1 < len(self.shapes) and self.shapes[i + 1][0].endswith(".up"):
+                n2 = self.shapes[i + 1][1]
+                N = (ctypes.c_int64 * 2)(n, n2)
+                W = (ctypes.c_void_p * 2)(self.W[i].data_ptr(), self.W[i + 1].data_ptr())
+                Y = (ctypes.c_void_p * 2)(yp + 4 * int(self.y_offsets[i]), yp + 4 * int(self.y_offsets[i + 1]))
+                st = lib.qmm_q8_gemv_multi(1, k, 32, 2, N, W, xp + 4 * int(self.x_offsets[i]), Y, flags, stream_handle)
+                if st != 0:
+                    raise qmm.QmmError(st, "qmm_q8_gemv_multi")
+                i += 2
+                continue
+            st = lib.qmm_q8_gemv_ex(1, n, k, 32, self.W[i].data_ptr(), xp + 4 * int(self.x_offsets[i]),
+                                    yp + 4 * int(self.y_offsets[i]), flags, stream_handle)
+            if st != 0:
+                raise qmm.QmmError(st, "qmm_q8_gemv_ex")
+            i += 1
+
     def logits(self):
         return self.Y[int(self.y_offsets[-2]):int(self.y_offsets[-1])]
 
@@ -294,6 +320,25 @@ def component_lm_head(qmm, step: DecodeStep, dev_peak_gbs, reps=20):
                     "frac_hbm": round(bytes_ / ms2 / 1e6 / dev_peak_gbs, 4)}
     del gr2, Ws
     return out
+
+
+def component_step_multi(qmm, step: DecodeStep, dev_peak_gbs, reps=200):
+    """The decode step's matmul set with gate and up of each layer sharing one
+    activation vector in one qmm_q8_gemv_multi launch (97 launches instead of
+    121; same bytes). A variant next to the headline, which keeps 121 GEMVs."""
+    import torch
+
+    s = torch.cuda.Stream()
+    flags = qmm.QMM_FLAG_EARLY_WEIGHTS
+    step.launch_multi(qmm, s.cuda_stream, flags)
+    torch.cuda.synchronize()
+    gr = capture(lambda h: step.launch_multi(qmm, h, flags), s)
+    time_graph(gr, s, 20)
+    ms = time_graph(gr, s, reps)
+    del gr
+    bytes_ = sum(n * (k // 32) * 34 + k * 4 + n * 4 for _, n, k in step.shapes)
+    return {"ms_per_step": round(ms, 5), "tok_s": round(1e3 / ms, 2), "launches": 97,
+            "GB_s": round(bytes_ / ms / 1e6, 1), "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4)}
 
 
 def component_gateup(qmm, dev_peak_gbs, m=8, n=17408, k=5120, reps=10):
@@ -720,6 +765,7 @@ def main(argv=None):
     components = None
     if rank == 0 and world == 1 and not args.no_components:
         components = {"lm_head_896x151936": component_lm_head(qmm, step, pk["hbm_gbs"]),
+                      "decode_step_gate_up_multi": component_step_multi(qmm, step, pk["hbm_gbs"]),
                       "single_gemv_896x1152": component_single_gemv(qmm, pk["hbm_gbs"]),
                       "q4_gateup_m8_k5120_n17408": component_gateup(qmm, pk["hbm_gbs"]),
                       "q8q8_gemv": component_q8q8(qmm, pk["hbm_gbs"]),

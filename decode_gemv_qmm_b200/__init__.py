@@ -31,6 +31,7 @@ QMM_FLAG_EARLY_WEIGHTS = 1
 BLOCK = 32
 MAX_DECODE_M = 8
 MAX_K = 32768
+MAX_PROJ = 4
 
 _i64, _int, _u32, _p = ctypes.c_int64, ctypes.c_int, ctypes.c_uint32, ctypes.c_void_p
 _SIGS = {
@@ -39,6 +40,7 @@ _SIGS = {
     "qmm_quantize_act_q8": [_i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q8q8_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_q8q8_gemv_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
+    "qmm_q8_gemv_multi": [_i64, _i64, _int, _int, _p, _p, _p, _p, _u32, _p],
     "qmm_q8q8_gemv_fused": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _u32, _p],
     "qmm_q4_swiglu_gateup": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_q4_swiglu_gateup_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
@@ -115,6 +117,20 @@ def qmm_q8_gemv(W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None
         st = lib.qmm_q8_gemv(M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), _stream(stream))
     _check(st, "qmm_q8_gemv")
     return Y
+
+
+def qmm_q8_gemv_multi(Ws, X: torch.Tensor, Ns, Ys=None, *, block: int = BLOCK, flags: int = 0, stream=None):
+    """[Y_i] = [X . dequant(W_i)^T]: several Q8_0 projections of the same X in one launch."""
+    M, K = X.shape
+    k = len(Ws)
+    if Ys is None:
+        Ys = [torch.empty((M, n), dtype=torch.float32, device=X.device) for n in Ns]
+    n_arr = (ctypes.c_int64 * k)(*[int(n) for n in Ns])
+    w_arr = (ctypes.c_void_p * k)(*[_ptr(w) for w in Ws])
+    y_arr = (ctypes.c_void_p * k)(*[_ptr(y) for y in Ys])
+    _check(lib.qmm_q8_gemv_multi(M, K, block, k, n_arr, w_arr, _ptr(X), y_arr, flags, _stream(stream)),
+           "qmm_q8_gemv_multi")
+    return Ys
 
 
 def qmm_quantize_act_q8(X: torch.Tensor, QX: torch.Tensor | None = None, DX: torch.Tensor | None = None, *,

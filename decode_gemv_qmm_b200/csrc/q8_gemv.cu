@@ -1107,13 +1107,18 @@ __global__ void __launch_bounds__(256, 2) q8_gemv_mma_kernel(const __grid_consta
 //    producer warp sums the K slices of each row in slice order when the
 //    stage is released and writes Y. Deterministic.
 
+constexpr int kMaxProj = 4;  // projections of one activation vector per launch
+
 struct alignas(64) DParams {
-  const uint8_t *W;
+  // Projections (weight matrix, its rows, output) sharing X; their row chunks
+  // form one chunk space, chunk0[s] the first chunk of projection s.
+  const uint8_t *Wp[kMaxProj];
+  float *Yp[kMaxProj];
+  int64_t Np[kMaxProj];
+  int64_t chunk0[kMaxProj + 1];
+  int nproj;
   const float *X;
-  float *Y;
-  int64_t N;
   int64_t row_bytes;
-  int64_t total_bytes;
   int K, KB;
   int grid;
   int tps;        // 16-row tiles per stage (1 or 2)
@@ -1171,13 +1176,24 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   // whole chunks per CTA: a chunk costs the same however few of its rows are
   // valid, so an even split of rows (every CTA ending in a one-row chunk)
   // costs a chunk per CTA more than an even split of chunks
-  const int64_t tchunks = (p.N + kRows - 1) / kRows;
+  const int64_t tchunks = p.chunk0[p.nproj];
   const int64_t c_begin = static_cast<int64_t>(blockIdx.x) * tchunks / p.grid;
   const int64_t c_end = static_cast<int64_t>(blockIdx.x + 1) * tchunks / p.grid;
-  const int64_t r_begin = c_begin * kRows;
-  const int64_t r_end = min(p.N, c_end * kRows);
   const int nchunks = static_cast<int>(c_end - c_begin);
   const int S = p.stages;
+  // chunk c of this CTA: its projection, first row and valid rows
+  struct Chunk {
+    int proj;
+    int64_t r0;
+    int rows;
+  };
+  auto chunk = [&](int c) -> Chunk {
+    const int64_t gc = c_begin + c;
+    int sg = 0;
+    while (sg + 1 < p.nproj && gc >= p.chunk0[sg + 1]) ++sg;
+    const int64_t r0 = (gc - p.chunk0[sg]) * kRows;
+    return {sg, r0, static_cast<int>(min(static_cast<int64_t>(kRows), p.Np[sg] - r0))};
+  };
 
   pdl_launch_dependents();
   if (tid == 0) {
@@ -1196,20 +1212,20 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     uint64_t policy = 0;
     auto issue = [&](int c) {
       const int s = c % S;
-      const int64_t r0 = r_begin + static_cast<int64_t>(c) * kRows;
-      const int64_t r1 = min(r0 + kRows, r_end);
-      const int64_t b0 = r0 * p.row_bytes, b1 = r1 * p.row_bytes;
+      const Chunk ch = chunk(c);
+      const uint8_t *W = p.Wp[ch.proj];
+      const int64_t b0 = ch.r0 * p.row_bytes, b1 = (ch.r0 + ch.rows) * p.row_bytes;
       const int64_t a0 = b0 & ~int64_t(15);
       int64_t a1 = (b1 + 15) & ~int64_t(15);
-      const int64_t lim = p.total_bytes & ~int64_t(15);
+      const int64_t lim = (p.Np[ch.proj] * p.row_bytes) & ~int64_t(15);
       uint8_t *dst = stage_mem + static_cast<int64_t>(s) * p.stage_bytes;
-      if (a1 > lim) {  // last chunk of W: bytes past the last 16-byte boundary by hand
-        for (int64_t t = max(lim, a0); t < b1; ++t) dst[t - a0] = p.W[t];
+      if (a1 > lim) {  // last chunk of a matrix: bytes past its last 16-byte boundary by hand
+        for (int64_t t = max(lim, a0); t < b1; ++t) dst[t - a0] = W[t];
         a1 = max(lim, a0);
       }
       const uint32_t bytes = static_cast<uint32_t>(a1 - a0);
       mbar_arrive_expect_tx(&full[s], bytes);
-      if (bytes) bulk_g2s(dst, p.W + a0, bytes, &full[s], policy);
+      if (bytes) bulk_g2s(dst, W + a0, bytes, &full[s], policy);
     };
     const int prologue = min(S, nchunks);
     if (lane == 0) {
@@ -1225,15 +1241,17 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
       if (!ok) break;
       // rows of chunk c: sum the K slices in order, scale by 2^(E - 188) (two exact steps)
       const int s = c % S;
-      const int64_t r0 = r_begin + static_cast<int64_t>(c) * kRows;
-      const int rows = static_cast<int>(min(static_cast<int64_t>(kRows), r_end - r0));
+      const Chunk ch = chunk(c);
+      const int64_t r0 = ch.r0;
+      const int rows = ch.rows;
+      float *Y = p.Yp[ch.proj];
       const int e = *emax - 188, e1 = max(e, -120);
       const float f1 = __int_as_float((127 + e1) << 23), f2 = __int_as_float((127 + e - e1) << 23);
       const float *rb = red + s * kSlices * kRows;
       for (int r = lane; r < rows; r += 32) {
         float v = rb[r];
         for (int k = 1; k < kSlices; ++k) v += rb[k * kRows + r];
-        p.Y[r0 + r] = (v * f1) * f2;
+        Y[r0 + r] = (v * f1) * f2;
       }
       __syncwarp();
       if (lane == 0 && issued < nchunks) {
@@ -1303,8 +1321,9 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
       if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
       return;  // the producer times out on this warp's missing arrival and drains
     }
-    const int64_t r0 = r_begin + static_cast<int64_t>(c) * kRows;
-    const int rows = static_cast<int>(min(static_cast<int64_t>(kRows), r_end - r0));
+    const Chunk ch = chunk(c);
+    const int64_t r0 = ch.r0;
+    const int rows = ch.rows;
     const uint32_t base = smem_u32(stage_mem) + s * p.stage_bytes + static_cast<uint32_t>((r0 * p.row_bytes) & 15);
     const int ra = tl * 16 + g, rb = ra + 8;  // rows of this lane
     const bool oka = ra < rows, okb = rb < rows;
@@ -1704,22 +1723,33 @@ bool try_launch_mma(const DevInfo &dev, int64_t N, int K, const void *W, const f
 
 // Integer tensor-core streaming variant for M = 1, K <= 2048 and enough rows
 // for two CTAs per SM (returns false when the shape does not suit it).
-bool try_launch_digits(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, float *Y,
-                       cudaStream_t stream, uint32_t flags, qmm_status *out) {
-  if (K > 2048) return false;
-  const int grid = 2 * dev.sms;
-  if (N < static_cast<int64_t>(grid) * 32) return false;
+bool try_launch_digits(const DevInfo &dev, int nproj, const int64_t *N, const void *const *W, int K, const float *X,
+                       float *const *Y, bool single, cudaStream_t stream, uint32_t flags, qmm_status *out) {
+  if (K > 2048 || nproj < 1 || nproj > kMaxProj) return false;
   const int KB = K / 32;
   const int tps = K <= 1024 ? 2 : 1;
   DParams p{};
-  p.W = static_cast<const uint8_t *>(W);
+  int64_t chunks = 0;
+  for (int i = 0; i < nproj; ++i) {
+    p.Wp[i] = static_cast<const uint8_t *>(W[i]);
+    p.Yp[i] = Y[i];
+    p.Np[i] = N[i];
+    p.chunk0[i] = chunks;
+    chunks += (N[i] + 16 * tps - 1) / (16 * tps);
+  }
+  p.chunk0[nproj] = chunks;
+  p.nproj = nproj;
+  int grid = 2 * dev.sms;
+  if (single) {
+    if (N[0] < static_cast<int64_t>(grid) * 32) return false;  // one GEMV takes this kernel only for many rows
+  } else {
+    grid = static_cast<int>(std::min<int64_t>(grid, chunks));  // every CTA at least one chunk
+  }
+  if (grid < 1) return false;
   p.X = X;
-  p.Y = Y;
-  p.N = N;
   p.K = K;
   p.KB = KB;
   p.row_bytes = 34ll * KB;
-  p.total_bytes = N * p.row_bytes;
   p.grid = grid;
   p.tps = tps;
   p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
@@ -1771,9 +1801,25 @@ qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
     if (rows_per_cta * K >= kMmaMinSliceWeights && K <= kMmaMaxK && try_launch_mma(dev, N, K, W, X, Y, stream, flags, &st))
       return st;
     if (try_launch_resident(dev, N, K, W, X, Y, stream, flags, &st)) return st;
-    if (try_launch_digits(dev, N, K, W, X, Y, stream, flags, &st)) return st;
+    const int64_t n1[1] = {N};
+    const void *w1[1] = {W};
+    float *y1[1] = {Y};
+    if (try_launch_digits(dev, 1, n1, w1, K, X, y1, true, stream, flags, &st)) return st;
   }
   return launch_stream<kModeF32>(dev, M, N, K, W, X, nullptr, nullptr, Y, nullptr, stream, flags);
+}
+
+qmm_status launch_q8_gemv_multi(const DevInfo &dev, int M, int K, int nproj, const int64_t *N, const void *const *W,
+                                const float *X, float *const *Y, cudaStream_t stream, uint32_t flags) {
+  qmm_status st;
+  // One launch over all projections: the integer streaming kernel (M = 1, K <= 2048).
+  if (M == 1 && try_launch_digits(dev, nproj, N, W, K, X, Y, false, stream, flags, &st)) return st;
+  // Otherwise one launch per projection.
+  for (int i = 0; i < nproj; ++i) {
+    st = launch_q8_gemv(dev, M, N[i], K, W[i], X, Y[i], stream, flags);
+    if (st != QMM_OK) return st;
+  }
+  return QMM_OK;
 }
 
 qmm_status launch_q8q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,

@@ -119,6 +119,41 @@ static qmm_status q8_gemv_impl(int64_t M, int64_t N, int64_t K, int block, const
   return launch_q8_gemv(dev, static_cast<int>(M), N, static_cast<int>(K), W, X, Y, s, flags);
 }
 
+static qmm_status multi_impl(int64_t M, int64_t K, int block, int nproj, const int64_t *N, const void *const *W,
+                             const float *X, float *const *Y, uint32_t user_flags, qmm_stream_t stream) {
+  const char *fn = "qmm_q8_gemv_multi";
+  t_last_error.clear();
+  if (nproj < 1 || nproj > QMM_MAX_PROJ) return set_error(QMM_ERR_SHAPE, "%s: nproj=%d outside 1..%d", fn, nproj, QMM_MAX_PROJ);
+  if (!N || !W || !Y) return set_error(QMM_ERR_NULL, "%s: N, W and Y arrays are required", fn);
+  if (user_flags & ~uint32_t(QMM_FLAG_EARLY_WEIGHTS))
+    return set_error(QMM_ERR_SHAPE, "%s: unknown flags 0x%x", fn, user_flags);
+  int64_t n[QMM_MAX_PROJ];
+  const void *w[QMM_MAX_PROJ];
+  float *y[QMM_MAX_PROJ];
+  int k = 0;
+  for (int i = 0; i < nproj; ++i) {
+    QMM_TRY(check_shape(fn, M, N[i], K, block, QMM_MAX_DECODE_M));
+    if (N[i] == 0 || M == 0) continue;
+    QMM_TRY(check_ptr(fn, "W[i]", W[i], K > 0, 16));
+    QMM_TRY(check_ptr(fn, "Y[i]", Y[i], true, 4));
+    n[k] = N[i];
+    w[k] = W[i];
+    y[k] = Y[i];
+    ++k;
+  }
+  if (k == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "X", X, K > 0, 16));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    for (int i = 0; i < k; ++i) QMM_TRY(zero_fill(y[i], M * n[i], s));
+    return QMM_OK;
+  }
+  uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
+  return launch_q8_gemv_multi(dev, static_cast<int>(M), static_cast<int>(K), k, n, w, X, y, s, flags);
+}
+
 static qmm_status quantize_impl(int64_t M, int64_t K, int block, const float *X, int8_t *QX, float *DX,
                                 qmm_stream_t stream) {
   const char *fn = "qmm_quantize_act_q8";
@@ -245,6 +280,12 @@ QMM_API qmm_status qmm_q8_gemv(int64_t M, int64_t N, int64_t K, int block, const
 QMM_API qmm_status qmm_q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
                                   float *Y, uint32_t flags, qmm_stream_t stream) {
   return q8_gemv_impl(M, N, K, block, W, X, Y, stream, flags);
+}
+
+QMM_API qmm_status qmm_q8_gemv_multi(int64_t M, int64_t K, int block, int nproj, const int64_t *N,
+                                     const void *const *W, const float *X, float *const *Y, uint32_t flags,
+                                     qmm_stream_t stream) {
+  return multi_impl(M, K, block, nproj, N, W, X, Y, flags, stream);
 }
 
 QMM_API qmm_status qmm_quantize_act_q8(int64_t M, int64_t K, int block, const float *X, int8_t *QX, float *DX,

@@ -32,6 +32,10 @@ qmm_status cuda_check(cudaError_t e, const char *what);
 qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
                           float *Y, cudaStream_t stream, uint32_t flags);
 
+// nproj (<= 4) projections of the same X in one launch where the shape allows.
+qmm_status launch_q8_gemv_multi(const DevInfo &dev, int M, int K, int nproj, const int64_t *N, const void *const *W,
+                                const float *X, float *const *Y, cudaStream_t stream, uint32_t flags);
+
 qmm_status launch_q8q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,
                             const float *DX, float *Y, cudaStream_t stream, uint32_t flags);
 qmm_status launch_q8q8_block_dots(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,

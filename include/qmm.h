@@ -95,6 +95,8 @@ typedef enum { QMM_Q8_0 = 0, QMM_Q4_0 = 1 } qmm_wtype;
 #define QMM_MAX_DECODE_M 8
 /* Largest K of every entry point. */
 #define QMM_MAX_K 32768
+/* Most projections per qmm_q8_gemv_multi call. */
+#define QMM_MAX_PROJ 4
 
 /* Option of the *_ex entry points: start streaming the weight blocks before
  * the preceding kernel in the stream has finished (programmatic dependent
@@ -127,6 +129,30 @@ QMM_API qmm_status qmm_q8_gemv(int64_t M, int64_t N, int64_t K, int block, const
  * are QMM_ERR_SHAPE). qmm_q8_gemv(...) == qmm_q8_gemv_ex(..., 0, stream). */
 QMM_API qmm_status qmm_q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, const void *W,
                                   const float *X, float *Y, uint32_t flags, qmm_stream_t stream);
+
+/*
+ * qmm_q8_gemv_multi -- several Q8_0 projections of the same activations in
+ * one launch: Y_i = X . dequant(W_i)^T for i < nproj, each the qmm_q8_gemv
+ * product of its matrix (same formula, same tolerance).
+ *
+ * "LSE v0.4.15", section "Changes" (several projections fed by one shared
+ * activation producer in one launch, instead of one launch per projection).
+ * At M = 1 and K <= 2048 the row chunks of all matrices form one work list
+ * of a single launch of the integer tensor-core streaming kernel; otherwise
+ * the call issues one qmm_q8_gemv launch per projection.
+ *
+ *   M         1 .. QMM_MAX_DECODE_M (0 = empty call)
+ *   K         shared row length (multiple of 32)
+ *   nproj     1 .. QMM_MAX_PROJ
+ *   N, W, Y   HOST arrays of nproj entries: rows of projection i, its
+ *             N[i] * K/32 Q8_0 blocks (device, 16-byte aligned) and its
+ *             M x N[i] fp32 output (device); N[i] = 0 skips projection i
+ *   X         M x K fp32 (device, 16-byte aligned)
+ *   flags     0 or QMM_FLAG_EARLY_WEIGHTS
+ */
+QMM_API qmm_status qmm_q8_gemv_multi(int64_t M, int64_t K, int block, int nproj, const int64_t *N,
+                                     const void *const *W, const float *X, float *const *Y, uint32_t flags,
+                                     qmm_stream_t stream);
 
 /*
  * qmm_quantize_act_q8 -- quantise fp32 activations to Q8 codes per 32-block.

@@ -19,7 +19,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     names = declared_symbols()
-    assert len(names) >= 14
+    assert len(names) >= 15
     for name in names:
         assert hasattr(lib, name), f"{name} declared in include/qmm.h but not exported"
 
@@ -86,3 +86,28 @@ def test_python_binding_raises_with_status():
     with pytest.raises(qmm.QmmError) as e:
         qmm.qmm_q8_gemv(torch.zeros(10, dtype=torch.uint8), torch.zeros(1, 33), 4, torch.zeros(1, 4), stream=0)
     assert e.value.status == qmm.QMM_ERR_SHAPE
+
+
+def test_multi_argument_errors_before_any_cuda_call():
+    i64, vp = ctypes.c_int64, ctypes.c_void_p
+    N = (i64 * 2)(8, 8)
+    W = (vp * 2)(P16, P16)
+    Y = (vp * 2)(P16, P16)
+    W_odd = (vp * 2)(P16, P_ODD)
+    Y_null = (vp * 2)(P16, 0)
+    cases = [
+        (lambda: lib.qmm_q8_gemv_multi(1, 64, 32, 0, N, W, P16, Y, 0, 0), "QMM_ERR_SHAPE"),
+        (lambda: lib.qmm_q8_gemv_multi(1, 64, 32, 5, N, W, P16, Y, 0, 0), "QMM_ERR_SHAPE"),
+        (lambda: lib.qmm_q8_gemv_multi(1, 64, 32, 2, None, W, P16, Y, 0, 0), "QMM_ERR_NULL"),
+        (lambda: lib.qmm_q8_gemv_multi(1, 64, 32, 2, N, W_odd, P16, Y, 0, 0), "QMM_ERR_ALIGN"),
+        (lambda: lib.qmm_q8_gemv_multi(1, 64, 32, 2, N, W, P16, Y_null, 0, 0), "QMM_ERR_NULL"),
+        (lambda: lib.qmm_q8_gemv_multi(1, 64, 32, 2, N, W, 0, Y, 0, 0), "QMM_ERR_NULL"),
+        (lambda: lib.qmm_q8_gemv_multi(9, 64, 32, 2, N, W, P16, Y, 0, 0), "QMM_ERR_SHAPE"),
+        (lambda: lib.qmm_q8_gemv_multi(1, 64, 16, 2, N, W, P16, Y, 0, 0), "QMM_ERR_BLOCK"),
+        (lambda: lib.qmm_q8_gemv_multi(1, 64, 32, 2, N, W, P16, Y, 4, 0), "QMM_ERR_SHAPE"),
+    ]
+    for call, expect in cases:
+        assert st_name(call()) == expect, lib.qmm_last_error_string()
+    zero = (i64 * 2)(0, 0)
+    assert lib.qmm_q8_gemv_multi(1, 64, 32, 2, zero, W, 0, Y, 0, 0) == 0  # nothing to do
+    assert lib.qmm_q8_gemv_multi(0, 64, 32, 2, N, W, 0, Y, 0, 0) == 0     # M = 0
