@@ -381,6 +381,35 @@ def component_gateup(qmm, dev_peak_gbs, m=8, n=17408, k=5120, reps=10):
     return out
 
 
+def component_q4_gemv(qmm, dev_peak_gbs, reps=10):
+    """Q4_0 GEMV (one projection): M=1 at K=5120, N=17408 and the M=8 down
+    projection K=17408, N=5120; three rotating weight copies (> L2) in a chain."""
+    import torch
+
+    out = {}
+    g = syn.rng(5)
+    for name, m, n, k in (("m1_k5120_n17408", 1, 17408, 5120), ("m8_k17408_n5120", 8, 5120, 17408)):
+        Ws = [torch.from_numpy(syn.q4_0_weights(g, n, k)[0]).cuda() for _ in range(3)]
+        x = torch.from_numpy(syn.act_f32(g, m, k)).cuda()
+        Y = torch.empty(m, n, device="cuda")
+        s = torch.cuda.Stream()
+
+        def fn(h):
+            for w in Ws:
+                assert qmm.lib.qmm_q4_gemv(m, n, k, 32, w.data_ptr(), x.data_ptr(), Y.data_ptr(),
+                                           qmm.QMM_FLAG_EARLY_WEIGHTS, h) == 0
+        fn(s.cuda_stream)
+        torch.cuda.synchronize()
+        gr = capture(fn, s)
+        time_graph(gr, s, 3)
+        ms = time_graph(gr, s, reps) / len(Ws)
+        bytes_ = n * (k // 32) * 18 + m * k * 4 + m * n * 4
+        out[name] = {"us": round(ms * 1e3, 2), "GB_s": round(bytes_ / ms / 1e6, 1),
+                     "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4), "bytes": bytes_}
+        del gr, Ws
+    return out
+
+
 def component_q8q8(qmm, dev_peak_gbs, reps_graph=4):
     """Q8xQ8 decode GEMV (M=1) at K=896/N=4864 and K=4864/N=896: the GEMV on
     quantized activations alone, activation quantization + GEMV as two launches
@@ -769,6 +798,7 @@ def main(argv=None):
                       "single_gemv_896x1152": component_single_gemv(qmm, pk["hbm_gbs"]),
                       "q4_gateup_m8_k5120_n17408": component_gateup(qmm, pk["hbm_gbs"]),
                       "q8q8_gemv": component_q8q8(qmm, pk["hbm_gbs"]),
+                      "q4_gemv": component_q4_gemv(qmm, pk["hbm_gbs"]),
                       "prefill": component_prefill(qmm, pk)}
 
     cpu = None

@@ -40,6 +40,7 @@ _SIGS = {
     "qmm_quantize_act_q8": [_i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q8q8_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_q8q8_gemv_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
+    "qmm_q4_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _u32, _p],
     "qmm_q8_gemv_multi": [_i64, _i64, _int, _int, _p, _p, _p, _p, _u32, _p],
     "qmm_q8q8_gemv_fused": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _u32, _p],
     "qmm_q4_swiglu_gateup": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
@@ -177,6 +178,15 @@ def qmm_q8q8_block_dots(W: torch.Tensor, QX: torch.Tensor, N: int, isum: torch.T
     _check(lib.qmm_q8q8_block_dots(M, N, K, block, _ptr(W), _ptr(QX), _ptr(isum), _stream(stream)),
            "qmm_q8q8_block_dots")
     return isum
+
+
+def qmm_q4_gemv(W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None = None, *,
+                block: int = BLOCK, flags: int = 0, stream=None) -> torch.Tensor:
+    """Y[M, N] = X[M, K] . dequant(W)^T for Q4_0 blocks W (uint8, N*K/32*18 bytes)."""
+    M, K = X.shape
+    Y = _out(Y, (M, N), X.device)
+    _check(lib.qmm_q4_gemv(M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), flags, _stream(stream)), "qmm_q4_gemv")
+    return Y
 
 
 def qmm_q4_swiglu_gateup(Wg: torch.Tensor, Wu: torch.Tensor, X: torch.Tensor, N: int,

@@ -81,7 +81,29 @@ struct alignas(64) Params {
   int grid;
   int nmat;              // 2 (fused) or 1 (projection)
   int prefetch_before_wait;
+  int split;             // K ranges per tile group (cluster size along x; 1 = none)
 };
+
+// ------------------------------------------------------------ cluster PTX
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of all CTAs of the cluster; orders shared-memory accesses across it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -182,6 +204,42 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
 }
 
+// Outputs o in [o_begin, o_end) (o = token * rows + row of the CTA's tiles) from
+// the partial sums red[warp][tile of the warp][mat][lane] (float4) of `nsrc`
+// CTAs of a cluster (nsrc = 1: this CTA's own): the eight block warps of a
+// tile in block order, ranks in rank order; then the SwiGLU (NMAT = 2) or the
+// projection itself.
+template <int NMAT>
+__device__ __forceinline__ void finish_outputs(const Params &p, uint32_t red_saddr, int nsrc, int tile0, int ntiles,
+                                               int tid, int nthreads, int o_begin, int o_end) {
+  const int rows = ntiles * 16;
+  for (int o = o_begin + tid; o < o_end; o += nthreads) {
+    const int tok = o / rows, rl = o - tok * rows;
+    const int i = rl >> 4, r = rl & 15;
+    const int src_lane = (r & 7) * 4 + (tok >> 1), idx = (r >> 3) * 2 + (tok & 1);
+    float v[2] = {0.f, 0.f};
+#pragma unroll
+    for (int mat = 0; mat < NMAT; ++mat) {
+      float sum = 0.f;
+      // the eight block warps that hold tile i, in block order
+      const int wbase = 8 * (i % kHalves), ii = i / kHalves;
+      for (int src = 0; src < nsrc; ++src) {
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          const uint32_t off =
+              4u * static_cast<uint32_t>(((((wbase + b) * (kTilesMax / kHalves) + ii) * 2 + mat) * 32 + src_lane) * 4 + idx);
+          const float x = nsrc == 1 ? *reinterpret_cast<const float *>(__cvta_shared_to_generic(red_saddr + off))
+                                    : ld_cluster_f32(map_rank(red_saddr + off, static_cast<uint32_t>(src)));
+          sum = __fadd_rn(sum, x);
+        }
+      }
+      v[mat] = sum;
+    }
+    const int64_t n = 16ll * tile0 + rl;
+    if (tok < p.M && n < p.N) p.Y[static_cast<int64_t>(tok) * p.N + n] = (NMAT == 2) ? silu_mul(v[0], v[1]) : v[0];
+  }
+}
+
 // DIRECT = false: TMA-fed shared-memory stages; true: reads global memory.
 // NMAT: 2 (fused gate/up) or 1 (one projection).
 template <bool DIRECT, int NMAT>
@@ -193,10 +251,18 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
   uint8_t *stages = smem + kBarBytes;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tile0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * p.tiles / p.grid);
-  const int tile1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * p.tiles / p.grid);
+  // Split K (few row tiles, long rows): the `split` CTAs of a cluster share a
+  // tile group and take consecutive stage ranges; their partial sums are added
+  // in rank order through distributed shared memory at the end.
+  const int split = DIRECT ? 1 : p.split;
+  const int rank = split > 1 ? static_cast<int>(cluster_rank()) : 0;
+  const int group = static_cast<int>(blockIdx.x) / split;
+  const int tile0 = static_cast<int>(static_cast<int64_t>(group) * p.tiles / p.grid);
+  const int tile1 = static_cast<int>(static_cast<int64_t>(group + 1) * p.tiles / p.grid);
   const int ntiles = tile1 - tile0;
-  const int nstages = (p.KB + kBlocksPerStage - 1) / kBlocksPerStage;
+  const int nstages_all = (p.KB + kBlocksPerStage - 1) / kBlocksPerStage;
+  const int j_lo = rank * nstages_all / split;
+  const int nstages = (rank + 1) * nstages_all / split - j_lo;  // this CTA's stages
 
   pdl_launch_dependents();
   if (!DIRECT) {
@@ -220,13 +286,13 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
       mbar_arrive_expect_tx(&full[s], wbytes + kXStageBytes);
       for (int mat = 0; mat < NMAT; ++mat)
         for (int t = 0; t < ntiles; ++t)
-          tma_load_2d(st + kXStageBytes + (mat * kTilesMax + t) * kTileBytes, &p.tm_w[mat], 72 * j,
+          tma_load_2d(st + kXStageBytes + (mat * kTilesMax + t) * kTileBytes, &p.tm_w[mat], 72 * (j_lo + j),
                       16 * (tile0 + t), &full[s]);
     };
     auto issue_x = [&](int j) {
       uint8_t *st = stages + (j % kStages) * kStageBytes;
       for (int b = 0; b < kBlocksPerStage; ++b)
-        tma_load_2d(st + b * 1024, &p.tm_x, 32 * (j * kBlocksPerStage + b), 0, &full[j % kStages]);
+        tma_load_2d(st + b * 1024, &p.tm_x, 32 * ((j_lo + j) * kBlocksPerStage + b), 0, &full[j % kStages]);
     };
     const int prologue = min(kStages, nstages);
     if (lane == 0) {
@@ -257,9 +323,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
             atomicOr(&g_q4_status, kDevTimeoutDrain);
       }
     }
-    return;
-  }
-
+    __syncwarp();
+    if (split == 1) return;
+  } else {
   // ---------------------------------------------------------------- consumers
   pdl_wait();
   const int g = lane >> 2, t = lane & 3;
@@ -277,9 +343,10 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
     const int s = j % kStages;
     if (!DIRECT && !mbar_wait(&full[s], static_cast<uint32_t>(j / kStages) & 1u)) {
       if (lane == 0) atomicOr(&g_q4_status, kDevTimeoutFull);
-      return;  // the producer gives up on this warp's missing arrival and drains
+      if (split == 1) return;  // the producer gives up on this warp's missing arrival and drains
+      break;                   // split K: still meet the cluster barriers
     }
-    const int kb = j * kBlocksPerStage + wb;  // this warp's block
+    const int kb = (j_lo + j) * kBlocksPerStage + wb;  // this warp's block
     if (kb < p.KB) {
       // activations of block kb for token g
       float4 x0, x1;
@@ -360,25 +427,20 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
     }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
-  const float *redf = reinterpret_cast<const float *>(red);
-  const int rows = ntiles * 16;
-  for (int o = tid; o < 8 * rows; o += kWarps * 32) {
-    const int tok = o / rows, rl = o - tok * rows;
-    const int i = rl >> 4, r = rl & 15;
-    const int src_lane = (r & 7) * 4 + (tok >> 1), idx = (r >> 3) * 2 + (tok & 1);
-    float v[2] = {0.f, 0.f};
-    for (int mat = 0; mat < NMAT; ++mat) {
-      float sum = 0.f;
-      // the eight block warps that hold tile i, in block order
-      const int wbase = 8 * (i % kHalves), ii = i / kHalves;
-#pragma unroll
-      for (int b = 0; b < 8; ++b)
-        sum = __fadd_rn(sum, redf[((((wbase + b) * (kTilesMax / kHalves) + ii) * 2 + mat) * 32 + src_lane) * 4 + idx]);
-      v[mat] = sum;
-    }
-    const int64_t n = 16ll * tile0 + rl;
-    if (tok < p.M && n < p.N) p.Y[static_cast<int64_t>(tok) * p.N + n] = (NMAT == 2) ? silu_mul(v[0], v[1]) : v[0];
+  if (split == 1) {
+    finish_outputs<NMAT>(p, smem_u32(red), 1, tile0, ntiles, tid, kWarps * 32, 0, 8 * ntiles * 16);
+    return;
   }
+  }  // consumers
+
+  // Split K: every rank's partials are in its own shared memory; rank r adds
+  // all ranks' partials (rank order, then block order) for its share of the
+  // outputs, then no rank leaves while another may still read its memory.
+  cluster_sync();
+  const int nout = 8 * ntiles * 16;
+  finish_outputs<NMAT>(p, smem_u32(stages), split, tile0, ntiles, tid, (kWarps + 1) * 32, rank * nout / split,
+                       (rank + 1) * nout / split);
+  cluster_sync();
 }
 
 __global__ void silu_mul_kernel(const float *__restrict__ G, const float *__restrict__ U, float *__restrict__ Y,
@@ -423,6 +485,16 @@ qmm_status launch_proj(const DevInfo &dev, int M, int64_t N, int K, const void *
   p.tiles = static_cast<int>(tiles);
   p.grid = static_cast<int>(std::max<int64_t>(std::min<int64_t>(tiles, dev.sms), (tiles + kTilesMax - 1) / kTilesMax));
   const bool direct = (p.KB % kBlocksPerStage) != 0;
+  // Split K when full tile groups leave at least half of the SMs idle (few
+  // rows, long K): groups of kTilesMax tiles, `split` CTAs per group.
+  p.split = 1;
+  const int64_t groups = (tiles + kTilesMax - 1) / kTilesMax;
+  const int nstages_all = (p.KB + kBlocksPerStage - 1) / kBlocksPerStage;
+  if (!direct && 2 * groups <= dev.sms) {
+    p.split = static_cast<int>(std::min<int64_t>({8, dev.sms / groups, nstages_all}));
+    if (p.split > 1) p.grid = static_cast<int>(groups);
+    else p.split = 1;
+  }
   if (!direct) {
     const uint64_t xd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
     const uint64_t xs[1] = {static_cast<uint64_t>(K) * 4};
@@ -439,16 +511,20 @@ qmm_status launch_proj(const DevInfo &dev, int M, int64_t N, int K, const void *
     }
   }
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(p.grid);
+  cfg.gridDim = dim3(p.grid * p.split);
   cfg.blockDim = dim3((kWarps + 1) * 32);
   cfg.dynamicSmemBytes = direct ? static_cast<size_t>(kWarps * (kTilesMax / kHalves) * 2 * 32 * 16 + 2048)
                                 : static_cast<size_t>(kBarBytes + kStages * kStageBytes + 1024);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(p.split);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.split > 1 ? 2 : 1;
   const cudaError_t e = nmat == 2 ? (direct ? launch<true, 2>(cfg, p) : launch<false, 2>(cfg, p))
                                   : (direct ? launch<true, 1>(cfg, p) : launch<false, 1>(cfg, p));
   return cuda_check(e, "q4_gateup launch");
@@ -460,6 +536,12 @@ qmm_status launch_q4_gateup(const DevInfo &dev, int M, int64_t N, int K, const v
                             const float *X, float *Y, cudaStream_t stream, uint32_t flags) {
   const void *W[2] = {Wg, Wu};
   return launch_proj(dev, M, N, K, W, 2, X, Y, stream, flags);
+}
+
+qmm_status launch_q4_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
+                          cudaStream_t stream, uint32_t flags) {
+  const void *Wp[1] = {W};
+  return launch_proj(dev, M, N, K, Wp, 1, X, Y, stream, flags);
 }
 
 qmm_status launch_q4_gateup_unfused(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,

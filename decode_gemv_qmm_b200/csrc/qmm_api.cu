@@ -215,6 +215,25 @@ static qmm_status q8q8_fused_impl(int64_t M, int64_t N, int64_t K, int block, co
   return launch_q8q8_gemv_fused(dev, static_cast<int>(M), N, static_cast<int>(K), W, X, QX, DX, Y, s, flags);
 }
 
+static qmm_status q4_gemv_impl(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X, float *Y,
+                               uint32_t user_flags, qmm_stream_t stream) {
+  const char *fn = "qmm_q4_gemv";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, N, K, block, QMM_MAX_DECODE_M));
+  if (user_flags & ~uint32_t(QMM_FLAG_EARLY_WEIGHTS))
+    return set_error(QMM_ERR_SHAPE, "%s: unknown flags 0x%x", fn, user_flags);
+  if (M == 0 || N == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "W", W, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "X", X, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "Y", Y, true, 4));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return zero_fill(Y, M * N, s);
+  uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
+  return launch_q4_gemv(dev, static_cast<int>(M), N, static_cast<int>(K), W, X, Y, s, flags);
+}
+
 static qmm_status gateup_impl(int64_t M, int64_t N, int64_t K, int block, const void *Wg, const void *Wu,
                               const float *X, float *G, float *U, float *Y, qmm_stream_t stream, bool unfused,
                               uint32_t user_flags) {
@@ -322,6 +341,11 @@ QMM_API qmm_status qmm_q4_swiglu_gateup_ex(int64_t M, int64_t N, int64_t K, int 
                                            const void *Wu, const float *X, float *Y, uint32_t flags,
                                            qmm_stream_t stream) {
   return gateup_impl(M, N, K, block, Wg, Wu, X, nullptr, nullptr, Y, stream, false, flags);
+}
+
+QMM_API qmm_status qmm_q4_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X, float *Y,
+                               uint32_t flags, qmm_stream_t stream) {
+  return q4_gemv_impl(M, N, K, block, W, X, Y, flags, stream);
 }
 
 QMM_API qmm_status qmm_q4_gateup_unfused(int64_t M, int64_t N, int64_t K, int block, const void *Wg, const void *Wu,

@@ -47,6 +47,9 @@ qmm_status launch_quantize_act_q8(const DevInfo &dev, int64_t M, int K, const fl
 
 qmm_status launch_q4_gateup(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
                             const float *X, float *Y, cudaStream_t stream, uint32_t flags);
+// One Q4_0 projection Y = X . dequant(W)^T (the gate/up kernel with one matrix).
+qmm_status launch_q4_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
+                          cudaStream_t stream, uint32_t flags);
 qmm_status launch_q4_gateup_unfused(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
                                     const float *X, float *G, float *U, float *Y, cudaStream_t stream);
 

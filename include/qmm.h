@@ -243,6 +243,29 @@ QMM_API qmm_status qmm_q4_swiglu_gateup_ex(int64_t M, int64_t N, int64_t K, int 
                                            qmm_stream_t stream);
 
 /*
+ * qmm_q4_gemv -- decode GEMV / small-M matmul on Q4_0 weights, fp32 activations.
+ *
+ * The Q4_0 counterpart of qmm_q8_gemv, for the rest of a Q4 model's matmul
+ * set: the M8 Q4 down projection that "LSE v0.4.16" keeps on its matrix
+ * cores (section "Retained optimizations and compatibility") and the Q4-native
+ * matmul that "Lumen v0.5.0" lists in its section "What's next":
+ *
+ *   Y[m][n] = sum_b d[n][b] * sum_j (q[n][b][j] - 8) * X[m][32b + j]   (fp32 accumulation)
+ *
+ * It runs the fused gate/up kernel with one matrix, so each output equals
+ * the corresponding gate (or up) projection of qmm_q4_swiglu_gateup's
+ * unfused form bit for bit.
+ *
+ *   M      1 .. QMM_MAX_DECODE_M (0 = empty call)
+ *   W      N * K/32 Q4_0 blocks (16-byte aligned)
+ *   X      M x K fp32 (16-byte aligned)
+ *   Y      M x N fp32 (written)
+ *   flags  0 or QMM_FLAG_EARLY_WEIGHTS
+ */
+QMM_API qmm_status qmm_q4_gemv(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
+                               float *Y, uint32_t flags, qmm_stream_t stream);
+
+/*
  * qmm_quant_matmul_prefill -- prefill panel Y = X . W^T on the tensor cores.
  *
  * "LSE v0.4.16", section "Retained optimizations and compatibility" (M1024
