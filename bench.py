@@ -218,6 +218,19 @@ class DecodeStep:
                 raise qmm.QmmError(st, "qmm_q8_gemv_ex")
             i += 1
 
+    def launch_auto(self, qmm, stream_handle: int, flags: int, qx, dx):
+        """The same matmul set through qmm_q8_gemv_auto: short-K GEMVs whose
+        slices fit on chip as fused Q8xQ8 (quantised activations), the rest fp32.
+        qx / dx: scratch for the codes and scales (largest K)."""
+        lib = qmm.lib
+        xp, yp = self.X.data_ptr(), self.Y.data_ptr()
+        for i, (_, n, k) in enumerate(self.shapes):
+            st = lib.qmm_q8_gemv_auto(1, n, k, 32, self.W[i].data_ptr(), xp + 4 * int(self.x_offsets[i]),
+                                      yp + 4 * int(self.y_offsets[i]), qx.data_ptr(), dx.data_ptr(), flags,
+                                      stream_handle)
+            if st != 0:
+                raise qmm.QmmError(st, "qmm_q8_gemv_auto")
+
     def logits(self):
         return self.Y[int(self.y_offsets[-2]):int(self.y_offsets[-1])]
 
@@ -339,6 +352,29 @@ def component_step_multi(qmm, step: DecodeStep, dev_peak_gbs, reps=200):
     bytes_ = sum(n * (k // 32) * 34 + k * 4 + n * 4 for _, n, k in step.shapes)
     return {"ms_per_step": round(ms, 5), "tok_s": round(1e3 / ms, 2), "launches": 97,
             "GB_s": round(bytes_ / ms / 1e6, 1), "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4)}
+
+
+def component_step_auto(qmm, step: DecodeStep, dev_peak_gbs, reps=200):
+    """The decode step's matmul set through the per-K choice (qmm_q8_gemv_auto):
+    short-K GEMVs as fused Q8xQ8 on quantised activations, long-K ones fp32 --
+    a different numerical contract from the headline's fp32 activations."""
+    import torch
+
+    kmax = max(k for _, _, k in step.shapes)
+    qx = torch.empty(kmax, dtype=torch.int8, device="cuda")
+    dx = torch.empty(kmax // 32, device="cuda")
+    s = torch.cuda.Stream()
+    flags = qmm.QMM_FLAG_EARLY_WEIGHTS
+    step.launch_auto(qmm, s.cuda_stream, flags, qx, dx)
+    torch.cuda.synchronize()
+    gr = capture(lambda h: step.launch_auto(qmm, h, flags, qx, dx), s)
+    time_graph(gr, s, 20)
+    ms = time_graph(gr, s, reps)
+    del gr
+    bytes_ = sum(n * (k // 32) * 34 + k * 4 + n * 4 for _, n, k in step.shapes)
+    return {"ms_per_step": round(ms, 5), "tok_s": round(1e3 / ms, 2),
+            "GB_s": round(bytes_ / ms / 1e6, 1), "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4),
+            "note": "qkv, wo, gate, up as fused Q8xQ8 (quantised activations); down and lm_head fp32"}
 
 
 def component_gateup(qmm, dev_peak_gbs, m=8, n=17408, k=5120, reps=10):
@@ -795,6 +831,7 @@ def main(argv=None):
     if rank == 0 and world == 1 and not args.no_components:
         components = {"lm_head_896x151936": component_lm_head(qmm, step, pk["hbm_gbs"]),
                       "decode_step_gate_up_multi": component_step_multi(qmm, step, pk["hbm_gbs"]),
+                      "decode_step_per_k_q8q8": component_step_auto(qmm, step, pk["hbm_gbs"]),
                       "single_gemv_896x1152": component_single_gemv(qmm, pk["hbm_gbs"]),
                       "q4_gateup_m8_k5120_n17408": component_gateup(qmm, pk["hbm_gbs"]),
                       "q8q8_gemv": component_q8q8(qmm, pk["hbm_gbs"]),

@@ -40,6 +40,7 @@ _SIGS = {
     "qmm_quantize_act_q8": [_i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q8q8_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_q8q8_gemv_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
+    "qmm_q8_gemv_auto": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _u32, _p],
     "qmm_q4_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _u32, _p],
     "qmm_q8_gemv_multi": [_i64, _i64, _int, _int, _p, _p, _p, _p, _u32, _p],
     "qmm_q8q8_gemv_fused": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _u32, _p],
@@ -118,6 +119,19 @@ def qmm_q8_gemv(W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None
         st = lib.qmm_q8_gemv(M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), _stream(stream))
     _check(st, "qmm_q8_gemv")
     return Y
+
+
+def qmm_q8_gemv_auto(W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None = None,
+                     QX: torch.Tensor | None = None, DX: torch.Tensor | None = None, *, block: int = BLOCK,
+                     flags: int = 0, stream=None):
+    """(Y, QX, DX): the Q8xQ8 GEMV for short K (activations quantised), else the fp32 GEMV."""
+    M, K = X.shape
+    Y = _out(Y, (M, N), X.device)
+    QX = _out(QX, (M, K), X.device, torch.int8)
+    DX = _out(DX, (M, K // BLOCK), X.device)
+    _check(lib.qmm_q8_gemv_auto(M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), _ptr(QX), _ptr(DX), flags,
+                                _stream(stream)), "qmm_q8_gemv_auto")
+    return Y, QX, DX
 
 
 def qmm_q8_gemv_multi(Ws, X: torch.Tensor, Ns, Ys=None, *, block: int = BLOCK, flags: int = 0, stream=None):

@@ -1809,6 +1809,18 @@ qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
   return launch_stream<kModeF32>(dev, M, N, K, W, X, nullptr, nullptr, Y, nullptr, stream, flags);
 }
 
+// Short rows (at most 64 blocks) at M = 1: the fused Q8xQ8 form when its
+// weight slice fits on chip; everything else the fp32-activation GEMV.
+constexpr int kAutoMaxKBlocks = 64;
+
+qmm_status launch_q8_gemv_auto(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
+                               int8_t *QX, float *DX, cudaStream_t stream, uint32_t flags) {
+  qmm_status st;
+  if (M == 1 && K / 32 <= kAutoMaxKBlocks && try_launch_q8q8_resident(dev, N, K, W, X, QX, DX, Y, stream, flags, &st))
+    return st;
+  return launch_q8_gemv(dev, M, N, K, W, X, Y, stream, flags);
+}
+
 qmm_status launch_q8_gemv_multi(const DevInfo &dev, int M, int K, int nproj, const int64_t *N, const void *const *W,
                                 const float *X, float *const *Y, cudaStream_t stream, uint32_t flags) {
   qmm_status st;

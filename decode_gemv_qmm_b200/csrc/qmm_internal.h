@@ -32,6 +32,9 @@ qmm_status cuda_check(cudaError_t e, const char *what);
 qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
                           float *Y, cudaStream_t stream, uint32_t flags);
 
+// Per-K choice between the fused Q8xQ8 form (short rows) and the fp32 GEMV.
+qmm_status launch_q8_gemv_auto(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
+                               int8_t *QX, float *DX, cudaStream_t stream, uint32_t flags);
 // nproj (<= 4) projections of the same X in one launch where the shape allows.
 qmm_status launch_q8_gemv_multi(const DevInfo &dev, int M, int K, int nproj, const int64_t *N, const void *const *W,
                                 const float *X, float *const *Y, cudaStream_t stream, uint32_t flags);

@@ -131,6 +131,27 @@ QMM_API qmm_status qmm_q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, co
                                   const float *X, float *Y, uint32_t flags, qmm_stream_t stream);
 
 /*
+ * qmm_q8_gemv_auto -- the per-K choice between the fp32-activation GEMV and
+ * the Q8xQ8 GEMV ("Lumen v0.4.0", section "Phase 7.P -- per-shape hybrid
+ * dispatch": short-K matmuls on the quantised-activation integer path, long-K
+ * ones on the fp32 path). Opt-in: the result depends on K.
+ *
+ * At M = 1 with K/32 <= 64 blocks, when each CTA's weight slice fits on chip,
+ * this is qmm_q8q8_gemv_fused (Y is the Q8xQ8 product of the activations
+ * quantised per 32-block, and QX / DX receive their codes and scales);
+ * otherwise it is qmm_q8_gemv_ex (fp32 activations; QX / DX untouched). The
+ * rule was measured on B200 in chains of dependent launches: 896 -> 4864
+ * takes 2.09 us as Q8xQ8 and 2.81 us as fp32; 4864 -> 896 takes 3.56 us and
+ * 3.39 us.
+ *
+ *   M, N, K, block, W, X, Y, flags   as qmm_q8_gemv_ex
+ *   QX, DX   M x K int8 (16-byte aligned) and M x K/32 fp32, caller-owned
+ *            (always required; written only by the Q8xQ8 form)
+ */
+QMM_API qmm_status qmm_q8_gemv_auto(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
+                                    float *Y, int8_t *QX, float *DX, uint32_t flags, qmm_stream_t stream);
+
+/*
  * qmm_q8_gemv_multi -- several Q8_0 projections of the same activations in
  * one launch: Y_i = X . dequant(W_i)^T for i < nproj, each the qmm_q8_gemv
  * product of its matrix (same formula, same tolerance).
