@@ -40,6 +40,8 @@ _SIGS = {
     "qmm_quantize_act_q8": [_i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q8q8_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_q8q8_gemv_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
+    "qmm_quantize_act_q8_0": [_i64, _i64, _int, _p, _p, _p],
+    "qmm_q8q8_gemv_q8_0": [_i64, _i64, _i64, _int, _p, _p, _p, _u32, _p],
     "qmm_q8_gemv_auto": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _u32, _p],
     "qmm_q4_gemv": [_i64, _i64, _i64, _int, _p, _p, _p, _u32, _p],
     "qmm_q8_gemv_multi": [_i64, _i64, _int, _int, _p, _p, _p, _p, _u32, _p],
@@ -118,6 +120,24 @@ def qmm_q8_gemv(W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None
     else:
         st = lib.qmm_q8_gemv(M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), _stream(stream))
     _check(st, "qmm_q8_gemv")
+    return Y
+
+
+def qmm_quantize_act_q8_0(X: torch.Tensor, XB: torch.Tensor | None = None, *, block: int = BLOCK, stream=None):
+    """XB uint8[M, K/32*34]: X quantised into ggml Q8_0 blocks (fp16 scale, ggml rule)."""
+    M, K = X.shape
+    XB = _out(XB, (M, (K // BLOCK) * 34), X.device, torch.uint8)
+    _check(lib.qmm_quantize_act_q8_0(M, K, block, _ptr(X), _ptr(XB), _stream(stream)), "qmm_quantize_act_q8_0")
+    return XB
+
+
+def qmm_q8q8_gemv_q8_0(W: torch.Tensor, XB: torch.Tensor, K: int, N: int, Y: torch.Tensor | None = None, *,
+                       block: int = BLOCK, flags: int = 0, stream=None) -> torch.Tensor:
+    """Y[M, N] from Q8_0 weights W and Q8_0 activation blocks XB (M rows of K/32 blocks)."""
+    M = XB.shape[0]
+    Y = _out(Y, (M, N), XB.device)
+    _check(lib.qmm_q8q8_gemv_q8_0(M, N, K, block, _ptr(W), _ptr(XB), _ptr(Y), flags, _stream(stream)),
+           "qmm_q8q8_gemv_q8_0")
     return Y
 
 

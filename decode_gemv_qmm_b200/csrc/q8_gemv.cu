@@ -72,6 +72,7 @@ struct alignas(64) Params {
   const float *X;    // fp32 activations (kModeF32)
   const int8_t *QX;  // int8 activation codes (kModeQ8, kModeQ8Dots)
   const float *DX;   // per-block activation scales (kModeQ8)
+  const uint8_t *XB; // kModeQ8 alternative to QX / DX: activations as Q8_0 blocks (fp16 scale)
   float *Y;
   int32_t *isum;     // block dots out (kModeQ8Dots)
   int64_t N;
@@ -369,7 +370,16 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
           for (int j = 0; j < 16; ++j) x2[m][j] = make_float2(0.f, 0.f);
         }
       } else {
-        if (valid) {
+        if (valid && MODE == kModeQ8 && p.XB) {
+          // a Q8_0 activation block: the fp16 scale, then the 32 codes as 16
+          // half-words (2-byte aligned: exactly the block's 34 bytes are read)
+          const uint16_t *bp =
+              reinterpret_cast<const uint16_t *>(p.XB + (static_cast<int64_t>(m0 + m) * p.KB + c) * 34);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            qx[m][j] = static_cast<uint32_t>(__ldg(bp + 1 + 2 * j)) | (static_cast<uint32_t>(__ldg(bp + 2 + 2 * j)) << 16);
+          dxr[m] = half_bits_to_float(__ldg(bp));
+        } else if (valid) {
           const int64_t off = static_cast<int64_t>(m0 + m) * p.K + 32 * c;
           uint4 lo, hi;
           if (xs) {
@@ -1389,12 +1399,14 @@ namespace {
 
 template <int MODE>
 qmm_status launch_stream(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, const int8_t *QX,
-                         const float *DX, float *Y, int32_t *isum, cudaStream_t stream, uint32_t flags) {
+                         const float *DX, float *Y, int32_t *isum, cudaStream_t stream, uint32_t flags,
+                         const uint8_t *XB = nullptr) {
   Params p{};
   p.W = static_cast<const uint8_t *>(W);
   p.X = X;
   p.QX = QX;
   p.DX = DX;
+  p.XB = XB;
   p.Y = Y;
   p.isum = isum;
   p.N = N;
@@ -1435,7 +1447,7 @@ qmm_status launch_stream(const DevInfo &dev, int M, int64_t N, int K, const void
   p.stages = S;
   const int red_bytes = p.cg > 1 ? S * M * p.cg * p.rows_chunk * 4 : 0;
   const int64_t xs_bytes = static_cast<int64_t>(M) * K * (MODE == kModeF32 ? 4 : 1);
-  const bool panel = xs_bytes <= kPanelBytes;
+  const bool panel = xs_bytes <= kPanelBytes && XB == nullptr;  // block-form activations: read directly
   p.xs_off = panel ? align_up(kBarBytes + red_bytes, 1024) : 0;  // 128-byte swizzle needs 1024-byte alignment
   p.xs_rows = panel ? static_cast<int>(xs_bytes / 128) : 0;
   p.xs_bytes = panel ? static_cast<int>(xs_bytes) : 0;
@@ -1848,6 +1860,11 @@ qmm_status launch_q8q8_gemv_fused(const DevInfo &dev, int M, int64_t N, int K, c
   st = launch_quantize_act_q8(dev, M, K, X, QX, DX, stream, kLaunchPdl);
   if (st != QMM_OK) return st;
   return launch_stream<kModeQ8>(dev, M, N, K, W, nullptr, QX, DX, Y, nullptr, stream, flags);
+}
+
+qmm_status launch_q8q8_gemv_q8_0(const DevInfo &dev, int M, int64_t N, int K, const void *W, const uint8_t *XB,
+                                 float *Y, cudaStream_t stream, uint32_t flags) {
+  return launch_stream<kModeQ8>(dev, M, N, K, W, nullptr, nullptr, nullptr, Y, nullptr, stream, flags, XB);
 }
 
 qmm_status launch_q8q8_block_dots(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,

@@ -119,6 +119,39 @@ static qmm_status q8_gemv_impl(int64_t M, int64_t N, int64_t K, int block, const
   return launch_q8_gemv(dev, static_cast<int>(M), N, static_cast<int>(K), W, X, Y, s, flags);
 }
 
+static qmm_status quantize_q8_0_impl(int64_t M, int64_t K, int block, const float *X, void *XB, qmm_stream_t stream) {
+  const char *fn = "qmm_quantize_act_q8_0";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, 0, K, block, -1));
+  if (M == 0 || K == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "X", X, true, 16));
+  QMM_TRY(check_ptr(fn, "XB", XB, true, 16));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  return launch_quantize_act_q8_0(dev, M, static_cast<int>(K), X, static_cast<uint8_t *>(XB),
+                                  reinterpret_cast<cudaStream_t>(stream), kLaunchPdl);
+}
+
+static qmm_status q8q8_q8_0_impl(int64_t M, int64_t N, int64_t K, int block, const void *W, const void *XB, float *Y,
+                                 uint32_t user_flags, qmm_stream_t stream) {
+  const char *fn = "qmm_q8q8_gemv_q8_0";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, N, K, block, QMM_MAX_DECODE_M));
+  if (user_flags & ~uint32_t(QMM_FLAG_EARLY_WEIGHTS))
+    return set_error(QMM_ERR_SHAPE, "%s: unknown flags 0x%x", fn, user_flags);
+  if (M == 0 || N == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "W", W, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "XB", XB, K > 0, 16));
+  QMM_TRY(check_ptr(fn, "Y", Y, true, 4));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return zero_fill(Y, M * N, s);
+  uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
+  return launch_q8q8_gemv_q8_0(dev, static_cast<int>(M), N, static_cast<int>(K), W, static_cast<const uint8_t *>(XB),
+                               Y, s, flags);
+}
+
 static qmm_status auto_impl(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X, float *Y,
                             int8_t *QX, float *DX, uint32_t user_flags, qmm_stream_t stream) {
   const char *fn = "qmm_q8_gemv_auto";
@@ -320,6 +353,16 @@ QMM_API qmm_status qmm_q8_gemv(int64_t M, int64_t N, int64_t K, int block, const
 QMM_API qmm_status qmm_q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
                                   float *Y, uint32_t flags, qmm_stream_t stream) {
   return q8_gemv_impl(M, N, K, block, W, X, Y, stream, flags);
+}
+
+QMM_API qmm_status qmm_quantize_act_q8_0(int64_t M, int64_t K, int block, const float *X, void *XB,
+                                         qmm_stream_t stream) {
+  return quantize_q8_0_impl(M, K, block, X, XB, stream);
+}
+
+QMM_API qmm_status qmm_q8q8_gemv_q8_0(int64_t M, int64_t N, int64_t K, int block, const void *W, const void *XB,
+                                      float *Y, uint32_t flags, qmm_stream_t stream) {
+  return q8q8_q8_0_impl(M, N, K, block, W, XB, Y, flags, stream);
 }
 
 QMM_API qmm_status qmm_q8_gemv_auto(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,

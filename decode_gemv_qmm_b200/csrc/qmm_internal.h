@@ -45,6 +45,10 @@ qmm_status launch_q8q8_block_dots(const DevInfo &dev, int M, int64_t N, int K, c
                                   int32_t *isum, cudaStream_t stream);
 qmm_status launch_q8q8_gemv_fused(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
                                   int8_t *QX, float *DX, float *Y, cudaStream_t stream, uint32_t flags);
+qmm_status launch_quantize_act_q8_0(const DevInfo &dev, int64_t M, int K, const float *X, uint8_t *XB,
+                                    cudaStream_t stream, uint32_t flags);
+qmm_status launch_q8q8_gemv_q8_0(const DevInfo &dev, int M, int64_t N, int K, const void *W, const uint8_t *XB,
+                                 float *Y, cudaStream_t stream, uint32_t flags);
 qmm_status launch_quantize_act_q8(const DevInfo &dev, int64_t M, int K, const float *X, int8_t *QX, float *DX,
                                   cudaStream_t stream, uint32_t flags);
 

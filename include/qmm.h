@@ -131,6 +131,42 @@ QMM_API qmm_status qmm_q8_gemv_ex(int64_t M, int64_t N, int64_t K, int block, co
                                   const float *X, float *Y, uint32_t flags, qmm_stream_t stream);
 
 /*
+ * qmm_quantize_act_q8_0 -- quantise fp32 activations into ggml Q8_0 blocks
+ * (34 bytes: fp16 scale d, then 32 int8 codes), the block format of the
+ * weights, so that quantised activations interchange with ggml's.
+ *
+ * The activation-quantisation step of "Lumen v0.4.0", section "Phase 7.M --
+ * Q8xQ8 AVX2 int dot", with the scale kept at fp16 and ggml's reference rule
+ * for the codes: amax = max_j |x_j|; d = amax / 127; id = 1 / d (0 when d ==
+ * 0); q_j = round-half-away-from-zero(x_j * id); each an IEEE binary32
+ * operation; the block stores binary16(d), rounded to nearest even (scales
+ * above 65504 become infinity, as in an fp16 conversion). Codes and scales are
+ * bit-exact functions of X. This differs from qmm_quantize_act_q8, which keeps
+ * d in fp32 and divides x_j / d.
+ *
+ *   M, K   rows and row length (K multiple of 32); M >= 0
+ *   X      M x K fp32 (device, 16-byte aligned)
+ *   XB     M x K/32 Q8_0 blocks, M * (K/32) * 34 bytes (device, 16-byte aligned, written)
+ */
+QMM_API qmm_status qmm_quantize_act_q8_0(int64_t M, int64_t K, int block, const float *X, void *XB,
+                                         qmm_stream_t stream);
+
+/*
+ * qmm_q8q8_gemv_q8_0 -- qmm_q8q8_gemv with the activations as Q8_0 blocks
+ * (fp16 scales), e.g. from qmm_quantize_act_q8_0 or from ggml:
+ *
+ *   Y[m][n] = sum_b (d[n][b] * dx[m][b]) * sum_j qs[n][b][j] * qx[m][b][j]   (exact int32 dots)
+ *
+ *   M      1 .. QMM_MAX_DECODE_M (0 = empty call)
+ *   W      N * K/32 Q8_0 blocks (16-byte aligned)
+ *   XB     M * K/32 Q8_0 blocks (16-byte aligned)
+ *   Y      M x N fp32 (written)
+ *   flags  0 or QMM_FLAG_EARLY_WEIGHTS
+ */
+QMM_API qmm_status qmm_q8q8_gemv_q8_0(int64_t M, int64_t N, int64_t K, int block, const void *W, const void *XB,
+                                      float *Y, uint32_t flags, qmm_stream_t stream);
+
+/*
  * qmm_q8_gemv_auto -- the per-K choice between the fp32-activation GEMV and
  * the Q8xQ8 GEMV ("Lumen v0.4.0", section "Phase 7.P -- per-shape hybrid
  * dispatch": short-K matmuls on the quantised-activation integer path, long-K

@@ -49,6 +49,9 @@ def _bind(lib):
     lib.ora_dequantize.argtypes = [ctypes.c_int, i64, i64, p, p]
     lib.ora_gemv.argtypes = [ctypes.c_int, i64, i64, i64, p, p, i64, i64, i64, i64, p, p]
     lib.ora_quantize_act_q8.argtypes = [i64, i64, p, p, p]
+    lib.ora_quantize_act_q8_0.argtypes = [i64, i64, p, p]
+    lib.ora_float_to_half_rne.argtypes = [ctypes.c_float]
+    lib.ora_float_to_half_rne.restype = ctypes.c_uint16
     lib.ora_q8q8_block_dots.restype = i64
     lib.ora_q8q8_block_dots.argtypes = [i64, i64, i64, p, p, i64, i64, i64, i64, p]
     lib.ora_q8q8_gemv.argtypes = [i64, i64, i64, p, p, p, i64, i64, i64, i64, p, p]
@@ -136,6 +139,32 @@ def quantize_act_q8(X: np.ndarray):
     DX = np.empty((M, K // BLOCK), dtype=np.float32)
     _load().ora_quantize_act_q8(M, K, _ptr(X), _ptr(QX), _ptr(DX))
     return QX, DX
+
+
+def float_to_half_bits(f: float) -> int:
+    """binary32 -> binary16 bits, round to nearest even."""
+    return int(_load().ora_float_to_half_rne(float(np.float32(f))))
+
+
+def quantize_act_q8_0(X: np.ndarray) -> np.ndarray:
+    """Activations as Q8_0 blocks with an fp16 scale (ggml rule); uint8[M, K/32*34]."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    M, K = X.shape
+    XB = np.empty((M, (K // BLOCK) * 34), dtype=np.uint8)
+    _load().ora_quantize_act_q8_0(M, K, _ptr(X), _ptr(XB))
+    return XB
+
+
+def split_q8_0_blocks(XB: np.ndarray, K: int):
+    """Q8_0 activation blocks -> (codes int8[M, K], scales float32[M, K/32] = the fp16 scales)."""
+    XB = np.ascontiguousarray(XB, dtype=np.uint8)
+    M = XB.shape[0]
+    kb = K // BLOCK
+    blk = XB.reshape(M, kb, 34)
+    codes = blk[:, :, 2:].copy().view(np.int8).reshape(M, K)
+    dbits = blk[:, :, 0].astype(np.uint16) | (blk[:, :, 1].astype(np.uint16) << 8)
+    scales = np.array([[half_to_double(int(b)) for b in row] for row in dbits], dtype=np.float32).reshape(M, kb)
+    return codes, scales
 
 
 def q8q8_block_dots(W: np.ndarray, QX: np.ndarray, N: int, window=None) -> np.ndarray:

@@ -18,6 +18,8 @@
  *    "Lumen v0.4.0 -- shape-aware VNNI/fp32 hybrid dispatch", section
  *    "Phase 7.M -- Q8xQ8 AVX2 int dot" (activations quantised to Q8 per
  *    32-block, per-block integer dot, then dequantised and accumulated).
+ *    The Q8_0-block form of the quantised activations (fp16 scale, the
+ *    ggml reference rule) is the ggml-interoperable variant of the same step.
  *  - Fused gate/up SwiGLU out = silu(x.Wg) * (x.Wu):
  *    "LSE v0.4.16", section "Combined M8 Q4 gate/up execution".
  *  - Prefill panels Y = X . W^T with bf16 activations:
@@ -153,6 +155,71 @@ void ora_quantize_act_q8(int64_t M, int64_t K, const float *X, int8_t *QX, float
           q = (int)r;
         }
         QX[m * K + b * ORA_BLOCK + j] = (int8_t)q;
+      }
+    }
+  }
+}
+
+/* ---- Q8_0 activation blocks with an fp16 scale (ggml-compatible form) ---- */
+
+/* binary32 -> IEEE binary16 bits, round to nearest even (subnormals, overflow
+ * to infinity). Written from the format definitions: sign, 5-bit exponent with
+ * bias 15, 10-bit fraction; values below 2^-14 are multiples of 2^-24. */
+uint16_t ora_float_to_half_rne(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  const uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  const uint32_t mag = u & 0x7fffffffu;
+  if (mag >= 0x7f800000u) return (uint16_t)(sign | (mag > 0x7f800000u ? 0x7e00u : 0x7c00u)); /* NaN / Inf */
+  const double a = fabs((double)f); /* exact */
+  if (a >= 65520.0) return (uint16_t)(sign | 0x7c00u); /* rounds to infinity (65504 + half an ulp of 32) */
+  /* the multiple of the binary16 spacing at a's binade, rounded to nearest even */
+  int e;
+  (void)frexp(a, &e);                /* a = m * 2^e, m in [0.5, 1) */
+  int exp16 = e - 1;                  /* a in [2^exp16, 2^(exp16+1)) */
+  if (exp16 < -14) exp16 = -14;       /* subnormal range: spacing 2^-24 */
+  const double ulp = ldexp(1.0, exp16 - 10);
+  double q = a / ulp;                 /* exact: a power-of-two division */
+  double r = floor(q);
+  const double rem = q - r;
+  if (rem > 0.5 || (rem == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+  const double v = r * ulp;           /* the rounded magnitude */
+  if (v == 0.0) return sign;
+  int ev;
+  (void)frexp(v, &ev);
+  const int ex = ev - 1;
+  if (ex < -14) return (uint16_t)(sign | (uint16_t)(v / ldexp(1.0, -24))); /* subnormal */
+  const uint16_t frac = (uint16_t)(v / ldexp(1.0, ex - 10) - 1024.0);
+  return (uint16_t)(sign | (uint16_t)((ex + 15) << 10) | frac);
+}
+
+/* Activations as ggml Q8_0 blocks (34 bytes: fp16 d, then 32 int8 codes),
+ * with ggml's reference rule: amax = max |x_j|; d = amax / 127; id = 1 / d
+ * (0 when d == 0); q_j = round-half-away(x_j * id); the block stores
+ * binary16(d) rounded to nearest even and the codes (|x_j * id| < 127.5, so
+ * the clamp to [-127, 127] never acts). XB: M x (K/32) blocks, row-major. */
+void ora_quantize_act_q8_0(int64_t M, int64_t K, const float *X, uint8_t *XB) {
+  int64_t kb = K / ORA_BLOCK;
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t b = 0; b < kb; ++b) {
+      const float *x = X + m * K + b * ORA_BLOCK;
+      uint8_t *blk = XB + (m * kb + b) * 34;
+      float amax = 0.0f;
+      for (int j = 0; j < ORA_BLOCK; ++j) {
+        float a = fabsf(x[j]);
+        if (a > amax) amax = a;
+      }
+      const float d = amax / 127.0f;
+      const float id = d != 0.0f ? 1.0f / d : 0.0f;
+      const uint16_t h = ora_float_to_half_rne(d);
+      blk[0] = (uint8_t)(h & 0xff);
+      blk[1] = (uint8_t)(h >> 8);
+      for (int j = 0; j < ORA_BLOCK; ++j) {
+        const float v = x[j] * id;
+        float r = roundf(v);
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        blk[2 + j] = (uint8_t)(int8_t)(int)r;
       }
     }
   }

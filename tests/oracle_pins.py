@@ -313,4 +313,54 @@ def pin_prefill_against_numpy():
         assert np.array_equal(y, yg)
 
 
+def pin_half_encoder_against_numpy():
+    """The oracle's binary32 -> binary16 (round to nearest even) against numpy's float16 cast."""
+    g = syn.rng(31)
+    edge = [0.0, -0.0, 1.0, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 2.0 ** -14, 2.0 ** -24, 2.0 ** -25,
+            3 * 2.0 ** -26, 2.0 ** -20, 65504.0, 65519.0, 65519.99, 65520.0, 1e30, -2.5, 0.1, 1 / 3]
+    vals = np.concatenate([np.array(edge, np.float32),
+                           (g.standard_normal(20000) * np.exp2(g.integers(-26, 17, 20000))).astype(np.float32)])
+    with np.errstate(over="ignore"):
+        ref = vals.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.float_to_half_bits(v) for v in vals], np.uint16)
+    assert np.array_equal(got, ref), vals[got != ref][:5]
+
+
+def pin_hand_q8_0_activation_blocks():
+    """Q8_0 activation blocks (ggml rule) worked out by hand."""
+    x = np.zeros((1, 160), np.float32)
+    # block 0: amax 127 -> d = 1 (fp16 0x3C00), id = 1, codes = round half away from zero
+    x[0, :7] = [127.0, -127.0, 2.5, -2.5, 0.5, -0.5, np.float32(1.5) - np.float32(2.0 ** -23)]
+    # block 1: amax = 127 (1 + 2^-11): d = 1 + 2^-11 exactly, halfway between two binary16 values -> even 0x3C00
+    x[0, 32] = 127.0 * (1 + 2.0 ** -11)
+    # block 2: amax = 127 (1 + 3 2^-11): d halfway between 1 + 2^-10 (odd) and 1 + 2^-9 (even) -> 0x3C02
+    x[0, 64] = -127.0 * (1 + 3 * 2.0 ** -11)
+    # block 3: amax = 127 2^-20: d = 2^-20 = 16 2^-24, a binary16 subnormal -> 0x0010
+    x[0, 96] = 127.0 * 2.0 ** -20
+    # block 4: all zero -> d = 0, codes 0
+    xb = oracle.quantize_act_q8_0(x).reshape(5, 34)
+    dbits = [int(b[0]) | int(b[1]) << 8 for b in xb]
+    assert dbits == [0x3C00, 0x3C00, 0x3C02, 0x0010, 0x0000], [hex(v) for v in dbits]
+    codes = xb[:, 2:].view(np.int8)
+    assert codes[0, :8].tolist() == [127, -127, 3, -3, 1, -1, 1, 0]
+    assert codes[1, 0] == 127 and codes[2, 0] == -127 and codes[3, 0] == 127
+    assert not codes[4].any() and not codes[0, 8:].any()
+
+
+def pin_q8_0_activation_properties():
+    """Codes within one of the fp32-scale quantiser's, |x - q d| <= d/2, scale = binary16(d)."""
+    g = syn.rng(32)
+    x = syn.act_f32(g, 3, 1024)
+    xb = oracle.quantize_act_q8_0(x)
+    codes, scales = oracle.split_q8_0_blocks(xb, 1024)
+    q, d = oracle.quantize_act_q8(x)
+    assert np.all(np.abs(codes.astype(np.int32) - q.astype(np.int32)) <= 1)
+    assert np.mean(codes == q) > 0.99
+    d64 = d.astype(np.float64)[..., None]
+    err = np.abs(x.reshape(3, 32, 32).astype(np.float64) - d64 * codes.reshape(3, 32, 32))
+    assert np.all(err <= d64 / 2 * (1 + 2.0 ** -20))
+    assert np.array_equal(scales.astype(np.float16).view(np.uint16),
+                          np.array([[oracle.float_to_half_bits(v) for v in row] for row in d], np.uint16))
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

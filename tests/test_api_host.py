@@ -19,7 +19,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     names = declared_symbols()
-    assert len(names) >= 17
+    assert len(names) >= 19
     for name in names:
         assert hasattr(lib, name), f"{name} declared in include/qmm.h but not exported"
 
@@ -61,6 +61,11 @@ def st_name(st):
     (lambda: lib.qmm_q4_swiglu_gateup(9, 8, 64, 32, P16, P16, P16, P16, 0), "QMM_ERR_SHAPE"),
     (lambda: lib.qmm_q4_swiglu_gateup(8, 8, 64, 32, P16, P_ODD, P16, P16, 0), "QMM_ERR_ALIGN"),
     (lambda: lib.qmm_q4_gateup_unfused(8, 8, 64, 32, P16, P16, P16, 0, P16, P16, 0), "QMM_ERR_NULL"),
+    (lambda: lib.qmm_quantize_act_q8_0(2, 64, 32, P16, P_ODD, 0), "QMM_ERR_ALIGN"),
+    (lambda: lib.qmm_quantize_act_q8_0(2, 48, 32, P16, P16, 0), "QMM_ERR_SHAPE"),
+    (lambda: lib.qmm_q8q8_gemv_q8_0(1, 8, 64, 32, P16, 0, P16, 0, 0), "QMM_ERR_NULL"),
+    (lambda: lib.qmm_q8q8_gemv_q8_0(1, 8, 64, 32, P16, P_ODD, P16, 0, 0), "QMM_ERR_ALIGN"),
+    (lambda: lib.qmm_q8q8_gemv_q8_0(9, 8, 64, 32, P16, P16, P16, 0, 0), "QMM_ERR_SHAPE"),
     (lambda: lib.qmm_q8_gemv_auto(1, 8, 64, 32, P16, P16, P16, 0, P16, 0, 0), "QMM_ERR_NULL"),
     (lambda: lib.qmm_q8_gemv_auto(1, 8, 64, 32, P16, P16, P16, P16, 0, 0, 0), "QMM_ERR_NULL"),
     (lambda: lib.qmm_q8_gemv_auto(1, 8, 64, 32, P16, P16, P16, P16, P16, 2, 0), "QMM_ERR_SHAPE"),

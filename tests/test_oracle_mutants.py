@@ -42,6 +42,11 @@ MUTANTS = [
     ("silu_sign", "g / (1.0 + exp(-g)) * U[i]", "g / (1.0 + exp(g)) * U[i]"),
     ("swiglu_gate_up_swapped", "OUT[i] = g / (1.0 + exp(-g)) * U[i];", "OUT[i] = U[i] / (1.0 + exp(-U[i])) * g;"),
     ("prefill_wrong_decoder", "ora_bf16_to_double(Xbf[", "ora_half_to_double(Xbf["),
+    ("half_round_half_up", "(rem == 0.5 && fmod(r, 2.0) != 0.0)", "(rem == 0.5)"),
+    ("half_subnormal_spacing", "if (exp16 < -14) exp16 = -14;", "if (exp16 < -15) exp16 = -15;"),
+    ("q8_0_codes_scaled_by_d", "const float v = x[j] * id;", "const float v = x[j] * d;"),
+    ("q8_0_scale_byte_order", "blk[0] = (uint8_t)(h & 0xff);\n      blk[1] = (uint8_t)(h >> 8);",
+     "blk[1] = (uint8_t)(h & 0xff);\n      blk[0] = (uint8_t)(h >> 8);"),
 ]
 
 
