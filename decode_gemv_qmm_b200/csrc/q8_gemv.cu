@@ -1167,7 +1167,7 @@ __device__ __forceinline__ float int_exact_f(int v) {  // |v| < 2^22
   return __int_as_float(v + 0x4B400000) - 12582912.0f;
 }
 
-template <int TPS>
+template <int TPS, bool MULTI>
 __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(const __grid_constant__ DParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw;
@@ -1186,7 +1186,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   // whole chunks per CTA: a chunk costs the same however few of its rows are
   // valid, so an even split of rows (every CTA ending in a one-row chunk)
   // costs a chunk per CTA more than an even split of chunks
-  const int64_t tchunks = p.chunk0[p.nproj];
+  const int64_t tchunks = MULTI ? p.chunk0[p.nproj] : (p.Np[0] + kRows - 1) / kRows;
   const int64_t c_begin = static_cast<int64_t>(blockIdx.x) * tchunks / p.grid;
   const int64_t c_end = static_cast<int64_t>(blockIdx.x + 1) * tchunks / p.grid;
   const int nchunks = static_cast<int>(c_end - c_begin);
@@ -1197,12 +1197,18 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     int64_t r0;
     int rows;
   };
+  const int64_t r_begin = c_begin * kRows, r_end = min(p.Np[0], c_end * kRows);  // one matrix
   auto chunk = [&](int c) -> Chunk {
-    const int64_t gc = c_begin + c;
-    int sg = 0;
-    while (sg + 1 < p.nproj && gc >= p.chunk0[sg + 1]) ++sg;
-    const int64_t r0 = (gc - p.chunk0[sg]) * kRows;
-    return {sg, r0, static_cast<int>(min(static_cast<int64_t>(kRows), p.Np[sg] - r0))};
+    if constexpr (MULTI) {
+      const int64_t gc = c_begin + c;
+      int sg = 0;
+      while (sg + 1 < p.nproj && gc >= p.chunk0[sg + 1]) ++sg;
+      const int64_t r0 = (gc - p.chunk0[sg]) * kRows;
+      return {sg, r0, static_cast<int>(min(static_cast<int64_t>(kRows), p.Np[sg] - r0))};
+    } else {
+      const int64_t r0 = r_begin + static_cast<int64_t>(c) * kRows;
+      return {0, r0, static_cast<int>(min(static_cast<int64_t>(kRows), r_end - r0))};
+    }
   };
 
   pdl_launch_dependents();
@@ -1223,11 +1229,11 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     auto issue = [&](int c) {
       const int s = c % S;
       const Chunk ch = chunk(c);
-      const uint8_t *W = p.Wp[ch.proj];
+      const uint8_t *W = MULTI ? p.Wp[ch.proj] : p.Wp[0];
       const int64_t b0 = ch.r0 * p.row_bytes, b1 = (ch.r0 + ch.rows) * p.row_bytes;
       const int64_t a0 = b0 & ~int64_t(15);
       int64_t a1 = (b1 + 15) & ~int64_t(15);
-      const int64_t lim = (p.Np[ch.proj] * p.row_bytes) & ~int64_t(15);
+      const int64_t lim = ((MULTI ? p.Np[ch.proj] : p.Np[0]) * p.row_bytes) & ~int64_t(15);
       uint8_t *dst = stage_mem + static_cast<int64_t>(s) * p.stage_bytes;
       if (a1 > lim) {  // last chunk of a matrix: bytes past its last 16-byte boundary by hand
         for (int64_t t = max(lim, a0); t < b1; ++t) dst[t - a0] = W[t];
@@ -1254,7 +1260,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
       const Chunk ch = chunk(c);
       const int64_t r0 = ch.r0;
       const int rows = ch.rows;
-      float *Y = p.Yp[ch.proj];
+      float *Y = MULTI ? p.Yp[ch.proj] : p.Yp[0];
       const int e = *emax - 188, e1 = max(e, -120);
       const float f1 = __int_as_float((127 + e1) << 23), f2 = __int_as_float((127 + e - e1) << 23);
       const float *rb = red + s * kSlices * kRows;
@@ -1785,17 +1791,20 @@ bool try_launch_digits(const DevInfo &dev, int nproj, const int64_t *N, const vo
   attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  void (*kern)(DParams) = tps == 2 ? q8_gemv_digits_kernel<2> : q8_gemv_digits_kernel<1>;
-  static bool configured[2][64] = {};
+  // the projection table is a compile-time choice: one matrix keeps the plain loop
+  const bool multi = nproj > 1;
+  void (*kern)(DParams) = tps == 2 ? (multi ? q8_gemv_digits_kernel<2, true> : q8_gemv_digits_kernel<2, false>)
+                                   : (multi ? q8_gemv_digits_kernel<1, true> : q8_gemv_digits_kernel<1, false>);
+  static bool configured[2][2][64] = {};
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  if (dev_id >= 0 && dev_id < 64 && !configured[tps - 1][dev_id]) {
+  if (dev_id >= 0 && dev_id < 64 && !configured[tps - 1][multi][dev_id]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBudget);
     if (e != cudaSuccess) {
       *out = cuda_check(e, "q8_gemv attribute");
       return true;
     }
-    configured[tps - 1][dev_id] = true;
+    configured[tps - 1][multi][dev_id] = true;
   }
   *out = cuda_check(cudaLaunchKernelEx(&cfg, kern, p), "q8_gemv launch");
   return true;
