@@ -181,6 +181,11 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
 __device__ __forceinline__ void st_cluster_b32(uint32_t addr, uint32_t a) {
   asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
 }
@@ -469,28 +474,46 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       const int row = 32 * quarter + lane;
       const int dst = (row * split + split - 1) / 128;  // owner rank of this row
       const int lr = row - dst * 128 / split;
-      const uint32_t raddr = map_rank(xbuf + static_cast<uint32_t>((zr * p.MT * p.red_pitch + lr) * 4),
-                                      static_cast<uint32_t>(dst));
+      const uint32_t laddr = xbuf + static_cast<uint32_t>((zr * p.MT * p.red_pitch + lr) * 4);
+      const uint32_t raddr = map_rank(laddr, static_cast<uint32_t>(dst));
+      const bool own = dst == zr;  // this rank's own rows: plain local stores
       const uint32_t cstride = static_cast<uint32_t>(p.red_pitch) * 4u;
       for (int c0 = col0; c0 < p.MT; c0 += 32 * (kDqWarps / 4)) {
         uint32_t v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(c0), v);
+        if (own) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c)  // MT is a multiple of 16: the last load may hold 16 columns
-          if (c0 + c < p.MT) st_cluster_b32(raddr + static_cast<uint32_t>(c0 + c) * cstride, v[c]);
+          for (int c = 0; c < 32; ++c)  // MT is a multiple of 16: the last load may hold 16 columns
+            if (c0 + c < p.MT)
+              asm volatile("st.shared.b32 [%0], %1;" ::"r"(laddr + static_cast<uint32_t>(c0 + c) * cstride), "r"(v[c])
+                           : "memory");
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c0 + c < p.MT) st_cluster_b32(raddr + static_cast<uint32_t>(c0 + c) * cstride, v[c]);
+        }
       }
     }
     cluster_sync_all();  // every partial has landed
+    // sum in rank order: warp w takes token columns w, w + nwarps, ...; its
+    // lanes 32 consecutive rows of the rank's share (contiguous in the buffer
+    // and in Y); no division per element
     const int rbase = zr * 128 / split, rown = (zr + 1) * 128 / split - rbase;
-    const float *buf = reinterpret_cast<const float *>(smem + p.off_x);
     if (!*abort_flag) {
-      for (int e = tid; e < rown * p.MT; e += kThreads) {
-        const int col = e / rown, lr = e - col * rown;
-        const int m = m0 + col;
+      const uint32_t srcstride = static_cast<uint32_t>(p.MT * p.red_pitch) * 4u;
+      for (int lr0 = 0; lr0 < rown; lr0 += 32) {
+        const int lr = lr0 + lane;
         const int64_t row = n0 + rbase + lr;
-        float acc = 0.f;
-        for (int src = 0; src < split; ++src) acc += buf[(src * p.MT + col) * p.red_pitch + lr];
-        if (m < p.M && row < p.N) p.Y[static_cast<int64_t>(m) * p.N + row] = acc;
+        const bool rok = lr < rown && row < p.N;
+        for (int col = warp; col < p.MT; col += kThreads / 32) {
+          const uint32_t a0 = xbuf + static_cast<uint32_t>((col * p.red_pitch + lr) * 4);
+          float acc = 0.f;
+#pragma unroll
+          for (int src = 0; src < kMaxSplit; ++src)
+            if (src < split) acc += lds_f32(a0 + static_cast<uint32_t>(src) * srcstride);
+          const int m = m0 + col;
+          if (rok && m < p.M) p.Y[static_cast<int64_t>(m) * p.N + row] = acc;
+        }
       }
     }
   }
