@@ -1,4 +1,5 @@
-// q4_gateup.cu -- fused gate/up projection with SwiGLU on Q4_0 weights (M <= 8).
+// q4_gateup.cu -- fused gate/up projection with SwiGLU on Q4_0 weights (M <= 8),
+// and with one matrix the Q4_0 GEMV (qmm_q4_gemv).
 //
 // Operation ("LSE v0.4.16", section "Combined M8 Q4 gate/up execution"): one
 // launch reads one shared activation panel X and accumulates the gate and up

@@ -44,6 +44,15 @@
 //    is filled before griddepcontrol.wait (W must not be written by the
 //    preceding kernel); X and Y are touched only after it. The CTA footprint
 //    is small enough for two launches to share an SM.
+//  * In Q8xQ8 mode the activations may also come as ggml Q8_0 blocks (fp16
+//    scale and codes interleaved), read with half-word loads.
+//
+// The file also holds the M = 1 kernels that launch_q8_gemv prefers when the
+// shape suits them (each described where it is defined): the fp32
+// register-resident kernel, the tensor-core resident kernel, the integer
+// tensor-core streaming kernel (which also serves several projections of one
+// activation vector in one launch), and the fused Q8xQ8 resident kernel that
+// quantises the activations itself.
 #include <algorithm>
 
 #include "qmm_common.cuh"

@@ -7,6 +7,8 @@
 //   q_j  = round-half-away-from-zero(x_j / d) (IEEE binary32 division),
 //          clamped to [-127, 127];  d == 0 gives all-zero codes.
 // Codes and scales are bit-exact functions of X (no reciprocal, no fast math).
+// A second kernel writes the ggml-compatible form: Q8_0 blocks (fp16 scale,
+// then the codes) with ggml's rule, codes round(x_j * (1 / d)).
 //
 // One warp per block: lane j owns x_j, the block maximum is one warp-wide
 // integer max over the bit patterns of |x_j| (non-negative floats order like
