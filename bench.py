@@ -650,6 +650,7 @@ def run_case(spec: str, reps: int, seed: int):
     gemv:N:K            qmm_q8_gemv, M=1
     q8q8:N:K            qmm_quantize_act_q8 + qmm_q8q8_gemv, M=1
     q8q8f:N:K           qmm_q8q8_gemv_fused, M=1
+    q4gemv:M:N:K        qmm_q4_gemv
     gateup:M:N:K        qmm_q4_swiglu_gateup
     prefill:q8|q4:M:N:K qmm_quant_matmul_prefill
     decode_step         the 121 GEMVs of one decode step
@@ -684,6 +685,12 @@ def run_case(spec: str, reps: int, seed: int):
         dx = torch.empty(1, k // 32, device="cuda")
         y = torch.empty(1, n, device="cuda")
         launches.append(lambda: qmm.qmm_q8q8_gemv_fused(W, x, n, y, qx, dx))
+    elif parts[0] == "q4gemv":
+        m, n, k = int(parts[1]), int(parts[2]), int(parts[3])
+        W = torch.from_numpy(syn.q4_0_weights(g, n, k)[0]).cuda()
+        x = torch.from_numpy(syn.act_f32(g, m, k)).cuda()
+        y = torch.empty(m, n, device="cuda")
+        launches.append(lambda: qmm.qmm_q4_gemv(W, x, n, y))
     elif parts[0] == "gateup":
         m, n, k = int(parts[1]), int(parts[2]), int(parts[3])
         Wg = torch.from_numpy(syn.q4_0_weights(g, n, k)[0]).cuda()
