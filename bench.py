@@ -510,7 +510,8 @@ def component_q8q8(qmm, dev_peak_gbs, reps_graph=4):
 
 def component_prefill(qmm, pk, reps=10):
     """Prefill panels on the tensor cores: TFLOP/s per shape (rotating weight copies
-    > L2 where the weights are small; activations bf16 N(0,1))."""
+    > L2 where the weights are small; activations bf16 N(0,1)); a chain of calls with
+    early weights (weight blocks streamed while the previous call finishes)."""
     import torch
 
     shapes = [("q8_m32_k896_n4864", syn.Q8_0, 32, 4864, 896), ("q8_m32_k4864_n896", syn.Q8_0, 32, 896, 4864),
@@ -530,7 +531,8 @@ def component_prefill(qmm, pk, reps=10):
 
         def fn(h, Ws=Ws, X=X, Y=Y, wt=wt, m=m, n=n, k=k):
             for w in Ws:
-                assert qmm.lib.qmm_quant_matmul_prefill(wt, m, n, k, 32, w.data_ptr(), X.data_ptr(), Y.data_ptr(), h) == 0
+                assert qmm.lib.qmm_quant_matmul_prefill_ex(wt, m, n, k, 32, w.data_ptr(), X.data_ptr(), Y.data_ptr(),
+                                                           qmm.QMM_FLAG_EARLY_WEIGHTS, h) == 0
         fn(s.cuda_stream)
         torch.cuda.synchronize()
         gr = capture(fn, s)

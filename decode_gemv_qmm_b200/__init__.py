@@ -49,6 +49,7 @@ _SIGS = {
     "qmm_q4_swiglu_gateup": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p],
     "qmm_q4_swiglu_gateup_ex": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _u32, _p],
     "qmm_quant_matmul_prefill": [_int, _i64, _i64, _i64, _int, _p, _p, _p, _p],
+    "qmm_quant_matmul_prefill_ex": [_int, _i64, _i64, _i64, _int, _p, _p, _p, _u32, _p],
     "qmm_q8q8_block_dots": [_i64, _i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q4_gateup_unfused": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p],
 }
@@ -247,10 +248,14 @@ def qmm_q4_gateup_unfused(Wg, Wu, X, N, G=None, U=None, Y=None, *, block: int = 
 
 
 def qmm_quant_matmul_prefill(wtype: int, W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None = None,
-                             *, block: int = BLOCK, stream=None) -> torch.Tensor:
+                             *, block: int = BLOCK, flags: int = 0, stream=None) -> torch.Tensor:
     """Y[M, N] = bf16 X[M, K] . bf16(dequant(W))^T with fp32 accumulation (tensor cores)."""
     M, K = X.shape
     Y = _out(Y, (M, N), X.device)
-    _check(lib.qmm_quant_matmul_prefill(wtype, M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), _stream(stream)),
-           "qmm_quant_matmul_prefill")
+    if flags:
+        st = lib.qmm_quant_matmul_prefill_ex(wtype, M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), flags,
+                                             _stream(stream))
+    else:
+        st = lib.qmm_quant_matmul_prefill(wtype, M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), _stream(stream))
+    _check(st, "qmm_quant_matmul_prefill")
     return Y

@@ -89,6 +89,7 @@ struct alignas(64) Params {
   int x_stage_bytes;
   int off_x, off_raw;  // shared-memory offsets (1024-aligned)
   int split;           // K ranges per output tile (cluster size along z)
+  int prefetch_before_wait;  // weights may be read before the preceding grid completes
   int red_pitch;       // floats per token column of the split-K exchange buffer (rows of one rank)
 };
 
@@ -271,7 +272,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();  // the preceding grid's writes (X, and any reader of Y) are done
+  // The preceding grid's writes (X, and any reader of Y) must be done before
+  // X is loaded and Y written. With early weights only the X producer waits
+  // here; the weight stream, the dequantisation and the MMAs start at once,
+  // and every thread waits again before the epilogue writes Y.
+  if (!p.prefetch_before_wait) pdl_wait();
 
   // Bounded wait shared by all roles: after any timeout every later wait
   // returns at once, so the CTA always reaches the cluster barriers and the
@@ -310,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // Two independent streams, so that neither waits behind the other's ring:
     // lane 0 feeds the X stages, lane 1 the raw chunks.
     if (lane == 0) {
+      if (p.prefetch_before_wait) pdl_wait();
       // stage slot and ring pass kept incrementally: a runtime division per
       // stage costs the serial issuers hundreds of cycles
       for (int i = 0, s = 0, pass = 0; i < nst; ++i) {
@@ -439,6 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   }
 
   // ------------------------------------------------------------ epilogue
+  pdl_wait();  // (already passed without early weights)
   const bool epi = warp >= 2;
   const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 belong to this warp
   const int col0 = warp >= 2 ? 32 * ((warp - 2) >> 2) : 0;  // the warps of a quarter take turns at 32 columns
@@ -539,6 +546,7 @@ int round_up(int v, int a) { return (v + a - 1) / a * a; }
 qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,
                           const uint16_t *X, float *Y, cudaStream_t stream, uint32_t flags) {
   Params p{};
+  p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
   p.W = static_cast<const uint8_t *>(W);
   p.Y = Y;
   p.M = static_cast<int>(M);

@@ -322,12 +322,14 @@ static qmm_status gateup_impl(int64_t M, int64_t N, int64_t K, int block, const 
 }
 
 static qmm_status prefill_impl(int wtype, int64_t M, int64_t N, int64_t K, int block, const void *W,
-                               const uint16_t *X, float *Y, qmm_stream_t stream) {
+                               const uint16_t *X, float *Y, qmm_stream_t stream, uint32_t user_flags) {
   const char *fn = "qmm_quant_matmul_prefill";
   t_last_error.clear();
   if (wtype != QMM_Q8_0 && wtype != QMM_Q4_0) return set_error(QMM_ERR_DTYPE, "%s: unknown weight type %d", fn, wtype);
   QMM_TRY(check_shape(fn, M, N, K, block, -1));
   if (M > (int64_t(1) << 24)) return set_error(QMM_ERR_SHAPE, "%s: M=%lld too large", fn, (long long)M);
+  if (user_flags & ~uint32_t(QMM_FLAG_EARLY_WEIGHTS))
+    return set_error(QMM_ERR_SHAPE, "%s: unknown flags 0x%x", fn, user_flags);
   if (M == 0 || N == 0) return QMM_OK;
   QMM_TRY(check_ptr(fn, "W", W, K > 0, 16));
   QMM_TRY(check_ptr(fn, "X", X, K > 0, 16));
@@ -336,7 +338,8 @@ static qmm_status prefill_impl(int wtype, int64_t M, int64_t N, int64_t K, int b
   QMM_TRY(current_device(&dev));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (K == 0) return zero_fill(Y, M * N, s);
-  return launch_prefill(dev, wtype, M, N, static_cast<int>(K), W, X, Y, s, kLaunchPdl);
+  const uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
+  return launch_prefill(dev, wtype, M, N, static_cast<int>(K), W, X, Y, s, flags);
 }
 
 }  // namespace qmm
@@ -424,7 +427,12 @@ QMM_API qmm_status qmm_q4_gateup_unfused(int64_t M, int64_t N, int64_t K, int bl
 
 QMM_API qmm_status qmm_quant_matmul_prefill(int wtype, int64_t M, int64_t N, int64_t K, int block, const void *W,
                                             const uint16_t *X, float *Y, qmm_stream_t stream) {
-  return prefill_impl(wtype, M, N, K, block, W, X, Y, stream);
+  return prefill_impl(wtype, M, N, K, block, W, X, Y, stream, 0u);
+}
+
+QMM_API qmm_status qmm_quant_matmul_prefill_ex(int wtype, int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                               const uint16_t *X, float *Y, uint32_t flags, qmm_stream_t stream) {
+  return prefill_impl(wtype, M, N, K, block, W, X, Y, stream, flags);
 }
 
 QMM_API const char *qmm_last_error_string(void) { return t_last_error.c_str(); }

@@ -341,6 +341,13 @@ QMM_API qmm_status qmm_quant_matmul_prefill(int wtype, int64_t M, int64_t N, int
                                     const void *W, const uint16_t *X, float *Y,
                                     qmm_stream_t stream);
 
+/* qmm_quant_matmul_prefill with options (0 or QMM_FLAG_EARLY_WEIGHTS: the
+ * weight blocks are streamed and decoded before the preceding kernel in the
+ * stream has finished; X is loaded and Y written only after it). */
+QMM_API qmm_status qmm_quant_matmul_prefill_ex(int wtype, int64_t M, int64_t N, int64_t K, int block,
+                                               const void *W, const uint16_t *X, float *Y, uint32_t flags,
+                                               qmm_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Test and utility exports (not on the hot path).                           */
 

@@ -19,7 +19,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     names = declared_symbols()
-    assert len(names) >= 19
+    assert len(names) >= 20
     for name in names:
         assert hasattr(lib, name), f"{name} declared in include/qmm.h but not exported"
 
@@ -76,6 +76,7 @@ def st_name(st):
     (lambda: lib.qmm_quant_matmul_prefill(2, 8, 8, 64, 32, P16, P16, P16, 0), "QMM_ERR_DTYPE"),
     (lambda: lib.qmm_quant_matmul_prefill(0, 8, 8, 64, 32, P16, P_ODD, P16, 0), "QMM_ERR_ALIGN"),
     (lambda: lib.qmm_quant_matmul_prefill(1, 8, -8, 64, 32, P16, P16, P16, 0), "QMM_ERR_SHAPE"),
+    (lambda: lib.qmm_quant_matmul_prefill_ex(0, 8, 8, 64, 32, P16, P16, P16, 2, 0), "QMM_ERR_SHAPE"),
 ])
 def test_argument_errors_before_any_cuda_call(call, expect):
     st = call()

@@ -96,3 +96,17 @@ def test_prefill_split_k_deterministic():
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert qmm.device_status() == 0
+
+
+@pytest.mark.parametrize("wtype,m,n,k", [(syn.Q8_0, 1024, 4864, 896), (syn.Q8_0, 32, 896, 4864),
+                                         (syn.Q4_0, 300, 129, 768), (syn.Q8_0, 64, 257, 160)])
+def test_prefill_early_weights_same_bits(wtype, m, n, k):
+    """With early weights the result is bit-identical (only the start of the weight stream moves)."""
+    g = syn.rng(m + n + k + 5)
+    W = dev(syn.weights(g, wtype, n, k))
+    X = dev(syn.act_bf16_bits(g, m, k))
+    Y0 = qmm.qmm_quant_matmul_prefill(wtype, W, X, n)
+    Y1 = qmm.qmm_quant_matmul_prefill(wtype, W, X, n, flags=qmm.QMM_FLAG_EARLY_WEIGHTS)
+    torch.cuda.synchronize()
+    assert torch.equal(Y0.view(torch.int32), Y1.view(torch.int32))
+    assert qmm.device_status() == 0
