@@ -52,6 +52,7 @@ _SIGS = {
     "qmm_quant_matmul_prefill_ex": [_int, _i64, _i64, _i64, _int, _p, _p, _p, _u32, _p],
     "qmm_q8q8_block_dots": [_i64, _i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q4_gateup_unfused": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p],
+    "qmm_prefill_plan": [_int, _i64, _i64, _i64, _int, _p],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(lib, _name, None)
@@ -259,3 +260,10 @@ def qmm_quant_matmul_prefill(wtype: int, W: torch.Tensor, X: torch.Tensor, N: in
         st = lib.qmm_quant_matmul_prefill(wtype, M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), _stream(stream))
     _check(st, "qmm_quant_matmul_prefill")
     return Y
+
+
+def qmm_prefill_plan(wtype: int, M: int, N: int, K: int, *, block: int = BLOCK) -> dict:
+    """The tiling qmm_quant_matmul_prefill launches for this problem on the current device."""
+    out = (ctypes.c_int32 * 4)()
+    _check(lib.qmm_prefill_plan(wtype, M, N, K, block, ctypes.addressof(out)), "qmm_prefill_plan")
+    return {"mt": out[0], "split": out[1], "stages": out[2], "ctas": out[3]}

@@ -8,10 +8,14 @@
 // round-to-nearest-even to bf16) and the products accumulate in fp32 in
 // tensor memory.
 //
-// B200 design (one CTA per 128 x MT output tile and K range, MT <= 256 tokens):
+// B200 design (one CTA per 128 x MT output tile and K range, MT <= 384 tokens):
 //  * MMA shape M = 128 weight rows, N = MT tokens, K = 16 (kind::f16, bf16
 //    inputs, fp32 accumulator in TMEM, one thread issues, cta_group::1). The
-//    accumulator D[n][m] lives in MT TMEM columns x 128 lanes.
+//    accumulator D[n][m] lives in MT TMEM columns x 128 lanes. A tile wider
+//    than 256 tokens (one MMA's limit) takes two MMAs per k step, tokens
+//    0..255 and 256..MT-1 of the same A; the launcher picks such tiles when
+//    they cut the number of waves (1024 tokens x 4864 rows: 114 tiles of 352
+//    tokens in one wave instead of 152 of 256 in two).
 //  * A (weights, 128 x 64 per stage) never touches shared memory: sixteen
 //    "dequant" warps in two groups that take alternate stages (each warp has
 //    two stages of MMA time per stage it converts) write each decoded row
@@ -63,7 +67,7 @@ constexpr int kDqWarps = 8 * kDqGroups; // dequant (then epilogue) warps: thread
 constexpr int kThreads = 64 + 32 * kDqWarps;  // warp 0 producer, warp 1 MMA, warps 2.. dequant + epilogue
 constexpr int kRawBlocks = 8;          // blocks per raw weight chunk
 constexpr int kStageK = 64;            // k per MMA stage (one 128-byte swizzle row of bf16)
-constexpr int kAccCols = 256;          // TMEM columns 0..255: the fp32 accumulator (MT <= 256)
+constexpr int kMaxMT = 384;            // widest token tile (two MMAs per k step above 256)
 constexpr int kACols = 32;             // TMEM columns per A stage: 128 rows x 64 bf16 (two per 32-bit cell)
 // Raw chunks in flight. Q8 chunks are twice the size of Q4 ones; two in flight
 // (eight stages of lead) leave room for four X stages instead of two, which
@@ -73,7 +77,8 @@ constexpr int raw_stages() { return WT == QMM_Q8_0 ? 2 : 4; }
 constexpr int kMaxSplit = 8;           // portable cluster size
 
 struct alignas(64) Params {
-  CUtensorMap tm_x;    // X: dims {K, M} bf16, box {64, MT}, 128-byte swizzle
+  CUtensorMap tm_x;    // X: dims {K, M} bf16, box {64, min(MT, 256)}, 128-byte swizzle
+  CUtensorMap tm_x2;   // MT > 256: the same X, box {64, MT - 256} (tokens 256.. of a tile)
   CUtensorMap tm_w;    // W as super-rows of rs rows: dims {rs * row_bytes / 2, N / rs} uint16, box {raw_pitch / 2, 128 / rs}
   const uint8_t *W;
   float *Y;
@@ -82,7 +87,8 @@ struct alignas(64) Params {
   int64_t row_bytes;
   int64_t tma_rows;    // rows loaded by TMA (whole super-rows); the rest by the dequant warps
   int rs;              // rows per super-row: the smallest of 1, 2, 4, 8 whose pitch is a multiple of 16
-  int MT;              // tokens per tile (multiple of 16, <= 256)
+  int MT;              // tokens per tile (multiple of 16; above 256 a multiple of 32, <= kMaxMT)
+  int acc_cols;        // TMEM columns of the accumulator (max(256, MT)); the A stages follow
   int tmem_cols;
   int stages;          // MMA stages in flight
   int raw_pitch;       // bytes per row of a raw chunk in shared memory (a chunk + up to 15 bytes in front)
@@ -223,7 +229,10 @@ __device__ __forceinline__ void q4_nib_bf16(uint32_t v, float d, uint32_t &o01, 
   o23 = bf16x2(f23.x, f23.y);
 }
 
-template <int WT>
+// WIDE: tiles of more than 256 tokens (two MMAs per k step); a template
+// parameter so that the narrow form's single-thread issue loop carries no
+// extra test.
+template <int WT, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -323,6 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         if (!*abort_flag) {
           mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.x_stage_bytes));
           tma_load_2d(smem + p.off_x + s * p.x_stage_bytes, &p.tm_x, (j_lo + i) * kStageK, m0, &full[s]);
+          if (WIDE)  // tokens 256.. of the tile: 8-row atoms continue 32 KB further on
+            tma_load_2d(smem + p.off_x + s * p.x_stage_bytes + 256 * 128, &p.tm_x2, (j_lo + i) * kStageK, m0 + 256,
+                        &full[s]);
         }
         if (++s == S) {
           s = 0;
@@ -336,7 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(p.MT);
+      const uint32_t idesc = idesc_bf16_f32(WIDE ? 256 : p.MT);
+      const uint32_t idesc2 = idesc_bf16_f32(WIDE ? p.MT - 256 : 16);  // tokens 256..MT-1
+      const uint32_t acc_cols = WIDE ? static_cast<uint32_t>(p.acc_cols) : 256u;
       // descriptors of stage 0; a stage / k step is an offset in 16-byte units
       // of the descriptor's address field (shared-memory addresses < 256 KB)
       const uint64_t bdesc0 = sw128_kmajor_desc(sbase + p.off_x);
@@ -345,11 +359,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         wait(&full[s], static_cast<uint32_t>(pass) & 1u);  // after a timeout: garbage in, discarded
         tc_fence_after();
         const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * xs16);
-        const uint32_t at = tmem + static_cast<uint32_t>(kAccCols + s * kACols);
-        umma_f16_ts(tmem, at, bd, idesc, i > 0);
-        umma_f16_ts(tmem, at + 8, bd + 2, idesc, true);
-        umma_f16_ts(tmem, at + 16, bd + 4, idesc, true);
-        umma_f16_ts(tmem, at + 24, bd + 6, idesc, true);
+        const uint32_t at = tmem + acc_cols + static_cast<uint32_t>(s * kACols);
+        if (!WIDE) {
+          umma_f16_ts(tmem, at, bd, idesc, i > 0);
+          umma_f16_ts(tmem, at + 8, bd + 2, idesc, true);
+          umma_f16_ts(tmem, at + 16, bd + 4, idesc, true);
+          umma_f16_ts(tmem, at + 24, bd + 6, idesc, true);
+        } else {
+          // tokens 256.. start 256 rows (32 KB = 2048 descriptor units) into the stage
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            umma_f16_ts(tmem, at + 8 * kk, bd + 2 * kk, idesc, i > 0 || kk > 0);
+            umma_f16_ts(tmem + 256, at + 8 * kk, bd + 2048 + 2 * kk, idesc2, i > 0 || kk > 0);
+          }
+        }
         umma_commit(&st_empty[s]);  // frees this stage's A and X buffers when the MMAs finish
         if (++s == S) {
           s = 0;
@@ -370,7 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const int r = 32 * quarter + lane, h = (dw >> 2) & 1;
     const int64_t n = n0 + r;
     const bool row_ok = n < p.N;
-    const uint32_t a_lane = tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(kAccCols + 16 * h);
+    const uint32_t a_lane = tmem + (static_cast<uint32_t>(32 * quarter) << 16) +
+                            static_cast<uint32_t>((WIDE ? p.acc_cols : 256) + 16 * h);
     constexpr int kWords = (kBlockBytes + 2 + 3) / 4;  // the block as words, plus the 16-bit shift (Q8: 9, Q4: 5)
     int s0 = dg, pass0 = 0;  // the slot and ring pass of stage dg (S >= kDqGroups)
     for (int i = dg, s = s0, pass = pass0; i < nst;
@@ -453,6 +477,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     if (epi) {
       tc_fence_after();
       const int64_t row = n0 + 32 * quarter + lane;
+      // a 32-column load past MT happens only for a single tile (MT = M
+      // rounded up to 16, M <= 256); tiles above 256 tokens are multiples of 32
       for (int c0 = col0; c0 < p.MT; c0 += 32 * (kDqWarps / 4)) {
         uint32_t v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(c0), v);
@@ -534,9 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   }
 }
 
-template <int WT>
+template <int WT, bool WIDE>
 void *kernel_ptr() {
-  return reinterpret_cast<void *>(prefill_kernel<WT>);
+  return reinterpret_cast<void *>(prefill_kernel<WT, WIDE>);
 }
 
 int round_up(int v, int a) { return (v + a - 1) / a * a; }
@@ -544,7 +570,7 @@ int round_up(int v, int a) { return (v + a - 1) / a * a; }
 }  // namespace
 
 qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,
-                          const uint16_t *X, float *Y, cudaStream_t stream, uint32_t flags) {
+                          const uint16_t *X, float *Y, cudaStream_t stream, uint32_t flags, PrefillPlan *plan) {
   Params p{};
   p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
   p.W = static_cast<const uint8_t *>(W);
@@ -558,45 +584,38 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
   p.rs = 1;
   while ((p.rs * p.row_bytes) % 16 != 0) p.rs *= 2;  // at most 8: 8 * 34 = 16 * 17, 8 * 18 = 16 * 9
   p.tma_rows = N / p.rs * p.rs;
-  p.MT = static_cast<int>(std::min<int64_t>(256, round_up(static_cast<int>(std::min<int64_t>(M, 256)), 16)));
-  p.tmem_cols = 512;  // accumulator in columns 0..MT-1, A stage s at 256 + 32 s
-  p.x_stage_bytes = p.MT * 128;
   // a row's chunk plus up to 15 bytes of alignment in front, rounded to 16
   // and then to 16 mod 32 (rows spread over eight 4-byte bank groups)
   p.raw_pitch = wtype == QMM_Q8_0 ? 304 : 176;
   const int raw_bytes = (wtype == QMM_Q8_0 ? raw_stages<QMM_Q8_0>() : raw_stages<QMM_Q4_0>()) * 128 * p.raw_pitch;
-  const int per_stage = p.x_stage_bytes;  // A lives in tensor memory
   const int budget = dev.smem_optin - 1024 /*align*/ - 1024 /*barriers*/ - round_up(raw_bytes, 1024);
-  p.stages = std::max(2, std::min(8, budget / per_stage));
-  p.off_x = 1024;
-  p.off_raw = p.off_x + p.stages * p.x_stage_bytes;
-  // Every CTA allocates all 512 TMEM columns, so never two CTAs on one SM (a
-  // second one would wait in tcgen05.alloc, and across clusters that wait
-  // could close a cycle): ask for more than half of the shared memory.
-  const size_t smem = std::max<size_t>(static_cast<size_t>(p.off_raw) + raw_bytes + 1024,
-                                       static_cast<size_t>(dev.smem_optin / 2 + 1024));
-  if (smem > static_cast<size_t>(dev.smem_optin))
-    return set_error(QMM_ERR_SHAPE, "prefill: tile needs %zu bytes of shared memory", smem);
+  // MMA stages of a tile MT tokens wide: X stages in shared memory (A lives in
+  // tensor memory), A stages in the TMEM columns past the accumulator
+  auto stages_for = [&](int mt) {
+    return std::min({8, budget / (mt * 128), (512 - std::max(256, mt)) / kACols});
+  };
+  auto smem_for = [&](int mt) {
+    // Every CTA allocates all 512 TMEM columns, so never two CTAs on one SM (a
+    // second one would wait in tcgen05.alloc, and across clusters that wait
+    // could close a cycle): ask for more than half of the shared memory.
+    return std::max<size_t>(static_cast<size_t>(1024 + stages_for(mt) * mt * 128) + raw_bytes + 1024,
+                            static_cast<size_t>(dev.smem_optin / 2 + 1024));
+  };
 
-  const uint64_t xd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-  const uint64_t xs[1] = {static_cast<uint64_t>(K) * 2};
-  const uint32_t xb[2] = {64, static_cast<uint32_t>(p.MT)};
-  qmm_status st = encode_tiled(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, xd, xs, xb, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != QMM_OK) return st;
-
-  const int64_t ntiles = (N + 127) / 128, mtiles = (M + p.MT - 1) / p.MT;
-  if (ntiles > 65535 || mtiles > 0x7fffffff) return set_error(QMM_ERR_SHAPE, "prefill: grid too large");
-  void *kern = wtype == QMM_Q8_0 ? kernel_ptr<QMM_Q8_0>() : kernel_ptr<QMM_Q4_0>();
+  void *kerns[2][2] = {{kernel_ptr<QMM_Q8_0, false>(), kernel_ptr<QMM_Q8_0, true>()},
+                       {kernel_ptr<QMM_Q4_0, false>(), kernel_ptr<QMM_Q4_0, true>()}};
   static bool configured[2][64] = {};
   if (dev.device >= 0 && dev.device < 64 && !configured[wtype][dev.device]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
-    if (e != cudaSuccess) return cuda_check(e, "prefill attribute");
+    for (int w = 0; w < 2; ++w) {
+      cudaError_t e = cudaFuncSetAttribute(kerns[wtype][w], cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
+      if (e != cudaSuccess) return cuda_check(e, "prefill attribute");
+    }
     configured[wtype][dev.device] = true;
   }
+  void *kern = kerns[wtype][0];  // split-K occupancy queries: narrow tiles
 
   cudaLaunchConfig_t cfg{};
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -604,19 +623,23 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
   attr[1].id = cudaLaunchAttributeClusterDimension;
   cfg.attrs = attr;
 
+  const int64_t ntiles = (N + 127) / 128;
+  const int nst_all = (p.KB + 1) / 2;
   // Split K over a cluster when the output tiles leave SMs idle: as many
   // ranks as fit one wave, each with at least one stage, the exchange buffer
   // inside the stage buffers, and every cluster resident at once.
-  const int64_t base = ntiles * mtiles;
-  const int nst_all = (p.KB + 1) / 2;
-  int split = 1;
-  if (base < dev.sms) {
-    split = static_cast<int>(std::min<int64_t>({kMaxSplit, nst_all, dev.sms / base}));
+  auto choose_split = [&](int mt) -> int {
+    const int64_t base = ntiles * ((M + mt - 1) / mt);
+    if (base >= dev.sms) return 1;
+    const int xbytes = stages_for(mt) * mt * 128;
+    int split = static_cast<int>(std::min<int64_t>({kMaxSplit, nst_all, dev.sms / base}));
     for (; split > 1; --split) {
       const int rmax = (128 + split - 1) / split;
       // the exchange buffer reuses the X stages and the raw chunks (all consumed by then)
-      if (static_cast<int64_t>(split) * p.MT * rmax * 4 > p.off_raw + raw_bytes - p.off_x) continue;
-      cfg.gridDim = dim3(static_cast<unsigned>(mtiles), static_cast<unsigned>(ntiles), static_cast<unsigned>(split));
+      if (static_cast<int64_t>(split) * mt * rmax * 4 > xbytes + raw_bytes) continue;
+      cfg.gridDim = dim3(static_cast<unsigned>((M + mt - 1) / mt), static_cast<unsigned>(ntiles),
+                         static_cast<unsigned>(split));
+      cfg.dynamicSmemBytes = smem_for(mt);
       attr[1].val.clusterDim.x = 1;
       attr[1].val.clusterDim.y = 1;
       attr[1].val.clusterDim.z = static_cast<unsigned>(split);
@@ -625,7 +648,62 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
       if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active >= base) break;
       cudaGetLastError();  // a refused query is not an error of this call
     }
+    return split;
+  };
+  // Makespan in units of one 64-k stage of one token: waves x stages per CTA x MT.
+  auto cost_of = [&](int mt, int split) -> int64_t {
+    const int64_t ctas = ntiles * ((M + mt - 1) / mt) * split;
+    return (ctas + dev.sms - 1) / dev.sms * ((nst_all + split - 1) / split) * mt;
+  };
+
+  // Token tile: up to 256 tokens (one MMA). When the tiles fill at least one
+  // wave (no split K), wider tiles (two MMAs per k step, at least three
+  // stages) are taken if they cut the makespan by 15% or more, i.e. when
+  // 256-token tiles leave a nearly empty last wave.
+  int mt = static_cast<int>(std::min<int64_t>(256, round_up(static_cast<int>(std::min<int64_t>(M, 256)), 16)));
+  int split = choose_split(mt);
+  if (M > 256 && split == 1) {
+    int64_t cost = cost_of(mt, 1);
+    for (int64_t c = (M + kMaxMT - 1) / kMaxMT; c < (M + 255) / 256; ++c) {
+      const int w = round_up(static_cast<int>((M + c - 1) / c), 32);
+      if (w <= 256 || w > kMaxMT || stages_for(w) < 3) continue;
+      const int64_t wc = cost_of(w, 1);
+      if (wc * 100 <= cost * 85) {
+        mt = w;
+        cost = wc;
+      }
+    }
   }
+  p.MT = mt;
+  p.acc_cols = std::max(256, mt);
+  p.tmem_cols = 512;  // accumulator in columns 0..acc_cols-1, A stage s at acc_cols + 32 s
+  p.x_stage_bytes = p.MT * 128;
+  p.stages = stages_for(mt);
+  if (p.stages < 2) return set_error(QMM_ERR_SHAPE, "prefill: no room for two stages of %d tokens", mt);
+  p.off_x = 1024;
+  p.off_raw = p.off_x + p.stages * p.x_stage_bytes;
+  const size_t smem = smem_for(mt);
+  if (smem > static_cast<size_t>(dev.smem_optin))
+    return set_error(QMM_ERR_SHAPE, "prefill: tile needs %zu bytes of shared memory", smem);
+  cfg.dynamicSmemBytes = smem;
+  const int64_t mtiles = (M + p.MT - 1) / p.MT;
+  if (ntiles > 65535 || mtiles > 0x7fffffff) return set_error(QMM_ERR_SHAPE, "prefill: grid too large");
+  if (plan) {
+    *plan = PrefillPlan{p.MT, split, p.stages, static_cast<int>(ntiles * mtiles * split)};
+    return QMM_OK;
+  }
+
+  const uint64_t xd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  const uint64_t xs[1] = {static_cast<uint64_t>(K) * 2};
+  const uint32_t xb[2] = {64, static_cast<uint32_t>(std::min(p.MT, 256))};
+  qmm_status st = encode_tiled(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, xd, xs, xb, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QMM_OK) return st;
+  if (p.MT > 256) {
+    const uint32_t xb2[2] = {64, static_cast<uint32_t>(p.MT - 256)};
+    st = encode_tiled(&p.tm_x2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, xd, xs, xb2, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != QMM_OK) return st;
+  }
+
   p.split = split;
   p.red_pitch = (128 + split - 1) / split;  // rows of the largest rank share
   if (p.rs == 1 && split == 1) p.raw_pitch = kRawBlocks * bb;  // chunks start on 16-byte boundaries: 272 / 144
@@ -642,7 +720,7 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
   attr[1].val.clusterDim.z = static_cast<unsigned>(split);
   cfg.numAttrs = split > 1 ? 2 : 1;
   void *args[] = {&p};
-  return cuda_check(cudaLaunchKernelExC(&cfg, kern, args), "prefill launch");
+  return cuda_check(cudaLaunchKernelExC(&cfg, kerns[wtype][p.MT > 256 ? 1 : 0], args), "prefill launch");
 }
 
 cudaError_t prefill_status(uint32_t *bits) {

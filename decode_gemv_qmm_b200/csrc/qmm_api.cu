@@ -435,6 +435,25 @@ QMM_API qmm_status qmm_quant_matmul_prefill_ex(int wtype, int64_t M, int64_t N, 
   return prefill_impl(wtype, M, N, K, block, W, X, Y, stream, flags);
 }
 
+QMM_API qmm_status qmm_prefill_plan(int wtype, int64_t M, int64_t N, int64_t K, int block, int32_t *plan) {
+  const char *fn = "qmm_prefill_plan";
+  t_last_error.clear();
+  if (plan == nullptr) return set_error(QMM_ERR_NULL, "%s: plan is NULL", fn);
+  if (wtype != QMM_Q8_0 && wtype != QMM_Q4_0) return set_error(QMM_ERR_DTYPE, "%s: unknown weight type %d", fn, wtype);
+  QMM_TRY(check_shape(fn, M, N, K, block, -1));
+  if (M < 1 || N < 1 || K < 32) return set_error(QMM_ERR_SHAPE, "%s: M, N must be >= 1 and K >= 32", fn);
+  if (M > (int64_t(1) << 24)) return set_error(QMM_ERR_SHAPE, "%s: M=%lld too large", fn, (long long)M);
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  PrefillPlan pl{};
+  QMM_TRY(launch_prefill(dev, wtype, M, N, static_cast<int>(K), nullptr, nullptr, nullptr, nullptr, 0u, &pl));
+  plan[0] = pl.mt;
+  plan[1] = pl.split;
+  plan[2] = pl.stages;
+  plan[3] = pl.ctas;
+  return QMM_OK;
+}
+
 QMM_API const char *qmm_last_error_string(void) { return t_last_error.c_str(); }
 
 QMM_API const char *qmm_version(void) { return "qmm 0.1.0 sm_100a"; }

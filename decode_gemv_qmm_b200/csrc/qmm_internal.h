@@ -60,8 +60,15 @@ qmm_status launch_q4_gemv(const DevInfo &dev, int M, int64_t N, int K, const voi
 qmm_status launch_q4_gateup_unfused(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
                                     const float *X, float *G, float *U, float *Y, cudaStream_t stream);
 
+// The tiling launch_prefill picks: tokens per tile, K ranges per tile
+// (cluster size), MMA stages in flight and CTAs of the launch.
+struct PrefillPlan {
+  int mt, split, stages, ctas;
+};
+// With `plan` set, only the tiling is computed (nothing is launched).
 qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,
-                          const uint16_t *X, float *Y, cudaStream_t stream, uint32_t flags);
+                          const uint16_t *X, float *Y, cudaStream_t stream, uint32_t flags,
+                          PrefillPlan *plan = nullptr);
 
 // Device status word of each kernel file: read and clear (synchronous).
 cudaError_t q8_gemv_status(uint32_t *bits);

@@ -372,6 +372,17 @@ QMM_API qmm_status qmm_q4_gateup_unfused(int64_t M, int64_t N, int64_t K, int bl
                                  const void *Wu, const float *X, float *G, float *U, float *Y,
                                  qmm_stream_t stream);
 
+/*
+ * qmm_prefill_plan -- the tiling qmm_quant_matmul_prefill would launch on the
+ * current device for this problem, without launching anything:
+ * plan[0] = tokens per output tile (MT; above 256 each k step takes two
+ * MMAs), plan[1] = K ranges per tile (thread-block cluster size, 1 = no
+ * split), plan[2] = MMA stages in flight, plan[3] = CTAs of the launch.
+ * Host memory `plan` (4 int32, written). Needs an sm_100 device
+ * (QMM_ERR_DEVICE otherwise); M, N >= 1, K >= 32 (QMM_ERR_SHAPE).
+ */
+QMM_API qmm_status qmm_prefill_plan(int wtype, int64_t M, int64_t N, int64_t K, int block, int32_t *plan);
+
 /* Text of the last error raised on the calling host thread ("" if none). */
 QMM_API const char *qmm_last_error_string(void);
 

@@ -77,6 +77,12 @@ def st_name(st):
     (lambda: lib.qmm_quant_matmul_prefill(0, 8, 8, 64, 32, P16, P_ODD, P16, 0), "QMM_ERR_ALIGN"),
     (lambda: lib.qmm_quant_matmul_prefill(1, 8, -8, 64, 32, P16, P16, P16, 0), "QMM_ERR_SHAPE"),
     (lambda: lib.qmm_quant_matmul_prefill_ex(0, 8, 8, 64, 32, P16, P16, P16, 2, 0), "QMM_ERR_SHAPE"),
+    (lambda: lib.qmm_prefill_plan(0, 1024, 4864, 896, 32, 0), "QMM_ERR_NULL"),
+    (lambda: lib.qmm_prefill_plan(2, 1024, 4864, 896, 32, P16), "QMM_ERR_DTYPE"),
+    (lambda: lib.qmm_prefill_plan(0, 1024, 4864, 896, 16, P16), "QMM_ERR_BLOCK"),
+    (lambda: lib.qmm_prefill_plan(0, 1024, 4864, 900, 32, P16), "QMM_ERR_SHAPE"),
+    (lambda: lib.qmm_prefill_plan(0, 0, 4864, 896, 32, P16), "QMM_ERR_SHAPE"),
+    (lambda: lib.qmm_prefill_plan(1, 8, 8, 0, 32, P16), "QMM_ERR_SHAPE"),
 ])
 def test_argument_errors_before_any_cuda_call(call, expect):
     st = call()

@@ -110,3 +110,30 @@ def test_prefill_early_weights_same_bits(wtype, m, n, k):
     torch.cuda.synchronize()
     assert torch.equal(Y0.view(torch.int32), Y1.view(torch.int32))
     assert qmm.device_status() == 0
+
+
+def test_prefill_plan_wide_tiles_for_a_nearly_empty_last_wave():
+    """1024 tokens x 4864 rows: 152 tiles of 256 tokens are two waves on 148 SMs, the second
+    nearly empty; 114 tiles of 352 tokens (two MMAs per k step) are one."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    p = qmm.qmm_prefill_plan(syn.Q8_0, 1024, 4864, 896)
+    if 114 <= sms < 152:
+        assert (p["mt"], p["split"], p["ctas"]) == (352, 1, 114), p
+        assert p["stages"] >= 3, p
+    # 544 tiles of 256 tokens against 408 of 352: four waves against three, no gain
+    assert qmm.qmm_prefill_plan(syn.Q4_0, 1024, 17408, 5120)["mt"] == 256
+    # few tiles: narrow tiles and split K
+    p = qmm.qmm_prefill_plan(syn.Q8_0, 32, 4864, 896)
+    assert p["mt"] == 32 and p["split"] > 1, p
+
+
+@pytest.mark.parametrize("wtype", [syn.Q8_0, syn.Q4_0])
+@pytest.mark.parametrize("m,n,k", [(520, 6390, 128),    # tiles of 288 tokens, the second one ragged
+                                   (600, 6400, 96),     # odd block count, super-row TMA of the weights
+                                   (1000, 4864, 256)])  # tiles of 352 tokens: 352 + 352 + 296
+def test_prefill_wide_token_tiles(wtype, m, n, k):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plan = qmm.qmm_prefill_plan(wtype, m, n, k)
+    if sms == 148:
+        assert plan["mt"] > 256 and plan["split"] == 1, plan
+    check_full(wtype, m, n, k, seed=7 * m + n + k)
