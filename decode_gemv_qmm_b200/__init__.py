@@ -264,6 +264,7 @@ def qmm_quant_matmul_prefill(wtype: int, W: torch.Tensor, X: torch.Tensor, N: in
 
 def qmm_prefill_plan(wtype: int, M: int, N: int, K: int, *, block: int = BLOCK) -> dict:
     """The tiling qmm_quant_matmul_prefill launches for this problem on the current device."""
-    out = (ctypes.c_int32 * 4)()
+    out = (ctypes.c_int32 * 5)()
     _check(lib.qmm_prefill_plan(wtype, M, N, K, block, ctypes.addressof(out)), "qmm_prefill_plan")
-    return {"mt": out[0], "split": out[1], "stages": out[2], "ctas": out[3]}
+    return {"mt": out[0], "split": out[1], "stages": out[2], "ctas": out[3],
+            "kernel": "small_m" if out[4] == 1 else "tcgen05"}

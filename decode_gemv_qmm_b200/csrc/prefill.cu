@@ -51,6 +51,11 @@
 //  * Every mbarrier wait is bounded; on a timeout the kernel records a status
 //    bit, finishes without waiting further (still meeting both cluster
 //    barriers) and frees its TMEM.
+//
+// Panels of at most 32 tokens run a second kernel in this file, the small-M
+// kernel (mma.sync on whole shares of W and X held in shared memory; see its
+// description below): at that size the work is bound by streaming the weights
+// and by latency, not by the tensor cores.
 #include <algorithm>
 
 #include "qmm_common.cuh"
@@ -191,6 +196,11 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
 }
 __device__ __forceinline__ void st_cluster_b32(uint32_t addr, uint32_t a) {
@@ -567,10 +577,581 @@ void *kernel_ptr() {
 
 int round_up(int v, int a) { return (v + a - 1) / a * a; }
 
+// ---------------------------------------------------------------------------
+// Small-M panels (M <= 32 tokens). Two to four MFLOP per weight row are no
+// work for the tensor cores; such a panel is bound by streaming its weights
+// from HBM once, plus launch and dependency latency. So no tensor-memory
+// pipeline: every CTA copies its whole share of W (rows [r0, r0 + R), K blocks
+// [kb0, kb1)) and the matching X slice into shared memory and multiplies with
+// mma.sync.m16n8k16 (bf16, fp32 accumulation), one block at a time:
+//  * Few, large copies (many small ones made the launch latency-bound: 65 bulk
+//    copies of 1-2 KB per CTA took 11.3 us where two take 6.9). Without split
+//    K the CTA's rows are one contiguous byte range of W and X is one
+//    contiguous range too: one bulk copy each. With split K the rows' segments
+//    come as one 2-D TMA box (W viewed as rows of 4-byte words; rows a
+//    multiple of 16 bytes long) and X as boxes of 256 k x 8 QM tokens (token
+//    rows past M read as zero); other row lengths fall back to a bulk copy
+//    per row segment.
+//  * The compute loop reads shared memory with plain loads (after the
+//    mbarrier waits, which order them) so that a warp's loads, conversions and
+//    mma instructions of several tiles and blocks overlap.
+//  * A = 16 weight rows x 16 k as bf16 holding the exact integer codes (Q8:
+//    q, Q4: n - 8); B = 16 k x 8 tokens of X; C = the block's dot for 16 rows
+//    x 8 tokens, exact products summed in fp32, then acc += d * C. The block
+//    scale is applied in fp32, so no decoded weight is rounded (the tcgen05
+//    path rounds q * d to bf16).
+//  * Inside a block k is permuted (the same way in A and B) so that each lane
+//    reads its codes as one run of bytes and its activations with one or two
+//    vector loads.
+//  * Consumer warp (kq, t) takes 16-row tile t and the kq-th quarter of the
+//    CTA's K blocks, for every token group; the four quarters' sums are added
+//    in order in shared memory. Rows too few for all SMs split K over a
+//    thread-block cluster (cluster rank = K range): each rank sends its sums
+//    for the rows another rank owns to that rank with remote shared-memory
+//    stores, and every rank adds, for its own rows, all ranks' sums in rank
+//    order. Deterministic, no global scratch.
+//  * With early weights the W copies are issued before the dependency wait;
+//    X is copied and Y written after it.
+
+constexpr int kSmMaxTiles = 4;  // 16-row weight tiles per CTA (R <= 64)
+constexpr int kSmKParts = 4;    // K ranges per tile inside a CTA
+constexpr int kSmWarps = kSmMaxTiles * kSmKParts;  // consumer warps: warp = (K range, tile)
+constexpr int kSmMaxM = 32;     // tokens
+
+struct alignas(64) SParams {
+  const uint8_t *W;
+  const uint16_t *X;
+  float *Y;
+  int64_t N;
+  int64_t row_bytes;
+  int64_t total_bytes;
+  int M, K, KB;
+  int groups;     // row groups (clusters of `split` CTAs)
+  int split;      // K ranges per row group
+  CUtensorMap tm_x;  // split K: X dims {K, M} bf16, box {256, 8 QM}
+  CUtensorMap tm_w;  // split K, rows a multiple of 16 bytes: W as {row_bytes / 4, N} words, box {seg_pitch / 4, rows}
+  int w_tma;         // the weight segments come as one tm_w box
+  int seg_pitch;     // split K: shared-memory bytes per weight-row segment (16-byte multiple)
+  int xjpb;          // K blocks per X row in shared memory (a box of them per 8 QM tokens)
+  int w_off, x_off, part_off;
+  int prefetch_before_wait;
+};
+
+__device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+// Not volatile: a pure function of its operands, so the compiler may overlap
+// it with the loads of the next tiles (volatile shared loads and mma kept
+// every load, conversion and mma of a warp in program order: 5 us of a 7 us
+// launch).
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Codes c0..c3 (bytes of w, two's complement) -> bf16 pairs (c0, c1), (c2, c3),
+// exact and without a conversion instruction (those issue slowly): c is exact
+// in fp32 after the 2^23 trick, and with at most 8 significant bits its bf16
+// is the upper half of that fp32.
+__device__ __forceinline__ void q8_codes_bf16(uint32_t w, uint32_t &o01, uint32_t &o23) {
+  const uint32_t q = w ^ 0x80808080u;
+  const float2 nb = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
+  float2 f01 = make_float2(__uint_as_float(__byte_perm(q, 0x4B000000u, 0x7440u)),
+                           __uint_as_float(__byte_perm(q, 0x4B000000u, 0x7441u)));
+  float2 f23 = make_float2(__uint_as_float(__byte_perm(q, 0x4B000000u, 0x7442u)),
+                           __uint_as_float(__byte_perm(q, 0x4B000000u, 0x7443u)));
+  f01 = __fadd2_rn(f01, nb);
+  f23 = __fadd2_rn(f23, nb);
+  o01 = __byte_perm(__float_as_uint(f01.x), __float_as_uint(f01.y), 0x7632u);
+  o23 = __byte_perm(__float_as_uint(f23.x), __float_as_uint(f23.y), 0x7632u);
+}
+// fp16 bits -> fp32 without a conversion instruction, exact for normal and
+// subnormal values: the exponent and fraction shifted into fp32 position read
+// as x * 2^-112 (an fp32 subnormal for an fp16 subnormal), times 2^112.
+__device__ __forceinline__ float half_bits_to_float_alu(uint32_t h) {
+  return __fmul_rn(__uint_as_float(((h & 0x8000u) << 16) | ((h & 0x7fffu) << 13)), 0x1p112f);
+}
+// Two nibbles in bits 0..3 and 16..19 of v -> bf16 pair (n - 8), exact:
+// 0x4300 | n is 128 + n, minus 136.
+__device__ __forceinline__ uint32_t q4_pair_bf16(uint32_t v) {
+  uint32_t t = (v & 0x000F000Fu) | 0x43004300u;
+  const __nv_bfloat162 k136 = __halves2bfloat162(__ushort_as_bfloat16(0x4308), __ushort_as_bfloat16(0x4308));
+  __nv_bfloat162 h = __hsub2(*reinterpret_cast<__nv_bfloat162 *>(&t), k136);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Shared-memory offset of weight row r's first block of the CTA's K range
+// (2-byte aligned): without split K the rows follow each other at the row
+// pitch from the range's offset modulo 16; with it each row segment has its
+// own slot.
+__device__ __forceinline__ uint32_t small_row_base(const SParams &p, int64_t r0, int kb0, int kbb, int r) {
+  if (p.split == 1) return static_cast<uint32_t>((r0 * p.row_bytes) & 15) + static_cast<uint32_t>(r * p.row_bytes);
+  return static_cast<uint32_t>(r * p.seg_pitch) +
+         static_cast<uint32_t>(((r0 + r) * p.row_bytes + static_cast<int64_t>(kb0) * kbb) & 15);
+}
+
+// A fragments (both k steps) and the scale of the block at shared-memory
+// offset blk; zero for a row past the last.
+template <int WT>
+__device__ __forceinline__ void small_row(const uint8_t *wbase, uint32_t blk, bool valid, int qd, uint32_t (&o)[4],
+                                          float &d) {
+  if (!valid) {
+    o[0] = o[1] = o[2] = o[3] = 0u;
+    d = 0.f;
+    return;
+  }
+  auto w32 = [&](uint32_t off) { return *reinterpret_cast<const uint32_t *>(wbase + off); };
+  d = half_bits_to_float_alu(*reinterpret_cast<const uint16_t *>(wbase + blk));
+  if constexpr (WT == QMM_Q8_0) {
+    // codes 8 qd .. 8 qd + 7 (2-byte aligned): k slots 2qd, 2qd+1 <- 0, 1 and
+    // 2qd+8, 2qd+9 <- 2, 3 (step 0); the same with 4..7 (step 1)
+    const uint32_t ca = blk + 2u + 8u * qd, mis = ca & 2u, wa = ca - mis;
+    const uint32_t v0 = w32(wa), v1 = w32(wa + 4), v2 = w32(wa + 8);
+    q8_codes_bf16(__funnelshift_r(v0, v1, mis << 3), o[0], o[1]);
+    q8_codes_bf16(__funnelshift_r(v1, v2, mis << 3), o[2], o[3]);
+  } else {
+    // bytes 4 qd .. 4 qd + 3: low nibbles = elements 4qd + i, high = 16 + 4qd + i;
+    // k slots 2qd, 2qd+1 <- elements (0, 2), 2qd+8, 2qd+9 <- (1, 3), low (step 0) then high (step 1)
+    const uint32_t ca = blk + 2u + 4u * qd, mis = ca & 2u, wa = ca - mis;
+    const uint32_t v = __funnelshift_r(w32(wa), w32(wa + 4), mis << 3);
+    o[0] = q4_pair_bf16(v);
+    o[1] = q4_pair_bf16(v >> 8);
+    o[2] = q4_pair_bf16(v >> 4);
+    o[3] = q4_pair_bf16(v >> 12);
+  }
+}
+
+template <int WT, int QM>  // QM token groups of eight (M <= 8 QM)
+__global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(const __grid_constant__ SParams p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint64_t *wbar = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *xbar = wbar + 1;
+  constexpr int kBB = WT == QMM_Q8_0 ? 34 : 18;
+  constexpr int kCols = 8 * QM;  // token columns of the partial sums
+  const int xrow = 64 * p.xjpb;            // bytes per token row of an X box
+  const int xbox = 8 * QM * xrow;           // bytes of one X box
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = p.split;
+  const int zr = split > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int grp = static_cast<int>(blockIdx.x) / split;
+  const int64_t r0 = static_cast<int64_t>(grp) * p.N / p.groups;
+  const int R = static_cast<int>((static_cast<int64_t>(grp) + 1) * p.N / p.groups - r0);
+  const int kb0 = zr * p.KB / split, kb1 = (zr + 1) * p.KB / split;
+  const int nb = kb1 - kb0;
+  const uint32_t sbase = smem_u32(smem);
+
+  pdl_launch_dependents();
+  if (tid == 0) {
+    mbar_init(wbar, 1);
+    mbar_init(xbar, 1);
+    fence_mbar_init();
+  }
+  // without split K, token rows M .. 8 QM - 1 of X are not copied: zero
+  if (split == 1)
+    for (int i = tid; i < (kCols - p.M) * xrow / 4; i += blockDim.x)
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(smem_u32(smem) + static_cast<uint32_t>(p.x_off + p.M * xrow + 4 * i)),
+                   "r"(0u)
+                   : "memory");
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // Weights: segment [s, e) of W widened to 16-byte boundaries [a, b); the
+    // bytes of the last stretch of W past its last 16-byte boundary `lim` by
+    // plain loads, before the arrival that counts the bulk bytes.
+    const int64_t lim = p.total_bytes & ~int64_t(15);
+    auto seg = [&](int i, int64_t &s0, int64_t &e0, int64_t &a, int64_t &b) {
+      if (split == 1) {  // all rows of the CTA: one contiguous range
+        s0 = r0 * p.row_bytes;
+        e0 = (r0 + R) * p.row_bytes;
+      } else {
+        s0 = (r0 + i) * p.row_bytes + static_cast<int64_t>(kb0) * kBB;
+        e0 = (r0 + i) * p.row_bytes + static_cast<int64_t>(kb1) * kBB;
+      }
+      a = s0 & ~int64_t(15);
+      b = min((e0 + 15) & ~int64_t(15), max(lim, a));
+    };
+    const int nseg = split == 1 ? (R > 0 ? 1 : 0) : R;
+    auto issue_w = [&]() {
+      if (p.w_tma) {  // every row segment of the group in one box (rows past N read as zero)
+        if (lane == 0 && R > 0) {
+          mbar_arrive_expect_tx(wbar, static_cast<uint32_t>(p.seg_pitch * ((p.N + p.groups - 1) / p.groups)));
+          tma_load_2d(smem + p.w_off, &p.tm_w, static_cast<int>(((static_cast<int64_t>(kb0) * kBB) & ~int64_t(15)) / 4),
+                      static_cast<int>(r0), wbar);
+        } else if (lane == 0) {
+          mbar_arrive(wbar);
+        }
+        return;
+      }
+      if (lane == 0) {
+        uint32_t bytes = 0;
+        for (int i = 0; i < nseg; ++i) {
+          int64_t s0, e0, a, b;
+          seg(i, s0, e0, a, b);
+          uint8_t *dst = smem + p.w_off + static_cast<int64_t>(i) * p.seg_pitch;
+          for (int64_t t = b; t < e0; ++t) dst[t - a] = p.W[t];
+          bytes += static_cast<uint32_t>(b - a);
+        }
+        mbar_arrive_expect_tx(wbar, bytes);
+      }
+      __syncwarp();
+      const uint64_t pol = l2_evict_first_policy();
+      for (int i = lane; i < nseg; i += 32) {
+        int64_t s0, e0, a, b;
+        seg(i, s0, e0, a, b);
+        uint8_t *dst = smem + p.w_off + static_cast<int64_t>(i) * p.seg_pitch;
+        for (int64_t o = 0; o < b - a; o += 65536)
+          bulk_g2s(dst + o, p.W + a + o, static_cast<uint32_t>(b - a - o < 65536 ? b - a - o : 65536), wbar, pol);
+      }
+    };
+    auto issue_x = [&]() {
+      if (lane != 0) return;
+      if (split == 1) {  // the whole of X: one range
+        const uint32_t len = static_cast<uint32_t>(p.M) * static_cast<uint32_t>(p.K) * 2u;
+        mbar_arrive_expect_tx(xbar, len);
+        const uint64_t pol = l2_evict_last_policy();
+        for (uint32_t o = 0; o < len; o += 65536)
+          bulk_g2s(smem + p.x_off + o, p.X + o / 2, len - o < 65536u ? len - o : 65536u, xbar, pol);
+      } else {  // boxes of xjpb blocks x 8 QM tokens
+        const int nbox = (nb + p.xjpb - 1) / p.xjpb;
+        mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(nbox * xbox));
+        for (int bx = 0; bx < nbox; ++bx)
+          tma_load_2d(smem + p.x_off + bx * xbox, &p.tm_x, 32 * (kb0 + p.xjpb * bx), 0, xbar);
+      }
+    };
+    if (p.prefetch_before_wait) {
+      issue_w();
+      pdl_wait();
+      issue_x();
+    } else {
+      pdl_wait();
+      issue_w();
+      issue_x();
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int cw = warp - 1;
+    const int t = cw % kSmMaxTiles, kq = cw / kSmMaxTiles;  // this warp's tile and K range
+    const int g = lane >> 2, qd = lane & 3;
+    float acc[QM][4];
+#pragma unroll
+    for (int q = 0; q < QM; ++q)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[q][i] = 0.f;
+    bool ok = mbar_wait(wbar, 0);
+    ok = mbar_wait(xbar, 0) && ok;
+    ok = __all_sync(0xffffffffu, ok);  // the mma.sync loop below needs the whole warp
+    if (!ok) {
+      // record, then wait once more for copies still in flight before the
+      // buffers are reused and the CTA exits
+      if (lane == 0) atomicOr(&g_prefill_status, kDevTimeoutFull);
+      if (!mbar_wait(wbar, 0) || !mbar_wait(xbar, 0))
+        if (lane == 0) atomicOr(&g_prefill_status, kDevTimeoutDrain);
+    }
+    const int T = (R + 15) / 16;
+    const uint8_t *wbase = smem + p.w_off;
+    const int jb = kq * nb / kSmKParts, je = (kq + 1) * nb / kSmKParts;
+    // loop-invariant addresses: rows 16t + g and + 8, token row g of block jb
+    // (block j of token 8q + g: box j / xjpb, row 8q + g, 64 bytes at (j mod xjpb) * 64)
+    const bool va = 16 * t + g < R, vb = 16 * t + g + 8 < R;
+    uint32_t ba = va ? small_row_base(p, r0, kb0, kBB, 16 * t + g) + static_cast<uint32_t>(jb * kBB) : 0u;
+    uint32_t bb = vb ? small_row_base(p, r0, kb0, kBB, 16 * t + g + 8) + static_cast<uint32_t>(jb * kBB) : 0u;
+    int jx = jb % p.xjpb;
+    const uint8_t *xg = smem + p.x_off + (jb / p.xjpb) * xbox + g * xrow + 64 * jx;
+    for (int j = jb; ok && t < T && j < je; ++j) {
+      // B fragments of block j for every token group: b[q][2 s + h]
+      uint32_t bq[QM][4];
+#pragma unroll
+      for (int q = 0; q < QM; ++q) {
+        const uint8_t *xr = xg + 8 * q * xrow;
+        if constexpr (WT == QMM_Q8_0) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(xr + 16 * qd);  // elements 8qd .. 8qd + 7
+          bq[q][0] = v.x;
+          bq[q][1] = v.y;
+          bq[q][2] = v.z;
+          bq[q][3] = v.w;
+        } else {
+          // elements 4qd .. 4qd + 3 and 16 + 4qd .. 16 + 4qd + 3
+          const uint2 lo = *reinterpret_cast<const uint2 *>(xr + 8 * qd);
+          const uint2 hi = *reinterpret_cast<const uint2 *>(xr + 32 + 8 * qd);
+          bq[q][0] = __byte_perm(lo.x, lo.y, 0x5410u);
+          bq[q][1] = __byte_perm(lo.x, lo.y, 0x7632u);
+          bq[q][2] = __byte_perm(hi.x, hi.y, 0x5410u);
+          bq[q][3] = __byte_perm(hi.x, hi.y, 0x7632u);
+        }
+      }
+      uint32_t oa[4], ob[4];
+      float da, db;
+      small_row<WT>(wbase, ba, va, qd, oa, da);
+      small_row<WT>(wbase, bb, vb, qd, ob, db);
+      ba += kBB;
+      bb += kBB;
+      xg += 64;
+      if (++jx == p.xjpb) {  // next box
+        jx = 0;
+        xg += xbox - 64 * p.xjpb;
+      }
+      const uint32_t a0[4] = {oa[0], ob[0], oa[1], ob[1]};  // k step 0
+      const uint32_t a1[4] = {oa[2], ob[2], oa[3], ob[3]};  // k step 1
+#pragma unroll
+      for (int q = 0; q < QM; ++q) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_bf16_16816(c, a0, bq[q][0], bq[q][1]);
+        mma_bf16_16816(c, a1, bq[q][2], bq[q][3]);
+        acc[q][0] = __fmaf_rn(da, c[0], acc[q][0]);
+        acc[q][1] = __fmaf_rn(da, c[1], acc[q][1]);
+        acc[q][2] = __fmaf_rn(db, c[2], acc[q][2]);
+        acc[q][3] = __fmaf_rn(db, c[3], acc[q][3]);
+      }
+    }
+    // every consumer is past its last read of W and X: their space takes the
+    // warps' sums red[warp][group][lane] (float4)
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kSmWarps) : "memory");
+    const uint32_t red = sbase + static_cast<uint32_t>(p.w_off);
+#pragma unroll
+    for (int q = 0; q < QM; ++q)
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                       red + static_cast<uint32_t>(((cw * QM + q) * 32 + lane) * 16)),
+                   "f"(acc[q][0]), "f"(acc[q][1]), "f"(acc[q][2]), "f"(acc[q][3])
+                   : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kSmWarps) : "memory");
+    // (r, m): the K ranges' sums in order; kept in part[r][m] without split K,
+    // else stored into the owner rank's slot recv[source rank][row of the owner][m]
+    const int ctid = tid - 32;
+    const int rpr = (R + split - 1) / split;  // rows per rank share (at most)
+    for (int o = ctid; o < R * kCols; o += 32 * kSmWarps) {
+      const int r = o / kCols, m = o % kCols;
+      const int tt = r >> 4, rr = r & 15, q = m >> 3, mm = m & 7;
+      const int ln = (rr & 7) * 4 + (mm >> 1), i = (rr >> 3) * 2 + (mm & 1);
+      float v = 0.f;
+#pragma unroll
+      for (int k = 0; k < kSmKParts; ++k)
+        v += lds_f32(red + static_cast<uint32_t>(((((k * kSmMaxTiles + tt) * QM + q) * 32 + ln) * 4 + i) * 4));
+      if (split == 1) {
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(sbase + static_cast<uint32_t>(p.part_off + 4 * (r * (kCols + 1) + m))),
+                     "f"(v)
+                     : "memory");
+      } else {
+        const int own = r / rpr;  // owner rank of row r
+        const uint32_t la =
+            sbase + static_cast<uint32_t>(p.part_off + 4 * (((zr * rpr) + (r - own * rpr)) * (kCols + 1) + m));
+        if (own == zr)
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(la), "f"(v) : "memory");
+        else
+          st_cluster_b32(map_rank(la, static_cast<uint32_t>(own)), __float_as_uint(v));
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ output
+  __syncthreads();
+  pdl_wait();  // (Y is written only after the preceding grid; a no-op by now)
+  if (split == 1) {
+    for (int o = tid; o < R * p.M; o += blockDim.x) {
+      const int m = o / R, r = o % R;
+      p.Y[static_cast<int64_t>(m) * p.N + r0 + r] =
+          lds_f32(sbase + static_cast<uint32_t>(p.part_off + 4 * (r * (kCols + 1) + m)));
+    }
+  } else {
+    cluster_sync_all();  // every rank's sums have landed in their owners' slots
+    const int rpr = (R + split - 1) / split;
+    const int rb = zr * rpr, re = min(R, rb + rpr);  // this rank's rows of the group
+    const uint32_t pa = sbase + static_cast<uint32_t>(p.part_off);
+    for (int o = tid; o < (re - rb) * p.M; o += blockDim.x) {
+      const int m = o / (re - rb), lr = o % (re - rb);
+      float v = 0.f;
+      for (int src = 0; src < split; ++src)
+        v += lds_f32(pa + static_cast<uint32_t>(4 * ((src * rpr + lr) * (kCols + 1) + m)));
+      p.Y[static_cast<int64_t>(m) * p.N + r0 + rb + lr] = v;
+    }
+    // no remote access after the barrier above: a rank may leave
+  }
+}
+
+template <int WT, int QM>
+void *small_kernel_ptr() {
+  return reinterpret_cast<void *>(prefill_small_kernel<WT, QM>);
+}
+
+// Small-M launch: one wave of clusters of `split` CTAs along K, each cluster a
+// group of at most 64 rows; the split is the one that moves the fewest bytes
+// into a CTA (its W share plus its X slice). False when M is too large or no
+// split fits (the tcgen05 path takes over).
+bool try_launch_small(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W, const uint16_t *X,
+                      float *Y, cudaStream_t stream, uint32_t flags, PrefillPlan *plan, qmm_status *out) {
+  if (M > kSmMaxM) return false;
+  const int KB = K / 32, bb = wtype == QMM_Q8_0 ? 34 : 18;
+  const int QM = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
+  void *kerns[2][3] = {{small_kernel_ptr<QMM_Q8_0, 1>(), small_kernel_ptr<QMM_Q8_0, 2>(), small_kernel_ptr<QMM_Q8_0, 4>()},
+                       {small_kernel_ptr<QMM_Q4_0, 1>(), small_kernel_ptr<QMM_Q4_0, 2>(), small_kernel_ptr<QMM_Q4_0, 4>()}};
+  void *kern = kerns[wtype][QM == 1 ? 0 : (QM == 2 ? 1 : 2)];
+  static bool configured[2][64] = {};
+  if (dev.device >= 0 && dev.device < 64 && !configured[wtype][dev.device]) {
+    for (int i = 0; i < 3; ++i) {
+      cudaError_t e = cudaFuncSetAttribute(kerns[wtype][i], cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
+      if (e != cudaSuccess) {
+        *out = cuda_check(e, "prefill attribute");
+        return true;
+      }
+    }
+    configured[wtype][dev.device] = true;
+  }
+
+  struct Layout {
+    int split, groups, rmax, seg_pitch, xjpb, w_tma, w_off, x_off, part_off;
+    size_t smem;
+    int64_t cost;
+  };
+  const int64_t row_bytes = static_cast<int64_t>(bb) * KB;
+  auto layout = [&](int split, int64_t groups) -> Layout {
+    Layout l{};
+    l.split = split;
+    l.groups = static_cast<int>(groups);
+    const int nbm = (KB + split - 1) / split;
+    const int R = static_cast<int>((N + groups - 1) / groups);
+    // split K: a slot per row segment, the segment plus up to 15 bytes of
+    // alignment on either side; otherwise the rows' contiguous range plus 32
+    l.rmax = R;
+    l.seg_pitch = round_up(nbm * bb + 30, 16);
+    l.w_tma = split > 1 && row_bytes % 16 == 0 && l.seg_pitch <= 1024;  // a TMA box row: at most 256 words
+    const int64_t wbytes = split == 1 ? R * row_bytes + 32 : static_cast<int64_t>(R) * l.seg_pitch;
+    // X rows: the whole K without split (one copy), else boxes of 8 blocks
+    l.xjpb = split == 1 ? KB : 8;
+    const int64_t xbytes = static_cast<int64_t>((nbm + l.xjpb - 1) / l.xjpb) * 8 * QM * 64 * l.xjpb;
+    const int red = kSmWarps * QM * 32 * 16;
+    l.w_off = 128;
+    if (wbytes + xbytes > (1 << 20)) {
+      l.smem = SIZE_MAX;
+      return l;
+    }
+    l.x_off = round_up(l.w_off + static_cast<int>(wbytes), 128);
+    l.part_off = round_up(std::max(l.x_off + static_cast<int>(xbytes), l.w_off + red), 16);
+    // part: R rows x (8 QM + 1) floats; with split K the owner's slots, split x ceil(R / split) rows
+    const int prow = split == 1 ? R : split * ((R + split - 1) / split);
+    l.smem = static_cast<size_t>(l.part_off) + static_cast<size_t>(prow) * (8 * QM + 1) * 4 + 128;  // + base alignment
+    l.cost = static_cast<int64_t>(R) * nbm * bb + M * nbm * 64;
+    return l;
+  };
+
+  cudaLaunchConfig_t cfg{};
+  cfg.blockDim = dim3((kSmWarps + 1) * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  cfg.attrs = attr;
+
+  // candidates by their cost with one wave of groups, then checked for
+  // cluster residency (fewer groups, larger ones, when not all fit at once)
+  const int64_t gmin = (N + kSmMaxTiles * 16 - 1) / (kSmMaxTiles * 16);
+  Layout cand[kMaxSplit];
+  int nc = 0;
+  for (int s = 1; s <= kMaxSplit && s <= KB; ++s) {
+    const int64_t gmax = std::min<int64_t>(dev.sms / s, N);
+    if (gmax < gmin) continue;
+    const Layout l = layout(s, gmax);
+    if (l.smem <= static_cast<size_t>(dev.smem_optin)) cand[nc++] = l;
+  }
+  std::sort(cand, cand + nc, [](const Layout &a, const Layout &b) {
+    return a.cost != b.cost ? a.cost < b.cost : a.split < b.split;
+  });
+  Layout best{};
+  bool found = false;
+  for (int i = 0; i < nc; ++i) {
+    if (found && cand[i].cost >= best.cost) break;
+    Layout l = cand[i];
+    if (l.split > 1) {
+      cfg.gridDim = dim3(static_cast<unsigned>(l.groups * l.split));
+      cfg.dynamicSmemBytes = l.smem;
+      attr[1].val.clusterDim.x = static_cast<unsigned>(l.split);
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = 1;
+      cfg.numAttrs = 2;
+      int active = 0;
+      if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();  // a refused query is not an error of this call
+        continue;
+      }
+      if (active < l.groups) {
+        if (active < gmin) continue;
+        l = layout(l.split, active);
+        if (l.smem > static_cast<size_t>(dev.smem_optin)) continue;
+      }
+    }
+    if (!found || l.cost < best.cost) {
+      best = l;
+      found = true;
+    }
+  }
+  if (!found) return false;
+
+  if (plan) {
+    *plan = PrefillPlan{8 * QM, best.split, 0, best.groups * best.split, 1};
+    *out = QMM_OK;
+    return true;
+  }
+  SParams p{};
+  p.W = static_cast<const uint8_t *>(W);
+  p.X = X;
+  p.Y = Y;
+  p.N = N;
+  p.row_bytes = static_cast<int64_t>(bb) * KB;
+  p.total_bytes = N * p.row_bytes;
+  p.M = static_cast<int>(M);
+  p.K = K;
+  p.KB = KB;
+  p.groups = best.groups;
+  p.split = best.split;
+  p.seg_pitch = best.seg_pitch;
+  p.xjpb = best.xjpb;
+  p.w_tma = best.w_tma;
+  if (best.split > 1) {
+    const uint64_t xd[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint64_t xs[1] = {static_cast<uint64_t>(K) * 2};
+    const uint32_t xb[2] = {256, static_cast<uint32_t>(8 * QM)};
+    qmm_status st = encode_tiled(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, xd, xs, xb, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st == QMM_OK && best.w_tma) {
+      const uint64_t wd[2] = {static_cast<uint64_t>(row_bytes / 4), static_cast<uint64_t>(N)};
+      const uint64_t ws[1] = {static_cast<uint64_t>(row_bytes)};
+      const uint32_t wb[2] = {static_cast<uint32_t>(best.seg_pitch / 4), static_cast<uint32_t>(best.rmax)};
+      st = encode_tiled(&p.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, W, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    if (st != QMM_OK) {
+      *out = st;
+      return true;
+    }
+  }
+  p.w_off = best.w_off;
+  p.x_off = best.x_off;
+  p.part_off = best.part_off;
+  p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
+  cfg.gridDim = dim3(static_cast<unsigned>(best.groups * best.split));
+  cfg.dynamicSmemBytes = best.smem;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(best.split);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.numAttrs = best.split > 1 ? 2 : 1;
+  void *args[] = {&p};
+  *out = cuda_check(cudaLaunchKernelExC(&cfg, kern, args), "prefill launch");
+  return true;
+}
+
 }  // namespace
 
 qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,
                           const uint16_t *X, float *Y, cudaStream_t stream, uint32_t flags, PrefillPlan *plan) {
+  {
+    qmm_status st = QMM_OK;
+    if (try_launch_small(dev, wtype, M, N, K, W, X, Y, stream, flags, plan, &st)) return st;
+  }
   Params p{};
   p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
   p.W = static_cast<const uint8_t *>(W);
@@ -689,7 +1270,7 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
   const int64_t mtiles = (M + p.MT - 1) / p.MT;
   if (ntiles > 65535 || mtiles > 0x7fffffff) return set_error(QMM_ERR_SHAPE, "prefill: grid too large");
   if (plan) {
-    *plan = PrefillPlan{p.MT, split, p.stages, static_cast<int>(ntiles * mtiles * split)};
+    *plan = PrefillPlan{p.MT, split, p.stages, static_cast<int>(ntiles * mtiles * split), 0};
     return QMM_OK;
   }
 

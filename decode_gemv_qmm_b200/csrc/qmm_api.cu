@@ -451,6 +451,7 @@ QMM_API qmm_status qmm_prefill_plan(int wtype, int64_t M, int64_t N, int64_t K, 
   plan[1] = pl.split;
   plan[2] = pl.stages;
   plan[3] = pl.ctas;
+  plan[4] = pl.kind;
   return QMM_OK;
 }
 

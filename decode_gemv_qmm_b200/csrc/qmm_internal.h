@@ -61,9 +61,10 @@ qmm_status launch_q4_gateup_unfused(const DevInfo &dev, int M, int64_t N, int K,
                                     const float *X, float *G, float *U, float *Y, cudaStream_t stream);
 
 // The tiling launch_prefill picks: tokens per tile, K ranges per tile
-// (cluster size), MMA stages in flight and CTAs of the launch.
+// (cluster size), MMA stages in flight (0 for the small-M kernel), CTAs of the
+// launch, and the kernel (0: tcgen05 tiles, 1: small-M mma.sync).
 struct PrefillPlan {
-  int mt, split, stages, ctas;
+  int mt, split, stages, ctas, kind;
 };
 // With `plan` set, only the tiling is computed (nothing is launched).
 qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,

@@ -377,8 +377,11 @@ QMM_API qmm_status qmm_q4_gateup_unfused(int64_t M, int64_t N, int64_t K, int bl
  * current device for this problem, without launching anything:
  * plan[0] = tokens per output tile (MT; above 256 each k step takes two
  * MMAs), plan[1] = K ranges per tile (thread-block cluster size, 1 = no
- * split), plan[2] = MMA stages in flight, plan[3] = CTAs of the launch.
- * Host memory `plan` (4 int32, written). Needs an sm_100 device
+ * split), plan[2] = MMA stages in flight (0 for the small-M kernel),
+ * plan[3] = CTAs of the launch, plan[4] = the kernel: 0 = tcgen05 tiles with
+ * the A operand in tensor memory, 1 = the small-M kernel (M <= 32: each CTA's
+ * weight share and X slice in shared memory, mma.sync bf16).
+ * Host memory `plan` (5 int32, written). Needs an sm_100 device
  * (QMM_ERR_DEVICE otherwise); M, N >= 1, K >= 32 (QMM_ERR_SHAPE).
  */
 QMM_API qmm_status qmm_prefill_plan(int wtype, int64_t M, int64_t N, int64_t K, int block, int32_t *plan);

@@ -122,9 +122,13 @@ def test_prefill_plan_wide_tiles_for_a_nearly_empty_last_wave():
         assert p["stages"] >= 3, p
     # 544 tiles of 256 tokens against 408 of 352: four waves against three, no gain
     assert qmm.qmm_prefill_plan(syn.Q4_0, 1024, 17408, 5120)["mt"] == 256
-    # few tiles: narrow tiles and split K
+    assert qmm.qmm_prefill_plan(syn.Q8_0, 1024, 4864, 896)["kernel"] == "tcgen05"
+    # 32 tokens: the small-M kernel, K split over a cluster where rows are few
     p = qmm.qmm_prefill_plan(syn.Q8_0, 32, 4864, 896)
-    assert p["mt"] == 32 and p["split"] > 1, p
+    assert p["kernel"] == "small_m" and p["split"] == 1 and p["ctas"] <= sms, p
+    p = qmm.qmm_prefill_plan(syn.Q8_0, 32, 896, 4864)
+    assert p["kernel"] == "small_m" and p["split"] > 1, p
+    assert qmm.qmm_prefill_plan(syn.Q8_0, 33, 896, 4864)["kernel"] == "tcgen05"
 
 
 @pytest.mark.parametrize("wtype", [syn.Q8_0, syn.Q4_0])
