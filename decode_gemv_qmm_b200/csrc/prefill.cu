@@ -728,7 +728,10 @@ __device__ __forceinline__ void small_row(const uint8_t *wbase, uint32_t blk, bo
 template <int WT, int QM>  // QM token groups of eight (M <= 8 QM)
 __global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(const __grid_constant__ SParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  // 128-byte aligned base, derived by pointer arithmetic on the shared array so
+  // that the compiler keeps plain loads through it in the shared address space
+  // (a round trip through an integer made them generic loads)
+  uint8_t *smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
   uint64_t *wbar = reinterpret_cast<uint64_t *>(smem);
   uint64_t *xbar = wbar + 1;
   constexpr int kBB = WT == QMM_Q8_0 ? 34 : 18;
