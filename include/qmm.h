@@ -51,7 +51,8 @@
  *
  * Tolerances the library is tested to (per output, S = sum_k |w_k * x_k|):
  *   fp32-accumulated paths: |y - exact| <= 1e-5 * S;
- *   bf16 tensor-core prefill: |y - exact| <= 4e-3 * S;
+ *   bf16 tensor-core prefill above 32 tokens: |y - exact| <= 4e-3 * S
+ *   (up to 32 tokens the prefill path is held to 1e-5 * S);
  *   activation codes and int32 block dots: bit-exact.
  */
 #ifndef QMM_H
@@ -326,10 +327,13 @@ QMM_API qmm_status qmm_q4_gemv(int64_t M, int64_t N, int64_t K, int block, const
  * qmm_quant_matmul_prefill -- prefill panel Y = X . W^T on the tensor cores.
  *
  * "LSE v0.4.16", section "Retained optimizations and compatibility" (M1024
- * prefill panels): a many-token matmul against block-quantized weights. The
- * blocks are decoded to bf16 (w = q*d rounded to nearest even) in shared
- * memory and multiplied by bf16 activations with fp32 accumulation on the
- * tcgen05 tensor cores.
+ * prefill panels): a many-token matmul against block-quantized weights.
+ * Above 32 tokens the blocks are decoded to bf16 (w = q*d rounded to nearest
+ * even) and multiplied by the bf16 activations with fp32 accumulation on the
+ * tcgen05 tensor cores (|y - exact| <= 4e-3 * S). Up to 32 tokens a small-M
+ * kernel multiplies the exact integer codes by the activations (mma.sync,
+ * fp32 accumulation) and applies each block's d in fp32, so no decoded weight
+ * is rounded (|y - exact| <= 1e-5 * S). qmm_prefill_plan tells which runs.
  *
  *   wtype   QMM_Q8_0 or QMM_Q4_0 (QMM_ERR_DTYPE otherwise)
  *   M       tokens, >= 0
