@@ -118,15 +118,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both K-major; accumulate when `acc`.
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc ? 1u : 0u)
-      : "memory");
-}
 // D[tmem] (+)= A[tmem] * B[smem]^T: A is 128 lanes (rows) x K packed two
 // bf16 per 32-bit column, B K-major in shared memory.
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, bool acc) {
@@ -163,8 +154,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-// Generic-proxy shared-memory writes -> visible to the async proxy (the MMA).
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // K-major, 128-byte swizzle, 8-row atoms 1024 bytes apart (SM100 descriptor).
 __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
@@ -196,11 +185,6 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
 }
 __device__ __forceinline__ void st_cluster_b32(uint32_t addr, uint32_t a) {
@@ -637,11 +621,6 @@ struct alignas(64) SParams {
   int prefetch_before_wait;
 };
 
-__device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
 // Not volatile: a pure function of its operands, so the compiler may overlap
 // it with the loads of the next tiles (volatile shared loads and mma kept
 // every load, conversion and mma of a warp in program order: 5 us of a 7 us
@@ -727,11 +706,11 @@ __device__ __forceinline__ void small_row(const uint8_t *wbase, uint32_t blk, bo
 
 template <int WT, int QM>  // QM token groups of eight (M <= 8 QM)
 __global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(const __grid_constant__ SParams p) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
+  extern __shared__ __align__(128) uint8_t smem_sm[];
   // 128-byte aligned base, derived by pointer arithmetic on the shared array so
   // that the compiler keeps plain loads through it in the shared address space
   // (a round trip through an integer made them generic loads)
-  uint8_t *smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+  uint8_t *smem = smem_sm + ((128u - (smem_u32(smem_sm) & 127u)) & 127u);
   uint64_t *wbar = reinterpret_cast<uint64_t *>(smem);
   uint64_t *xbar = wbar + 1;
   constexpr int kBB = WT == QMM_Q8_0 ? 34 : 18;
