@@ -4,7 +4,7 @@ Argument marshalling only -- every step of every operation runs in the CUDA
 kernels of libqmm.so. Functions carry the names of the C entry points
 (include/qmm.h) and take torch tensors for device buffers; PyTorch supplies
 device memory and streams, nothing else. Importing this package fails loudly
-if the library has not been built (``python -m decode_gemv_qmm_b200.build``);
+if the library has not been built (``python decode_gemv_qmm_b200/build.py``);
 there is no fallback of any kind.
 """
 from __future__ import annotations
@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqmm.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m decode_gemv_qmm_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python decode_gemv_qmm_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 

@@ -1,6 +1,6 @@
 """Build libqmm.so in-tree with nvcc for sm_100a (no GPU needed to build).
 
-    python -m decode_gemv_qmm_b200.build [--force] [-v]
+    python decode_gemv_qmm_b200/build.py [--force] [-v]
 
 Each csrc/*.cu is compiled to an object under _build/ (in parallel, only when
 it or a header changed) and the objects are linked into
