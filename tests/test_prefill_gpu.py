@@ -141,3 +141,15 @@ def test_prefill_wide_token_tiles(wtype, m, n, k):
     if sms == 148:
         assert plan["mt"] > 256 and plan["split"] == 1, plan
     check_full(wtype, m, n, k, seed=7 * m + n + k)
+
+
+@pytest.mark.parametrize("wtype", [syn.Q8_0, syn.Q4_0])
+@pytest.mark.parametrize("m,n,k", [(16, 12000, 256), (32, 9600, 288)])
+def test_prefill_few_tokens_many_rows_on_tcgen05_tiles(wtype, m, n, k):
+    """At most 32 tokens but more rows than one wave of 64-row groups: the small-M kernel
+    does not apply and the tcgen05 tiles (16 / 32 tokens wide) take the panel."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plan = qmm.qmm_prefill_plan(wtype, m, n, k)
+    if (n + 63) // 64 > sms:
+        assert plan["kernel"] == "tcgen05" and plan["mt"] == m, plan
+    check_full(wtype, m, n, k, seed=11 * m + n + k)
