@@ -485,7 +485,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
 // loads its whole weight slice (before griddepcontrol.wait when allowed),
 // decodes every block it owns into registers as exact fp32 codes (plus the
 // block scale), and after the activations arrive does only packed FMAs, one
-// multiply by d per block, one reduce-scatter and the store.
+// multiply by d per block, one reduce-scatter and the store. With four rows a
+// warp (long rows) the codes are held as exact fp16 pairs instead, half the
+// registers, and widened to fp32 after the wait (the products are the same).
 //
 // Warp (window cw, row slot k) owns block column 32*cw + lane of rows
 // r_begin + k + U*... (U rows, stride wpw); windows of a row are added by the
@@ -514,7 +516,10 @@ struct alignas(64) RParams {
 };
 
 template <int U>
-__global__ void __launch_bounds__(U == 1 ? 512 : (U == 2 ? 512 : 352), 1)
+// At most 112 registers for U = 4: 320 threads x 112 fit one SM beside a CTA
+// of the tensor-core resident kernel (224 x 128), so the down projection can
+// start and fetch its weights while the preceding up projection runs.
+__global__ void __maxnreg__(U == 4 ? 112 : 128)
 q8_gemv_resident_kernel(const __grid_constant__ RParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -572,7 +577,11 @@ q8_gemv_resident_kernel(const __grid_constant__ RParams p) {
   const int col = cw * 32 + lane;
   const bool act = col < p.KB;
   const uint32_t wbase = smem_u32(smem + p.w_off) + static_cast<uint32_t>(b0 - a0);
-  float2 wq[U][16];
+  // U = 4 (long rows, 168 registers with fp32 codes): the codes are kept as
+  // exact fp16 pairs, half the registers, widened to fp32 after the wait
+  constexpr bool kH = U == 4;
+  float2 wq[kH ? 1 : U][16];
+  uint32_t wh[kH ? U : 1][16];
   float wd[U];
   bool ok = mbar_wait(wbar, 0);
   if (!ok && lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
@@ -588,20 +597,33 @@ q8_gemv_resident_kernel(const __grid_constant__ RParams p) {
       const uint32_t r8 = mis << 3, sh = 16u + r8;
       wd[u] = half_bits_to_float(__funnelshift_rc(w[0], w[1], r8));
       const float2 nb = make_float2(-8388736.0f, -8388736.0f);
+      const __half2 k1152 = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint32_t q4 = __funnelshift_rc(w[i], w[i + 1], sh) ^ 0x80808080u;
-        const float2 f01 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7440u)),
-                                       __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7441u)));
-        const float2 f23 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7442u)),
-                                       __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7443u)));
-        wq[u][2 * i] = __fadd2_rn(f01, nb);  // exact codes q
-        wq[u][2 * i + 1] = __fadd2_rn(f23, nb);
+        if constexpr (kH) {
+          // 0x6400 | (q + 128) is 1024 + q + 128 in fp16; minus 1152: q, exact
+          uint32_t t01 = __byte_perm(q4, 0x6464u, 0x5140u), t23 = __byte_perm(q4, 0x6464u, 0x5342u);
+          __half2 h01 = __hsub2(*reinterpret_cast<__half2 *>(&t01), k1152);
+          __half2 h23 = __hsub2(*reinterpret_cast<__half2 *>(&t23), k1152);
+          wh[u][2 * i] = *reinterpret_cast<uint32_t *>(&h01);
+          wh[u][2 * i + 1] = *reinterpret_cast<uint32_t *>(&h23);
+        } else {
+          const float2 f01 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7440u)),
+                                         __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7441u)));
+          const float2 f23 = make_float2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7442u)),
+                                         __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7443u)));
+          wq[kH ? 0 : u][2 * i] = __fadd2_rn(f01, nb);  // exact codes q
+          wq[kH ? 0 : u][2 * i + 1] = __fadd2_rn(f23, nb);
+        }
       }
     } else {
       wd[u] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) wq[u][i] = make_float2(0.f, 0.f);
+      for (int i = 0; i < 16; ++i) {
+        if constexpr (kH) wh[u][i] = 0u;
+        else wq[kH ? 0 : u][i] = make_float2(0.f, 0.f);
+      }
     }
   }
 
@@ -630,10 +652,14 @@ q8_gemv_resident_kernel(const __grid_constant__ RParams p) {
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     float2 a[4];
+    auto wv = [&](int i) -> float2 {
+      if constexpr (kH) return __half22float2(*reinterpret_cast<const __half2 *>(&wh[u][i]));
+      else return wq[kH ? 0 : u][i];
+    };
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = __fmul2_rn(wq[u][i], x2[i]);
+    for (int i = 0; i < 4; ++i) a[i] = __fmul2_rn(wv(i), x2[i]);
 #pragma unroll
-    for (int i = 4; i < 16; ++i) a[i & 3] = __ffma2_rn(wq[u][i], x2[i], a[i & 3]);
+    for (int i = 4; i < 16; ++i) a[i & 3] = __ffma2_rn(wv(i), x2[i], a[i & 3]);
     const float2 t = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
     part[u] = wd[u] * (t.x + t.y);
   }
