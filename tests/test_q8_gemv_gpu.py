@@ -179,8 +179,8 @@ def test_single_row_zero_activation_gives_exact_zero():
     (1200, 2048),  # one or two groups per CTA, seven warps of five block pairs
     (3000, 1024),  # three groups per CTA
     (9000, 512),   # eight groups per CTA
-    (600, 5120),   # long rows: register-resident kernel (fp16 codes with four rows a warp)
-    (893, 4864),   # long rows, ragged N: the same
+    (600, 5120),   # long rows: register-resident kernel, two rows a warp (fp32 codes)
+    (893, 4864),   # long rows, ragged N: four rows a warp (fp16 codes)
 ])
 def test_single_row_large_slices(n, k):
     # M = 1 slices large enough for the tensor-core resident kernel (short rows)
