@@ -847,7 +847,9 @@ __global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(c
     uint32_t bb = vb ? small_row_base(p, r0, kb0, kBB, 16 * t + g + 8) + static_cast<uint32_t>(jb * kBB) : 0u;
     int jx = jb % p.xjpb;
     const uint8_t *xg = smem + p.x_off + (jb / p.xjpb) * xbox + g * xrow + 64 * jx;
-    for (int j = jb; ok && t < T && j < je; ++j) {
+    if (ok && t < T)
+#pragma unroll 2
+    for (int j = jb; j < je; ++j) {
       // B fragments of block j for every token group: b[q][2 s + h]
       uint32_t bq[QM][4];
 #pragma unroll
