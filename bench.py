@@ -628,8 +628,8 @@ def run_reference(args):
 # --------------------------------------------------------------------------- traffic from the committed ncu summary
 
 def committed_traffic(kernel_src: str, summary: str):
-    """DRAM bytes per launch recorded in a profiles/ summary, if the kernel source
-    is unchanged since (the summary records the source's sha1)."""
+    """DRAM bytes of one decode step recorded in a profiles/ summary, if the kernel
+    source is unchanged since (the summary records the source's sha1)."""
     try:
         text = open(os.path.join(ROOT, "profiles", summary)).read()
         src = open(os.path.join(ROOT, "decode_gemv_qmm_b200", "csrc", kernel_src), "rb").read()
