@@ -157,48 +157,71 @@ class ClockSampler:
 # --------------------------------------------------------------------------- the decode-step workload
 
 class DecodeStep:
-    """121 Q8_0 weight matrices resident in HBM, their activations and outputs."""
+    """121 Q8_0 weight matrices resident in HBM, their activations and outputs.
 
-    def __init__(self, seed: int, device, keep_host: bool):
+    Default: every matmul reads its own activation vector (N(0,1), one slice of
+    one concatenated buffer) -- the decode-step workload as specified. With
+    chain=True the matmuls read each other's outputs along the model's data
+    flow (synthetic.decode_step_sources: qkv <- previous down, wo <- qkv,
+    gate/up <- wo, down <- up, lm_head <- last down) and the Q8_0 scales are
+    drawn with synthetic.chain_dscale, so 121 chained products stay O(1); only
+    the first input vector comes from the host."""
+
+    def __init__(self, seed: int, device, keep_host: bool, chain: bool = False):
         import torch
 
         self.shapes = syn.decode_step_shapes()
+        self.chain = chain
         self.host_w = [] if keep_host else None
         self.host_x = []
         self.W = []
         xs = []
         for i, (_, n, k) in enumerate(self.shapes):
             g = syn.rng(syn.sub_seed(seed, i))
-            wb, _, _ = syn.q8_0_weights(g, n, k)
-            x = syn.act_f32(g, 1, k)
+            if chain:
+                wb, _, _ = syn.q8_0_weights(g, n, k, dscale=syn.chain_dscale(k))
+            else:
+                wb, _, _ = syn.q8_0_weights(g, n, k)
             self.W.append(torch.from_numpy(wb).to(device))
             if keep_host:
                 self.host_w.append(wb)
-            self.host_x.append(x)
-            xs.append(x.reshape(-1))
+            if not chain or i == 0:
+                x = syn.act_f32(g, 1, k)
+                self.host_x.append(x)
+                xs.append(x.reshape(-1))
         self.x_offsets = np.cumsum([0] + [x.size for x in xs])
         self.y_offsets = np.cumsum([0] + [n for _, n, _ in self.shapes])
         self.host_xcat = torch.from_numpy(np.concatenate(xs)).pin_memory()
         self.X = self.host_xcat.to(device)
         self.Y = torch.zeros(int(self.y_offsets[-1]), dtype=torch.float32, device=device)
         self.host_logits = torch.empty(self.shapes[-1][1], dtype=torch.float32).pin_memory()
+        xp, yp = self.X.data_ptr(), self.Y.data_ptr()
+        self.y_ptrs = [yp + 4 * int(self.y_offsets[i]) for i in range(len(self.shapes))]
+        if chain:
+            src = syn.decode_step_sources()
+            self.sources = src
+            self.x_ptrs = [xp if j < 0 else self.y_ptrs[j] for j in src]
+        else:
+            self.sources = None
+            self.x_ptrs = [xp + 4 * int(self.x_offsets[i]) for i in range(len(self.shapes))]
 
     def launch(self, qmm, stream_handle: int, flags: int):
+        """The 121 matmuls, one qmm_q8_gemv_ex call each."""
         lib = qmm.lib
-        xp, yp = self.X.data_ptr(), self.Y.data_ptr()
         for i, (_, n, k) in enumerate(self.shapes):
-            st = lib.qmm_q8_gemv_ex(1, n, k, 32, self.W[i].data_ptr(), xp + 4 * int(self.x_offsets[i]),
-                                    yp + 4 * int(self.y_offsets[i]), flags, stream_handle)
+            st = lib.qmm_q8_gemv_ex(1, n, k, 32, self.W[i].data_ptr(), self.x_ptrs[i], self.y_ptrs[i], flags,
+                                    stream_handle)
             if st != 0:
                 raise qmm.QmmError(st, "qmm_q8_gemv_ex")
 
     def launch_multi(self, qmm, stream_handle: int, flags: int):
         """The same matmul set with each layer's gate and up projections as one
-        qmm_q8_gemv_multi launch over the gate's activation vector (97 launches)."""
+        qmm_q8_gemv_multi launch over their shared activation vector (97 launches).
+        Without chain=True gate and up have different inputs; the launch then
+        reads the gate's for both (same bytes, same kernels)."""
         import ctypes
 
         lib = qmm.lib
-        xp, yp = self.X.data_ptr(), self.Y.data_ptr()
         i = 0
         while i < len(self.shapes):
             name, n, k = self.shapes[i]
@@ -206,14 +229,14 @@ class DecodeStep:
                 n2 = self.shapes[i + 1][1]
                 N = (ctypes.c_int64 * 2)(n, n2)
                 W = (ctypes.c_void_p * 2)(self.W[i].data_ptr(), self.W[i + 1].data_ptr())
-                Y = (ctypes.c_void_p * 2)(yp + 4 * int(self.y_offsets[i]), yp + 4 * int(self.y_offsets[i + 1]))
-                st = lib.qmm_q8_gemv_multi(1, k, 32, 2, N, W, xp + 4 * int(self.x_offsets[i]), Y, flags, stream_handle)
+                Y = (ctypes.c_void_p * 2)(self.y_ptrs[i], self.y_ptrs[i + 1])
+                st = lib.qmm_q8_gemv_multi(1, k, 32, 2, N, W, self.x_ptrs[i], Y, flags, stream_handle)
                 if st != 0:
                     raise qmm.QmmError(st, "qmm_q8_gemv_multi")
                 i += 2
                 continue
-            st = lib.qmm_q8_gemv_ex(1, n, k, 32, self.W[i].data_ptr(), xp + 4 * int(self.x_offsets[i]),
-                                    yp + 4 * int(self.y_offsets[i]), flags, stream_handle)
+            st = lib.qmm_q8_gemv_ex(1, n, k, 32, self.W[i].data_ptr(), self.x_ptrs[i], self.y_ptrs[i], flags,
+                                    stream_handle)
             if st != 0:
                 raise qmm.QmmError(st, "qmm_q8_gemv_ex")
             i += 1
@@ -223,16 +246,43 @@ class DecodeStep:
         slices fit on chip as fused Q8xQ8 (quantised activations), the rest fp32.
         qx / dx: scratch for the codes and scales (largest K)."""
         lib = qmm.lib
-        xp, yp = self.X.data_ptr(), self.Y.data_ptr()
         for i, (_, n, k) in enumerate(self.shapes):
-            st = lib.qmm_q8_gemv_auto(1, n, k, 32, self.W[i].data_ptr(), xp + 4 * int(self.x_offsets[i]),
-                                      yp + 4 * int(self.y_offsets[i]), qx.data_ptr(), dx.data_ptr(), flags,
-                                      stream_handle)
+            st = lib.qmm_q8_gemv_auto(1, n, k, 32, self.W[i].data_ptr(), self.x_ptrs[i], self.y_ptrs[i],
+                                      qx.data_ptr(), dx.data_ptr(), flags, stream_handle)
             if st != 0:
                 raise qmm.QmmError(st, "qmm_q8_gemv_auto")
 
+    def schedule(self, name: str):
+        """The launch function of a named schedule ("gemv": 121 launches, "multi": 97)."""
+        return {"gemv": self.launch, "multi": self.launch_multi}[name]
+
+    def launches(self, name: str) -> int:
+        return len(self.shapes) if name == "gemv" else len(self.shapes) - QWEN_LAYERS
+
+    def x_of(self, i: int, Y_host=None):
+        """Host copy of matmul i's input vector (from Y_host, the step's outputs, in chain mode)."""
+        k = self.shapes[i][2]
+        if self.chain and self.sources[i] >= 0:
+            j = self.sources[i]
+            return np.asarray(Y_host[int(self.y_offsets[j]):int(self.y_offsets[j]) + k], dtype=np.float32).reshape(1, k)
+        return self.host_x[0 if self.chain else i]
+
     def logits(self):
         return self.Y[int(self.y_offsets[-2]):int(self.y_offsets[-1])]
+
+
+QWEN_LAYERS = syn.QWEN05B_LAYERS
+
+
+def step_graph(qmm, step: DecodeStep, stream, schedule: str, flags: int):
+    """The benchmark's decode step as a CUDA graph: one eager call of the
+    schedule (outside capture), then the same calls captured on `stream`."""
+    import torch
+
+    fn = step.schedule(schedule)
+    fn(qmm, stream.cuda_stream, flags)
+    torch.cuda.synchronize()
+    return capture(lambda h: fn(qmm, h, flags), stream)
 
 
 def capture(fn, stream):
@@ -569,21 +619,30 @@ def oracle_step_sample(step_w, step_x, shapes, frac: float, threads: int):
 
 
 def cpu_baseline(step_w, step_x, shapes, budget_s: float = 10.0):
-    """The oracle timed on the host cores: whole decode steps (or a row fraction of
-    one when a step is slower than the budget), repeated until ~budget_s of work."""
+    """The oracle timed on the host cores: on all of them (the reported value) and
+    on one thread, each on whole decode steps or a row fraction of one when a
+    step is slower than the budget, repeated until ~budget_s of work."""
+    def timed(threads, budget):
+        t_probe = oracle_step_sample(step_w, step_x, shapes, 0.01, threads)
+        full_est = t_probe / 0.01
+        frac = min(1.0, max(0.001, budget / max(full_est, 1e-9)))
+        done = t = 0.0
+        steps = 0
+        while t < budget and steps < 200:
+            t += oracle_step_sample(step_w, step_x, shapes, frac, threads)
+            done += frac
+            steps += 1
+        return done / t, steps, frac, t
+
     threads = os.cpu_count() or 1
-    t_probe = oracle_step_sample(step_w, step_x, shapes, 0.01, threads)
-    full_est = t_probe / 0.01
-    frac = min(1.0, max(0.01, budget_s / max(full_est, 1e-9)))
-    done = t = 0.0
-    steps = 0
-    while t < budget_s and steps < 200:
-        t += oracle_step_sample(step_w, step_x, shapes, frac, threads)
-        done += frac
-        steps += 1
-    return {"value": round(done / t, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{steps} x first {frac:.0%} of the rows of all 121 GEMVs of a decode step (fp64 C oracle, "
-                      f"{threads} threads over row windows), {t:.1f} s; tok/s = steps done / time"}
+    v_all, steps, frac, t = timed(threads, budget_s)
+    v_one, steps1, frac1, t1 = timed(1, budget_s / 2)
+    return {"value": round(v_all, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{steps} x first {frac:.1%} of the rows of all 121 GEMVs of a decode step (fp64 C oracle, "
+                      f"{threads} threads over row windows), {t:.1f} s; tok/s = steps done / time",
+            "single_thread": {"value": round(v_one, 3), "unit": UNIT, "cores": 1,
+                              "sample": f"{steps1} x first {frac1:.1%} of the rows of all 121 GEMVs, one thread, "
+                                        f"{t1:.1f} s"}}
 
 
 def run_reference(args):
@@ -739,6 +798,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None, help="launch one named kernel (see run_case) instead of the benchmark")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--schedule", default="gemv", choices=["gemv", "multi"],
+                    help="decode-step schedule: 121 qmm_q8_gemv_ex launches, or gate+up of each layer in one "
+                         "qmm_q8_gemv_multi launch (97)")
     args = ap.parse_args(argv)
     if args.case:
         return run_case(args.case, args.reps, args.seed)
@@ -768,9 +830,7 @@ def main(argv=None):
     step = DecodeStep(args.seed, device, keep_host=want_cpu)
     stream = torch.cuda.Stream()
     flags = qmm.QMM_FLAG_EARLY_WEIGHTS
-    step.launch(qmm, stream.cuda_stream, flags)  # first call outside capture
-    torch.cuda.synchronize()
-    graph = capture(lambda h: step.launch(qmm, h, flags), stream)
+    graph = step_graph(qmm, step, stream, args.schedule, flags)
 
     def barrier():
         if world > 1:
@@ -823,14 +883,14 @@ def main(argv=None):
 
     wb, xb, yb = step_bytes()
     bytes_step = wb + xb + yb
-    launches = len(step.shapes)
+    launches = step.launches(args.schedule)
     achieved_gbs = bytes_step / (ms_step * 1e6)
     traffic = committed_traffic("q8_gemv.cu", "q8_gemv_decode_step.md")
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved_gbs / pk["hbm_gbs"], 4),
                 "traffic": (round(traffic / launches) if traffic else None),
-                "kernel": "q8_gemv (121 launches per step: fp32 register-resident, tensor-core resident and "
-                          "streaming variants)",
+                "kernel": f"q8_gemv ({launches} launches per step: fp32 register-resident, tensor-core resident "
+                          "and streaming variants)",
                 "per_launch": {"algorithmic_bytes": round(bytes_step / launches),
                                "avg_duration_us": round(ms_step * 1e3 / launches, 3)},
                 "peak_source": pk["source"], "vs_8TBs_spec": round(achieved_gbs / 8000.0, 4)}
@@ -857,8 +917,10 @@ def main(argv=None):
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": {"workload": WORKLOAD, "M": 1, "weight_format": "Q8_0", "bytes_per_step": bytes_step,
                            "l2": "inputs larger than L2 (524,833,792 weight bytes per step; no flush)",
-                           "launch": "CUDA graph of 121 qmm_q8_gemv_ex calls, programmatic dependent launch, "
-                                     "QMM_FLAG_EARLY_WEIGHTS",
+                           "launch": (("CUDA graph of 121 qmm_q8_gemv_ex calls" if args.schedule == "gemv" else
+                                       "CUDA graph of 97 calls: qkv, wo, down, lm_head by qmm_q8_gemv_ex, gate + up "
+                                       "of each layer by one qmm_q8_gemv_multi")
+                                      + ", programmatic dependent launch, QMM_FLAG_EARLY_WEIGHTS"),
                            "parallelism": f"dp{world} (independent decode per rank)"},
                 "GB_s": round(achieved_gbs, 1), "roofline": roofline, "clocks": clocks,
                 "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,

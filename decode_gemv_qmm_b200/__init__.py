@@ -53,6 +53,9 @@ _SIGS = {
     "qmm_q8q8_block_dots": [_i64, _i64, _i64, _int, _p, _p, _p, _p],
     "qmm_q4_gateup_unfused": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p],
     "qmm_prefill_plan": [_int, _i64, _i64, _i64, _int, _p],
+    "qmm_q8q8_gemv_fused_dots": [_i64, _i64, _i64, _int, _p, _p, _p, _p, _p, _p, _p],
+    "qmm_q8q8_block_dots_q8_0": [_i64, _i64, _i64, _int, _p, _p, _p, _p],
+    "qmm_test_withheld_copy": [_int, _i64, _i64, _i64, _int, _p, _p, _p, ctypes.c_uint64, _p],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(lib, _name, None)
@@ -100,9 +103,13 @@ def version() -> str:
 
 
 def device_status() -> int:
-    """Synchronise and read-and-clear the kernels' device status word (0 = clean)."""
+    """Synchronise and read-and-clear the kernels' device status words (0 = clean;
+    the library reports recorded bits as QMM_ERR_DEVICE_CHECK, returned here as
+    the bits themselves)."""
     bits = ctypes.c_uint32(0)
-    _check(lib.qmm_device_status(ctypes.byref(bits)), "qmm_device_status")
+    st = lib.qmm_device_status(ctypes.byref(bits))
+    if st != QMM_ERR_DEVICE_CHECK:
+        _check(st, "qmm_device_status")
     return bits.value
 
 
@@ -214,6 +221,37 @@ def qmm_q8q8_block_dots(W: torch.Tensor, QX: torch.Tensor, N: int, isum: torch.T
     _check(lib.qmm_q8q8_block_dots(M, N, K, block, _ptr(W), _ptr(QX), _ptr(isum), _stream(stream)),
            "qmm_q8q8_block_dots")
     return isum
+
+
+def qmm_q8q8_gemv_fused_dots(W: torch.Tensor, X: torch.Tensor, N: int, *, block: int = BLOCK, stream=None):
+    """(Y, QX, DX, isum): qmm_q8q8_gemv_fused plus its exact int32 block dots isum[M, N, K/32]."""
+    M, K = X.shape
+    Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    QX = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    DX = torch.empty((M, K // BLOCK), dtype=torch.float32, device=X.device)
+    isum = torch.empty((M, N, K // BLOCK), dtype=torch.int32, device=X.device)
+    _check(lib.qmm_q8q8_gemv_fused_dots(M, N, K, block, _ptr(W), _ptr(X), _ptr(QX), _ptr(DX), _ptr(Y), _ptr(isum),
+                                        _stream(stream)), "qmm_q8q8_gemv_fused_dots")
+    return Y, QX, DX, isum
+
+
+def qmm_q8q8_block_dots_q8_0(W: torch.Tensor, XB: torch.Tensor, K: int, N: int, *, block: int = BLOCK,
+                             stream=None) -> torch.Tensor:
+    """isum[M, N, K/32]: the exact block dots of qmm_q8q8_gemv_q8_0."""
+    M = XB.shape[0]
+    isum = torch.empty((M, N, K // BLOCK), dtype=torch.int32, device=XB.device)
+    _check(lib.qmm_q8q8_block_dots_q8_0(M, N, K, block, _ptr(W), _ptr(XB), _ptr(isum), _stream(stream)),
+           "qmm_q8q8_block_dots_q8_0")
+    return isum
+
+
+def qmm_test_withheld_copy(kernel: int, W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor, wait_ns: int, *,
+                           block: int = BLOCK, stream=None) -> None:
+    """Failure-path test launch (kernel 0: streaming Q8_0 GEMV, 1: small-M prefill): one copy of
+    CTA 0 is never issued, so its waits give up after wait_ns; read the result with device_status()."""
+    M, K = X.shape
+    _check(lib.qmm_test_withheld_copy(kernel, M, N, K, block, _ptr(W), _ptr(X), _ptr(Y), wait_ns, _stream(stream)),
+           "qmm_test_withheld_copy")
 
 
 def qmm_q4_gemv(W: torch.Tensor, X: torch.Tensor, N: int, Y: torch.Tensor | None = None, *,

@@ -1,5 +1,7 @@
-// prefill.cu -- many-token matmul Y = X . W^T on the tcgen05 tensor cores, with
-// W in Q8_0 or Q4_0 blocks decoded to bf16 in shared memory.
+// prefill.cu -- many-token matmul Y = X . W^T on Q8_0 or Q4_0 blocks: above 32
+// tokens on the tcgen05 tensor cores, each block decoded to bf16 and written
+// into tensor memory as the A operand; up to 32 tokens by a small-M mma.sync
+// kernel on the exact integer codes held in shared memory.
 //
 // Operation ("LSE v0.4.16", section "Retained optimizations and
 // compatibility": the M1024 prefill panels): Y[m][n] = sum_k X[m][k] W[n][k]
@@ -619,6 +621,10 @@ struct alignas(64) SParams {
   int xjpb;          // K blocks per X row in shared memory (a box of them per 8 QM tokens)
   int w_off, x_off, part_off;
   int prefetch_before_wait;
+  // failure-path test only (defaults: kWaitLimitNs, 0): the limit of the
+  // consumers' waits, and whether CTA 0 withholds its whole weight copy
+  uint64_t wait_ns;
+  int withhold;
 };
 
 // Not volatile: a pure function of its operands, so the compiler may overlap
@@ -728,10 +734,14 @@ __global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(c
   const int nb = kb1 - kb0;
   const uint32_t sbase = smem_u32(smem);
 
+  // abort flag (shared word after the two barriers): set when copies may still
+  // be landing in W / X on an error path
+  const uint32_t abort_sa = smem_u32(smem) + 16u;
   pdl_launch_dependents();
   if (tid == 0) {
     mbar_init(wbar, 1);
     mbar_init(xbar, 1);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(abort_sa), "r"(0u) : "memory");
     fence_mbar_init();
   }
   // without split K, token rows M .. 8 QM - 1 of X are not copied: zero
@@ -761,6 +771,7 @@ __global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(c
     };
     const int nseg = split == 1 ? (R > 0 ? 1 : 0) : R;
     auto issue_w = [&]() {
+      if (p.withhold && blockIdx.x == 0) return;  // failure-path test: W never lands in this CTA
       if (p.w_tma) {  // every row segment of the group in one box (rows past N read as zero)
         if (lane == 0 && R > 0) {
           mbar_arrive_expect_tx(wbar, static_cast<uint32_t>(p.seg_pitch * ((p.N + p.groups - 1) / p.groups)));
@@ -827,15 +838,20 @@ __global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(c
     for (int q = 0; q < QM; ++q)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[q][i] = 0.f;
-    bool ok = mbar_wait(wbar, 0);
-    ok = mbar_wait(xbar, 0) && ok;
+    bool ok = mbar_wait(wbar, 0, p.wait_ns);
+    ok = mbar_wait(xbar, 0, p.wait_ns) && ok;
     ok = __all_sync(0xffffffffu, ok);  // the mma.sync loop below needs the whole warp
     if (!ok) {
       // record, then wait once more for copies still in flight before the
       // buffers are reused and the CTA exits
       if (lane == 0) atomicOr(&g_prefill_status, kDevTimeoutFull);
-      if (!mbar_wait(wbar, 0) || !mbar_wait(xbar, 0))
-        if (lane == 0) atomicOr(&g_prefill_status, kDevTimeoutDrain);
+      const bool drained = mbar_wait(wbar, 0, p.wait_ns) && mbar_wait(xbar, 0, p.wait_ns);
+      if (!__all_sync(0xffffffffu, drained) && lane == 0) {
+        // a copy may still be writing W / X, whose space the reduction below
+        // reuses: this CTA then stores no partial sums and no output
+        atomicOr(&g_prefill_status, kDevTimeoutDrain);
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(abort_sa), "r"(1u) : "memory");
+      }
     }
     const int T = (R + 15) / 16;
     const uint8_t *wbase = smem + p.w_off;
@@ -847,70 +863,74 @@ __global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(c
     uint32_t bb = vb ? small_row_base(p, r0, kb0, kBB, 16 * t + g + 8) + static_cast<uint32_t>(jb * kBB) : 0u;
     int jx = jb % p.xjpb;
     const uint8_t *xg = smem + p.x_off + (jb / p.xjpb) * xbox + g * xrow + 64 * jx;
-    if (ok && t < T)
+    if (ok && t < T) {
 #pragma unroll 2
-    for (int j = jb; j < je; ++j) {
-      // B fragments of block j for every token group: b[q][2 s + h]
-      uint32_t bq[QM][4];
+      for (int j = jb; j < je; ++j) {
+        // B fragments of block j for every token group: b[q][2 s + h]
+        uint32_t bq[QM][4];
 #pragma unroll
-      for (int q = 0; q < QM; ++q) {
-        const uint8_t *xr = xg + 8 * q * xrow;
-        if constexpr (WT == QMM_Q8_0) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(xr + 16 * qd);  // elements 8qd .. 8qd + 7
-          bq[q][0] = v.x;
-          bq[q][1] = v.y;
-          bq[q][2] = v.z;
-          bq[q][3] = v.w;
-        } else {
-          // elements 4qd .. 4qd + 3 and 16 + 4qd .. 16 + 4qd + 3
-          const uint2 lo = *reinterpret_cast<const uint2 *>(xr + 8 * qd);
-          const uint2 hi = *reinterpret_cast<const uint2 *>(xr + 32 + 8 * qd);
-          bq[q][0] = __byte_perm(lo.x, lo.y, 0x5410u);
-          bq[q][1] = __byte_perm(lo.x, lo.y, 0x7632u);
-          bq[q][2] = __byte_perm(hi.x, hi.y, 0x5410u);
-          bq[q][3] = __byte_perm(hi.x, hi.y, 0x7632u);
+        for (int q = 0; q < QM; ++q) {
+          const uint8_t *xr = xg + 8 * q * xrow;
+          if constexpr (WT == QMM_Q8_0) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(xr + 16 * qd);  // elements 8qd .. 8qd + 7
+            bq[q][0] = v.x;
+            bq[q][1] = v.y;
+            bq[q][2] = v.z;
+            bq[q][3] = v.w;
+          } else {
+            // elements 4qd .. 4qd + 3 and 16 + 4qd .. 16 + 4qd + 3
+            const uint2 lo = *reinterpret_cast<const uint2 *>(xr + 8 * qd);
+            const uint2 hi = *reinterpret_cast<const uint2 *>(xr + 32 + 8 * qd);
+            bq[q][0] = __byte_perm(lo.x, lo.y, 0x5410u);
+            bq[q][1] = __byte_perm(lo.x, lo.y, 0x7632u);
+            bq[q][2] = __byte_perm(hi.x, hi.y, 0x5410u);
+            bq[q][3] = __byte_perm(hi.x, hi.y, 0x7632u);
+          }
         }
-      }
-      uint32_t oa[4], ob[4];
-      float da, db;
-      small_row<WT>(wbase, ba, va, qd, oa, da);
-      small_row<WT>(wbase, bb, vb, qd, ob, db);
-      ba += kBB;
-      bb += kBB;
-      xg += 64;
-      if (++jx == p.xjpb) {  // next box
-        jx = 0;
-        xg += xbox - 64 * p.xjpb;
-      }
-      const uint32_t a0[4] = {oa[0], ob[0], oa[1], ob[1]};  // k step 0
-      const uint32_t a1[4] = {oa[2], ob[2], oa[3], ob[3]};  // k step 1
+        uint32_t oa[4], ob[4];
+        float da, db;
+        small_row<WT>(wbase, ba, va, qd, oa, da);
+        small_row<WT>(wbase, bb, vb, qd, ob, db);
+        ba += kBB;
+        bb += kBB;
+        xg += 64;
+        if (++jx == p.xjpb) {  // next box
+          jx = 0;
+          xg += xbox - 64 * p.xjpb;
+        }
+        const uint32_t a0[4] = {oa[0], ob[0], oa[1], ob[1]};  // k step 0
+        const uint32_t a1[4] = {oa[2], ob[2], oa[3], ob[3]};  // k step 1
 #pragma unroll
-      for (int q = 0; q < QM; ++q) {
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_bf16_16816(c, a0, bq[q][0], bq[q][1]);
-        mma_bf16_16816(c, a1, bq[q][2], bq[q][3]);
-        acc[q][0] = __fmaf_rn(da, c[0], acc[q][0]);
-        acc[q][1] = __fmaf_rn(da, c[1], acc[q][1]);
-        acc[q][2] = __fmaf_rn(db, c[2], acc[q][2]);
-        acc[q][3] = __fmaf_rn(db, c[3], acc[q][3]);
+        for (int q = 0; q < QM; ++q) {
+          float c[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_bf16_16816(c, a0, bq[q][0], bq[q][1]);
+          mma_bf16_16816(c, a1, bq[q][2], bq[q][3]);
+          acc[q][0] = __fmaf_rn(da, c[0], acc[q][0]);
+          acc[q][1] = __fmaf_rn(da, c[1], acc[q][1]);
+          acc[q][2] = __fmaf_rn(db, c[2], acc[q][2]);
+          acc[q][3] = __fmaf_rn(db, c[3], acc[q][3]);
+        }
       }
     }
     // every consumer is past its last read of W and X: their space takes the
     // warps' sums red[warp][group][lane] (float4)
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kSmWarps) : "memory");
+    const bool aborted = lds_u32(abort_sa) != 0u;  // uniform: read after the barrier
     const uint32_t red = sbase + static_cast<uint32_t>(p.w_off);
+    if (!aborted) {
 #pragma unroll
-    for (int q = 0; q < QM; ++q)
-      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
-                       red + static_cast<uint32_t>(((cw * QM + q) * 32 + lane) * 16)),
-                   "f"(acc[q][0]), "f"(acc[q][1]), "f"(acc[q][2]), "f"(acc[q][3])
-                   : "memory");
+      for (int q = 0; q < QM; ++q)
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         red + static_cast<uint32_t>(((cw * QM + q) * 32 + lane) * 16)),
+                     "f"(acc[q][0]), "f"(acc[q][1]), "f"(acc[q][2]), "f"(acc[q][3])
+                     : "memory");
+    }
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kSmWarps) : "memory");
     // (r, m): the K ranges' sums in order; kept in part[r][m] without split K,
     // else stored into the owner rank's slot recv[source rank][row of the owner][m]
     const int ctid = tid - 32;
     const int rpr = (R + split - 1) / split;  // rows per rank share (at most)
-    for (int o = ctid; o < R * kCols; o += 32 * kSmWarps) {
+    for (int o = aborted ? R * kCols : ctid; o < R * kCols; o += 32 * kSmWarps) {
       const int r = o / kCols, m = o % kCols;
       const int tt = r >> 4, rr = r & 15, q = m >> 3, mm = m & 7;
       const int ln = (rr & 7) * 4 + (mm >> 1), i = (rr >> 3) * 2 + (mm & 1);
@@ -937,8 +957,9 @@ __global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(c
   // ------------------------------------------------------------ output
   __syncthreads();
   pdl_wait();  // (Y is written only after the preceding grid; a no-op by now)
+  const bool aborted = lds_u32(abort_sa) != 0u;
   if (split == 1) {
-    for (int o = tid; o < R * p.M; o += blockDim.x) {
+    for (int o = aborted ? R * p.M : tid; o < R * p.M; o += blockDim.x) {
       const int m = o / R, r = o % R;
       p.Y[static_cast<int64_t>(m) * p.N + r0 + r] =
           lds_f32(sbase + static_cast<uint32_t>(p.part_off + 4 * (r * (kCols + 1) + m)));
@@ -948,7 +969,7 @@ __global__ void __launch_bounds__((kSmWarps + 1) * 32, 1) prefill_small_kernel(c
     const int rpr = (R + split - 1) / split;
     const int rb = zr * rpr, re = min(R, rb + rpr);  // this rank's rows of the group
     const uint32_t pa = sbase + static_cast<uint32_t>(p.part_off);
-    for (int o = tid; o < (re - rb) * p.M; o += blockDim.x) {
+    for (int o = aborted ? (re - rb) * p.M : tid; o < (re - rb) * p.M; o += blockDim.x) {
       const int m = o / (re - rb), lr = o % (re - rb);
       float v = 0.f;
       for (int src = 0; src < split; ++src)
@@ -969,15 +990,16 @@ void *small_kernel_ptr() {
 // into a CTA (its W share plus its X slice). False when M is too large or no
 // split fits (the tcgen05 path takes over).
 bool try_launch_small(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W, const uint16_t *X,
-                      float *Y, cudaStream_t stream, uint32_t flags, PrefillPlan *plan, qmm_status *out) {
+                      float *Y, cudaStream_t stream, uint32_t flags, PrefillPlan *plan, qmm_status *out,
+                      uint64_t wait_ns = kWaitLimitNs, int withhold = 0) {
   if (M > kSmMaxM) return false;
   const int KB = K / 32, bb = wtype == QMM_Q8_0 ? 34 : 18;
   const int QM = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
   void *kerns[2][3] = {{small_kernel_ptr<QMM_Q8_0, 1>(), small_kernel_ptr<QMM_Q8_0, 2>(), small_kernel_ptr<QMM_Q8_0, 4>()},
                        {small_kernel_ptr<QMM_Q4_0, 1>(), small_kernel_ptr<QMM_Q4_0, 2>(), small_kernel_ptr<QMM_Q4_0, 4>()}};
   void *kern = kerns[wtype][QM == 1 ? 0 : (QM == 2 ? 1 : 2)];
-  static bool configured[2][64] = {};
-  if (dev.device >= 0 && dev.device < 64 && !configured[wtype][dev.device]) {
+  static DeviceFlags configured[2];
+  if (!configured[wtype].done(dev.device)) {
     for (int i = 0; i < 3; ++i) {
       cudaError_t e = cudaFuncSetAttribute(kerns[wtype][i], cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
       if (e != cudaSuccess) {
@@ -985,7 +1007,7 @@ bool try_launch_small(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K
         return true;
       }
     }
-    configured[wtype][dev.device] = true;
+    configured[wtype].set(dev.device);
   }
 
   struct Layout {
@@ -1117,6 +1139,8 @@ bool try_launch_small(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K
   p.x_off = best.x_off;
   p.part_off = best.part_off;
   p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
+  p.wait_ns = wait_ns;
+  p.withhold = withhold;
   cfg.gridDim = dim3(static_cast<unsigned>(best.groups * best.split));
   cfg.dynamicSmemBytes = best.smem;
   attr[1].val.clusterDim.x = static_cast<unsigned>(best.split);
@@ -1129,6 +1153,14 @@ bool try_launch_small(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K
 }
 
 }  // namespace
+
+qmm_status launch_prefill_small_withheld(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,
+                                         const uint16_t *X, float *Y, uint64_t wait_ns, cudaStream_t stream) {
+  qmm_status st = QMM_OK;
+  if (try_launch_small(dev, wtype, M, N, K, W, X, Y, stream, kLaunchPdl, nullptr, &st, wait_ns, 1)) return st;
+  return set_error(QMM_ERR_SHAPE, "prefill: M=%lld N=%lld K=%d does not take the small-M kernel", (long long)M,
+                   (long long)N, K);
+}
 
 qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,
                           const uint16_t *X, float *Y, cudaStream_t stream, uint32_t flags, PrefillPlan *plan) {
@@ -1169,13 +1201,13 @@ qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, i
 
   void *kerns[2][2] = {{kernel_ptr<QMM_Q8_0, false>(), kernel_ptr<QMM_Q8_0, true>()},
                        {kernel_ptr<QMM_Q4_0, false>(), kernel_ptr<QMM_Q4_0, true>()}};
-  static bool configured[2][64] = {};
-  if (dev.device >= 0 && dev.device < 64 && !configured[wtype][dev.device]) {
+  static DeviceFlags configured[2];
+  if (!configured[wtype].done(dev.device)) {
     for (int w = 0; w < 2; ++w) {
       cudaError_t e = cudaFuncSetAttribute(kerns[wtype][w], cudaFuncAttributeMaxDynamicSharedMemorySize, dev.smem_optin);
       if (e != cudaSuccess) return cuda_check(e, "prefill attribute");
     }
-    configured[wtype][dev.device] = true;
+    configured[wtype].set(dev.device);
   }
   void *kern = kerns[wtype][0];  // split-K occupancy queries: narrow tiles
 

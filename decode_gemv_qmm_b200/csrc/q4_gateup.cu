@@ -455,14 +455,14 @@ __global__ void silu_mul_kernel(const float *__restrict__ G, const float *__rest
 
 template <bool DIRECT, int NMAT>
 cudaError_t launch(const cudaLaunchConfig_t &cfg, const Params &p) {
-  static bool configured[64] = {};
+  static DeviceFlags configured;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  if (!configured.done(dev)) {
     cudaError_t e = cudaFuncSetAttribute(q4_gateup_kernel<DIRECT, NMAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kBarBytes + kStages * kStageBytes + 1024);
     if (e != cudaSuccess) return e;
-    configured[dev] = true;
+    configured.set(dev);
   }
   return cudaLaunchKernelEx(&cfg, q4_gateup_kernel<DIRECT, NMAT>, p);
 }

@@ -100,6 +100,10 @@ struct alignas(64) Params {
   int cs;  // column slots (consumer warps side by side along K)
   int rs;  // row slots (consumer warps side by side along N)
   int prefetch_before_wait;
+  // failure-path test only (defaults: kWaitLimitNs, 0): the limit of every
+  // barrier wait, and whether CTA 0 withholds the copy of its first weight stage
+  uint64_t wait_ns;
+  int withhold;
 };
 
 // Convert four int8 codes (one 32-bit word) and multiply-accumulate them
@@ -271,6 +275,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
         a1 = lim;
       }
       const uint32_t bytes = static_cast<uint32_t>(a1 - a0);
+      if (p.withhold && blockIdx.x == 0 && c == 0) return;  // failure-path test: stage 0 never fills
       mbar_arrive_expect_tx(&full[s], bytes);
       if (bytes) bulk_g2s(dst, p.W + a0, bytes, &full[s], policy);
     };
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
     int issued = prologue;
     for (int c = 0; c < nchunks && ok; ++c) {
       // chunk c is released once every consumer warp arrived on empty[c % S]
-      ok = mbar_wait(&empty[c % S], static_cast<uint32_t>(c / S) & 1u);
+      ok = mbar_wait(&empty[c % S], static_cast<uint32_t>(c / S) & 1u, p.wait_ns);
       if (!ok) break;
       __syncwarp();
       finish(c);
@@ -334,7 +339,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
     if (!ok && lane == 0) {  // error path: record, then drain copies still in flight
       atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
       for (int c = max(0, issued - S); c < issued; ++c)
-        if (!mbar_wait(&full[c % S], static_cast<uint32_t>(c / S) & 1u))
+        if (!mbar_wait(&full[c % S], static_cast<uint32_t>(c / S) & 1u, p.wait_ns))
           atomicOr(&g_q8_gemv_status, kDevTimeoutDrain);
     }
     return;
@@ -350,7 +355,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
   // shared-memory phase (consecutive c) read eight different bank groups.
   const bool xs = p.xs_off != 0;
   const uint32_t xs_sa = smem_u32(smem) + p.xs_off;
-  if (xs && !mbar_wait(xbar, 0)) {
+  if (xs && !mbar_wait(xbar, 0, p.wait_ns)) {
     if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
     return;
   }
@@ -379,7 +384,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
           for (int j = 0; j < 16; ++j) x2[m][j] = make_float2(0.f, 0.f);
         }
       } else {
-        if (valid && MODE == kModeQ8 && p.XB) {
+        if (valid && p.XB) {
           // a Q8_0 activation block: the fp16 scale, then the 32 codes as 16
           // half-words (2-byte aligned: exactly the block's 34 bytes are read)
           const uint16_t *bp =
@@ -414,7 +419,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32) q8_gemv_kernel(c
 
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % S;
-    if (!mbar_wait(&full[s], static_cast<uint32_t>(c / S) & 1u)) {
+    if (!mbar_wait(&full[s], static_cast<uint32_t>(c / S) & 1u, p.wait_ns)) {
       if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
       return;  // the producer times out on this warp's missing arrival and drains
     }
@@ -513,6 +518,7 @@ struct alignas(64) RParams {
   int qx_off, dx_off;
   int8_t *QXo;
   float *DXo;
+  int32_t *isum;  // fused Q8xQ8, dump instance only: the exact block dots, N x K/32
 };
 
 template <int U>
@@ -700,7 +706,9 @@ q8_gemv_resident_kernel(const __grid_constant__ RParams p) {
 // over |x| bit patterns, then q8_act_scale / q8_act_code. CTA 0 also writes the
 // codes and scales to QX / DX.
 
-template <int U>
+// DOTS: the test instance, which also writes every exact block dot to p.isum
+// (the arithmetic is the same code).
+template <int U, bool DOTS>
 __global__ void __launch_bounds__(512, 1) q8q8_resident_kernel(const __grid_constant__ RParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -843,6 +851,10 @@ __global__ void __launch_bounds__(512, 1) q8q8_resident_kernel(const __grid_cons
       s1 = __dp4a(static_cast<int>(wc[u][i + 1]), static_cast<int>(qa[i + 1]), s1);
     }
     part[u] = (wd[u] * dxv) * static_cast<float>(s0 + s1);  // |isum| <= 2^19: exact in fp32
+    if constexpr (DOTS) {
+      const int rl = k + u * p.wpw;
+      if (ok && act && rl < rows) p.isum[(r_begin + rl) * p.KB + col] = s0 + s1;
+    }
   }
   if (!ok && tid == 0) {  // error path: give copies still in flight a bounded chance to land
     if (!mbar_wait(wbar, 0) || !mbar_wait(xbar, 0)) atomicOr(&g_q8_gemv_status, kDevTimeoutDrain);
@@ -1421,15 +1433,15 @@ int align_up(int64_t v, int a) { return static_cast<int>((v + a - 1) / a * a); }
 
 template <int MODE, int MP, int RG>
 cudaError_t launch(const cudaLaunchConfig_t &cfg, const Params &p) {
-  static bool configured[64] = {};
+  static DeviceFlags configured;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  if (!configured.done(dev)) {
     int optin = 0;
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     cudaError_t e = cudaFuncSetAttribute(q8_gemv_kernel<MODE, MP, RG>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e != cudaSuccess) return e;
-    configured[dev] = true;
+    configured.set(dev);
   }
   return cudaLaunchKernelEx(&cfg, q8_gemv_kernel<MODE, MP, RG>, p);
 }
@@ -1441,8 +1453,10 @@ namespace {
 template <int MODE>
 qmm_status launch_stream(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, const int8_t *QX,
                          const float *DX, float *Y, int32_t *isum, cudaStream_t stream, uint32_t flags,
-                         const uint8_t *XB = nullptr) {
+                         const uint8_t *XB = nullptr, uint64_t wait_ns = kWaitLimitNs, int withhold = 0) {
   Params p{};
+  p.wait_ns = wait_ns;
+  p.withhold = withhold;
   p.W = static_cast<const uint8_t *>(W);
   p.X = X;
   p.QX = QX;
@@ -1586,14 +1600,14 @@ bool try_launch_resident(const DevInfo &dev, int64_t N, int K, const void *W, co
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   auto go = [&](auto kern) -> cudaError_t {
-    static bool configured[3][64] = {};
+    static DeviceFlags configured[3];
     int dev_id = 0;
     cudaGetDevice(&dev_id);
     const int idx = U == 1 ? 0 : U == 2 ? 1 : 2;
-    if (dev_id >= 0 && dev_id < 64 && !configured[idx][dev_id]) {
+    if (!configured[idx].done(dev_id)) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
       if (e != cudaSuccess) return e;
-      configured[idx][dev_id] = true;
+      configured[idx].set(dev_id);
     }
     return cudaLaunchKernelEx(&cfg, kern, p);
   };
@@ -1607,7 +1621,8 @@ bool try_launch_resident(const DevInfo &dev, int64_t N, int K, const void *W, co
 // CTA are capped so that two CTAs' registers fit one SM (the next launch in the
 // stream can then start, and prefetch its weights, while this one runs).
 bool try_launch_q8q8_resident(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, int8_t *QX,
-                              float *DX, float *Y, cudaStream_t stream, uint32_t flags, qmm_status *out) {
+                              float *DX, float *Y, cudaStream_t stream, uint32_t flags, qmm_status *out,
+                              int32_t *isum = nullptr) {
   constexpr int64_t kMaxSlice = 96 * 1024;
   const int KB = K / 32;
   const int cg = (KB + 31) / 32;
@@ -1646,6 +1661,7 @@ bool try_launch_q8q8_resident(const DevInfo &dev, int64_t N, int K, const void *
   p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
   p.QXo = QX;
   p.DXo = DX;
+  p.isum = isum;
   p.xs_off = 1024;
   p.qx_off = align_up(p.xs_off + KB * 128, 128);
   p.dx_off = align_up(p.qx_off + KB * 32, 128);
@@ -1674,19 +1690,24 @@ bool try_launch_q8q8_resident(const DevInfo &dev, int64_t N, int K, const void *
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   auto go = [&](auto kern) -> cudaError_t {
-    static bool configured[3][64] = {};
+    static DeviceFlags configured[2][3];
     int dev_id = 0;
     cudaGetDevice(&dev_id);
     const int idx = U == 1 ? 0 : U == 2 ? 1 : 2;
-    if (dev_id >= 0 && dev_id < 64 && !configured[idx][dev_id]) {
+    if (!configured[isum != nullptr][idx].done(dev_id)) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemAttr));
       if (e != cudaSuccess) return e;
-      configured[idx][dev_id] = true;
+      configured[isum != nullptr][idx].set(dev_id);
     }
     return cudaLaunchKernelEx(&cfg, kern, p);
   };
-  cudaError_t e = U == 1 ? go(q8q8_resident_kernel<1>) : U == 2 ? go(q8q8_resident_kernel<2>)
-                                                                : go(q8q8_resident_kernel<4>);
+  cudaError_t e;
+  if (isum)
+    e = U == 1 ? go(q8q8_resident_kernel<1, true>) : U == 2 ? go(q8q8_resident_kernel<2, true>)
+                                                            : go(q8q8_resident_kernel<4, true>);
+  else
+    e = U == 1 ? go(q8q8_resident_kernel<1, false>) : U == 2 ? go(q8q8_resident_kernel<2, false>)
+                                                             : go(q8q8_resident_kernel<4, false>);
   *out = cuda_check(e, "q8q8_gemv_fused launch");
   return true;
 }
@@ -1758,16 +1779,16 @@ bool try_launch_mma(const DevInfo &dev, int64_t N, int K, const void *W, const f
   attr[0].val.programmaticStreamSerializationAllowed = (flags & kLaunchPdl) ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  static bool configured[kInsts][64] = {};
+  static DeviceFlags configured[kInsts];
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  if (dev_id >= 0 && dev_id < 64 && !configured[pick][dev_id]) {
+  if (!configured[pick].done(dev_id)) {
     cudaError_t e = cudaFuncSetAttribute(in.kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
     if (e != cudaSuccess) {
       *out = cuda_check(e, "q8_gemv attribute");
       return true;
     }
-    configured[pick][dev_id] = true;
+    configured[pick].set(dev_id);
   }
   *out = cuda_check(cudaLaunchKernelEx(&cfg, in.kern, p), "q8_gemv launch");
   return true;
@@ -1830,16 +1851,16 @@ bool try_launch_digits(const DevInfo &dev, int nproj, const int64_t *N, const vo
   const bool multi = nproj > 1;
   void (*kern)(DParams) = tps == 2 ? (multi ? q8_gemv_digits_kernel<2, true> : q8_gemv_digits_kernel<2, false>)
                                    : (multi ? q8_gemv_digits_kernel<1, true> : q8_gemv_digits_kernel<1, false>);
-  static bool configured[2][2][64] = {};
+  static DeviceFlags configured[2][2];
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  if (dev_id >= 0 && dev_id < 64 && !configured[tps - 1][multi][dev_id]) {
+  if (!configured[tps - 1][multi].done(dev_id)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBudget);
     if (e != cudaSuccess) {
       *out = cuda_check(e, "q8_gemv attribute");
       return true;
     }
-    configured[tps - 1][multi][dev_id] = true;
+    configured[tps - 1][multi].set(dev_id);
   }
   *out = cuda_check(cudaLaunchKernelEx(&cfg, kern, p), "q8_gemv launch");
   return true;
@@ -1912,8 +1933,26 @@ qmm_status launch_q8q8_gemv_q8_0(const DevInfo &dev, int M, int64_t N, int K, co
 }
 
 qmm_status launch_q8q8_block_dots(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,
-                                  int32_t *isum, cudaStream_t stream) {
+                                  const uint8_t *XB, int32_t *isum, cudaStream_t stream) {
+  return launch_stream<kModeQ8Dots>(dev, M, N, K, W, nullptr, QX, nullptr, nullptr, isum, stream, kLaunchPdl, XB);
+}
+
+qmm_status launch_q8q8_gemv_fused_dots(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
+                                       int8_t *QX, float *DX, float *Y, int32_t *isum, cudaStream_t stream) {
+  qmm_status st;
+  // the kernel choice of launch_q8q8_gemv_fused; its resident kernel in the dump instance
+  if (M == 1 && try_launch_q8q8_resident(dev, N, K, W, X, QX, DX, Y, stream, kLaunchPdl, &st, isum)) return st;
+  st = launch_quantize_act_q8(dev, M, K, X, QX, DX, stream, kLaunchPdl);
+  if (st != QMM_OK) return st;
+  st = launch_stream<kModeQ8>(dev, M, N, K, W, nullptr, QX, DX, Y, nullptr, stream, kLaunchPdl);
+  if (st != QMM_OK) return st;
   return launch_stream<kModeQ8Dots>(dev, M, N, K, W, nullptr, QX, nullptr, nullptr, isum, stream, kLaunchPdl);
+}
+
+qmm_status launch_q8_gemv_withheld(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
+                                   float *Y, uint64_t wait_ns, cudaStream_t stream) {
+  return launch_stream<kModeF32>(dev, M, N, K, W, X, nullptr, nullptr, Y, nullptr, stream, kLaunchPdl, nullptr,
+                                 wait_ns, 1);
 }
 
 cudaError_t q8_gemv_status(uint32_t *bits) {

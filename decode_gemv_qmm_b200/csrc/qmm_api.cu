@@ -243,7 +243,7 @@ static qmm_status q8q8_impl(int64_t M, int64_t N, int64_t K, int block, const vo
   QMM_TRY(current_device(&dev));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (K == 0) return isum ? QMM_OK : zero_fill(Y, M * N, s);
-  if (isum) return launch_q8q8_block_dots(dev, static_cast<int>(M), N, static_cast<int>(K), W, QX, isum, s);
+  if (isum) return launch_q8q8_block_dots(dev, static_cast<int>(M), N, static_cast<int>(K), W, QX, nullptr, isum, s);
   uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
   return launch_q8q8_gemv(dev, static_cast<int>(M), N, static_cast<int>(K), W, QX, DX, Y, s, flags);
 }
@@ -267,6 +267,61 @@ static qmm_status q8q8_fused_impl(int64_t M, int64_t N, int64_t K, int block, co
   if (K == 0) return zero_fill(Y, M * N, s);
   uint32_t flags = kLaunchPdl | ((user_flags & QMM_FLAG_EARLY_WEIGHTS) ? kPrefetchBeforeWait : 0u);
   return launch_q8q8_gemv_fused(dev, static_cast<int>(M), N, static_cast<int>(K), W, X, QX, DX, Y, s, flags);
+}
+
+static qmm_status fused_dots_impl(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X,
+                                  int8_t *QX, float *DX, float *Y, int32_t *isum, qmm_stream_t stream) {
+  const char *fn = "qmm_q8q8_gemv_fused_dots";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, N, K, block, QMM_MAX_DECODE_M));
+  if (M == 0 || N == 0 || K == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "W", W, true, 16));
+  QMM_TRY(check_ptr(fn, "X", X, true, 16));
+  QMM_TRY(check_ptr(fn, "QX", QX, true, 16));
+  QMM_TRY(check_ptr(fn, "DX", DX, true, 4));
+  QMM_TRY(check_ptr(fn, "Y", Y, true, 4));
+  QMM_TRY(check_ptr(fn, "isum", isum, true, 4));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  return launch_q8q8_gemv_fused_dots(dev, static_cast<int>(M), N, static_cast<int>(K), W, X, QX, DX, Y, isum,
+                                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+static qmm_status dots_q8_0_impl(int64_t M, int64_t N, int64_t K, int block, const void *W, const void *XB,
+                                 int32_t *isum, qmm_stream_t stream) {
+  const char *fn = "qmm_q8q8_block_dots_q8_0";
+  t_last_error.clear();
+  QMM_TRY(check_shape(fn, M, N, K, block, QMM_MAX_DECODE_M));
+  if (M == 0 || N == 0 || K == 0) return QMM_OK;
+  QMM_TRY(check_ptr(fn, "W", W, true, 16));
+  QMM_TRY(check_ptr(fn, "XB", XB, true, 16));
+  QMM_TRY(check_ptr(fn, "isum", isum, true, 4));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  return launch_q8q8_block_dots(dev, static_cast<int>(M), N, static_cast<int>(K), W, nullptr,
+                                static_cast<const uint8_t *>(XB), isum, reinterpret_cast<cudaStream_t>(stream));
+}
+
+static qmm_status withheld_impl(int kernel, int64_t M, int64_t N, int64_t K, int block, const void *W, const void *X,
+                                float *Y, uint64_t wait_ns, qmm_stream_t stream) {
+  const char *fn = "qmm_test_withheld_copy";
+  t_last_error.clear();
+  if (kernel != 0 && kernel != 1) return set_error(QMM_ERR_SHAPE, "%s: kernel=%d, expected 0 or 1", fn, kernel);
+  QMM_TRY(check_shape(fn, M, N, K, block, kernel == 0 ? QMM_MAX_DECODE_M : 32));
+  if (M < 1 || N < 1 || K < 32) return set_error(QMM_ERR_SHAPE, "%s: M, N must be >= 1 and K >= 32", fn);
+  if (wait_ns < 1000 || wait_ns > 2000000000ull)
+    return set_error(QMM_ERR_SHAPE, "%s: wait_ns=%llu outside 1e3 .. 2e9", fn, (unsigned long long)wait_ns);
+  QMM_TRY(check_ptr(fn, "W", W, true, 16));
+  QMM_TRY(check_ptr(fn, "X", X, true, 16));
+  QMM_TRY(check_ptr(fn, "Y", Y, true, 4));
+  DevInfo dev;
+  QMM_TRY(current_device(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (kernel == 0)
+    return launch_q8_gemv_withheld(dev, static_cast<int>(M), N, static_cast<int>(K), W, static_cast<const float *>(X), Y,
+                                   wait_ns, s);
+  return launch_prefill_small_withheld(dev, QMM_Q8_0, M, N, static_cast<int>(K), W, static_cast<const uint16_t *>(X), Y,
+                                       wait_ns, s);
 }
 
 static qmm_status q4_gemv_impl(int64_t M, int64_t N, int64_t K, int block, const void *W, const float *X, float *Y,
@@ -404,6 +459,22 @@ QMM_API qmm_status qmm_q8q8_block_dots(int64_t M, int64_t N, int64_t K, int bloc
   return q8q8_impl(M, N, K, block, W, QX, nullptr, nullptr, isum, stream, 0u);
 }
 
+QMM_API qmm_status qmm_q8q8_gemv_fused_dots(int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                            const float *X, int8_t *QX, float *DX, float *Y, int32_t *isum,
+                                            qmm_stream_t stream) {
+  return fused_dots_impl(M, N, K, block, W, X, QX, DX, Y, isum, stream);
+}
+
+QMM_API qmm_status qmm_q8q8_block_dots_q8_0(int64_t M, int64_t N, int64_t K, int block, const void *W, const void *XB,
+                                            int32_t *isum, qmm_stream_t stream) {
+  return dots_q8_0_impl(M, N, K, block, W, XB, isum, stream);
+}
+
+QMM_API qmm_status qmm_test_withheld_copy(int kernel, int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                          const void *X, float *Y, uint64_t wait_ns, qmm_stream_t stream) {
+  return withheld_impl(kernel, M, N, K, block, W, X, Y, wait_ns, stream);
+}
+
 QMM_API qmm_status qmm_q4_swiglu_gateup(int64_t M, int64_t N, int64_t K, int block, const void *Wg, const void *Wu,
                                         const float *X, float *Y, qmm_stream_t stream) {
   return gateup_impl(M, N, K, block, Wg, Wu, X, nullptr, nullptr, Y, stream, false, 0u);
@@ -474,6 +545,7 @@ QMM_API qmm_status qmm_device_status(uint32_t *bits) {
   e = prefill_status(&b);
   if (e != cudaSuccess) return cuda_check(e, "status read");
   *bits |= b;
+  if (*bits) return set_error(QMM_ERR_DEVICE_CHECK, "qmm_device_status: a kernel recorded a failure (bits 0x%x)", *bits);
   return QMM_OK;
 }
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/qmm.h"
 
 namespace qmm {
@@ -15,6 +17,18 @@ struct DevInfo {
   int cc_major = 0, cc_minor = 0;
   int smem_optin = 0;  // max dynamic shared memory per block (opt-in)
   int l2_bytes = 0;
+};
+
+// Once-per-device flags for a kernel's attribute set-up (devices 0..63; others
+// always read as done, and their launches use the default attributes).
+// Concurrent first calls may both run the set-up, which is idempotent; the
+// flags themselves are atomic, so the check is free of data races.
+struct DeviceFlags {
+  std::atomic<bool> f[64];
+  bool done(int dev) const { return dev < 0 || dev >= 64 || f[dev].load(std::memory_order_acquire); }
+  void set(int dev) {
+    if (dev >= 0 && dev < 64) f[dev].store(true, std::memory_order_release);
+  }
 };
 
 // Launch options carried from the entry points to the launchers.
@@ -41,8 +55,17 @@ qmm_status launch_q8_gemv_multi(const DevInfo &dev, int M, int K, int nproj, con
 
 qmm_status launch_q8q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,
                             const float *DX, float *Y, cudaStream_t stream, uint32_t flags);
+// The exact block dots of the streaming Q8xQ8 kernel (activations as QX codes,
+// or as Q8_0 blocks XB when XB is set).
 qmm_status launch_q8q8_block_dots(const DevInfo &dev, int M, int64_t N, int K, const void *W, const int8_t *QX,
-                                  int32_t *isum, cudaStream_t stream);
+                                  const uint8_t *XB, int32_t *isum, cudaStream_t stream);
+// launch_q8q8_gemv_fused with the exact block dots written to isum as well.
+qmm_status launch_q8q8_gemv_fused_dots(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
+                                       int8_t *QX, float *DX, float *Y, int32_t *isum, cudaStream_t stream);
+// Failure-path test: the streaming fp32 GEMV with the given wait limit and the
+// first weight stage of CTA 0 withheld.
+qmm_status launch_q8_gemv_withheld(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
+                                   float *Y, uint64_t wait_ns, cudaStream_t stream);
 qmm_status launch_q8q8_gemv_fused(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X,
                                   int8_t *QX, float *DX, float *Y, cudaStream_t stream, uint32_t flags);
 qmm_status launch_quantize_act_q8_0(const DevInfo &dev, int64_t M, int K, const float *X, uint8_t *XB,
@@ -70,6 +93,11 @@ struct PrefillPlan {
 qmm_status launch_prefill(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,
                           const uint16_t *X, float *Y, cudaStream_t stream, uint32_t flags,
                           PrefillPlan *plan = nullptr);
+
+// Failure-path test: the small-M prefill kernel with the given wait limit and
+// CTA 0's weight copy withheld (QMM_ERR_SHAPE if the shape does not take it).
+qmm_status launch_prefill_small_withheld(const DevInfo &dev, int wtype, int64_t M, int64_t N, int K, const void *W,
+                                         const uint16_t *X, float *Y, uint64_t wait_ns, cudaStream_t stream);
 
 // Device status word of each kernel file: read and clear (synchronous).
 cudaError_t q8_gemv_status(uint32_t *bits);

@@ -47,7 +47,9 @@
  *   - A kernel that waits too long on one of its own pipeline barriers (about
  *     two seconds) stops, records the fact in a device status word and returns
  *     instead of hanging; qmm_device_status() reads and clears that word.
- *   - Calls are thread-safe. The entry points keep no state between calls.
+ *   - Calls are thread-safe. What persists between calls is a once-per-device
+ *     kernel attribute set-up and the device status words that
+ *     qmm_device_status() reads and clears; no call's result depends on them.
  *
  * Tolerances the library is tested to (per output, S = sum_k |w_k * x_k|):
  *   fp32-accumulated paths: |y - exact| <= 1e-5 * S;
@@ -365,6 +367,50 @@ QMM_API qmm_status qmm_q8q8_block_dots(int64_t M, int64_t N, int64_t K, int bloc
                                const int8_t *QX, int32_t *isum, qmm_stream_t stream);
 
 /*
+ * qmm_q8q8_gemv_fused_dots -- qmm_q8q8_gemv_fused with its exact int32 block
+ * dots written out as well: isum[n*(K/32) + b] for M = 1, in general
+ * isum[(m*N + n)*(K/32) + b] (M x N x K/32 int32, device, written). The
+ * kernel choice is qmm_q8q8_gemv_fused's; where that is the resident kernel,
+ * its dump instance runs (the same arithmetic plus the store of each dot), so
+ * the per-block integer part of the fused path ("Lumen v0.4.0", section
+ * "Phase 7.M -- Q8xQ8 AVX2 int dot") can be tested bit for bit. Y, QX and DX
+ * are written exactly as by qmm_q8q8_gemv_fused. No options (no early
+ * weights).
+ */
+QMM_API qmm_status qmm_q8q8_gemv_fused_dots(int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                            const float *X, int8_t *QX, float *DX, float *Y, int32_t *isum,
+                                            qmm_stream_t stream);
+
+/*
+ * qmm_q8q8_block_dots_q8_0 -- the exact int32 block dots of
+ * qmm_q8q8_gemv_q8_0 (activations as Q8_0 blocks XB), written out as
+ * isum[(m*N + n)*(K/32) + b]; the same device code as that entry point's.
+ */
+QMM_API qmm_status qmm_q8q8_block_dots_q8_0(int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                            const void *XB, int32_t *isum, qmm_stream_t stream);
+
+/*
+ * qmm_test_withheld_copy -- exercises the bounded-wait failure path (the
+ * "guards" of "LSE v0.4.15", section "Qualification and measurements") without
+ * any fault: one kernel launch in which CTA 0 never issues one of its copies,
+ * so its waits on that copy give up after wait_ns nanoseconds (1e3 .. 2e9).
+ *   kernel 0: the streaming Q8_0 GEMV (M 1..8, X fp32); the first weight
+ *             stage of CTA 0 is withheld.
+ *   kernel 1: the small-M prefill kernel on Q8_0 weights (M 1..32, X bf16;
+ *             QMM_ERR_SHAPE unless qmm_prefill_plan reports that kernel);
+ *             the whole weight copy of CTA 0 (cluster rank 0) is withheld, and
+ *             with split K the other ranks still meet it at the cluster
+ *             barrier.
+ * The starved CTA records kDevTimeout bits in the device status word,
+ * finishes without touching the withheld buffer and returns; the outputs it
+ * owns are left unwritten or undefined, the others are computed as usual.
+ * qmm_device_status() then reports the bits (QMM_ERR_DEVICE_CHECK) and clears
+ * them; later calls are unaffected. Not for production use.
+ */
+QMM_API qmm_status qmm_test_withheld_copy(int kernel, int64_t M, int64_t N, int64_t K, int block, const void *W,
+                                          const void *X, float *Y, uint64_t wait_ns, qmm_stream_t stream);
+
+/*
  * qmm_q4_gateup_unfused -- the unfused counterpart of qmm_q4_swiglu_gateup:
  * writes the gate and up projections G, U (M x N fp32 each) with two separate
  * projection launches, then Y = silu(G) * U with a third launch. Each
@@ -398,9 +444,12 @@ QMM_API const char *qmm_version(void);
 
 /*
  * qmm_device_status -- synchronises the current device, then reads and clears
- * the device-side status word that kernels set when a bounded wait gives up.
- * *bits receives the word (0 = no failure recorded). Returns QMM_OK, or
- * QMM_ERR_CUDA if the synchronisation itself failed.
+ * the device-side status words that kernels set when a bounded wait gives up.
+ * *bits receives their OR (0 = no failure recorded; 1 = a copy or stage never
+ * arrived, 2 = a copy in flight could not be drained on the error path, 4 = a
+ * tensor-core commit never arrived). Returns QMM_OK when *bits == 0,
+ * QMM_ERR_DEVICE_CHECK when a failure was recorded, or QMM_ERR_CUDA if the
+ * synchronisation itself failed.
  */
 QMM_API qmm_status qmm_device_status(uint32_t *bits);
 

@@ -125,3 +125,35 @@ def decode_step_shapes():
 def sub_seed(seed: int, index: int) -> int:
     """Per-tensor seed of tensor ``index`` of a workload drawn with ``seed``."""
     return seed * 1000 + index
+
+
+def decode_step_sources():
+    """Data flow of the decode step's matmuls: for each of the 121, the index of
+    the matmul whose output holds its input (-1: the step's input vector).
+    qkv reads the previous layer's down output, wo reads (the first 896 values
+    of) qkv, gate and up both read wo, down reads up, lm_head the last down."""
+    shapes = decode_step_shapes()
+    src = []
+    last_down = -1
+    for i, (name, _, _) in enumerate(shapes):
+        kind = name.split(".")[-1]
+        if kind == "qkv" or kind == "lm_head":
+            src.append(last_down)
+        elif kind == "wo":
+            src.append(i - 1)
+        elif kind in ("gate", "up"):
+            src.append(i - 1 if kind == "gate" else i - 2)
+        elif kind == "down":
+            src.append(i - 1)
+            last_down = i
+        else:
+            raise ValueError(name)
+    return src
+
+
+def chain_dscale(k: int) -> float:
+    """Scale factor c of Q8_0 scales d = |N(0,1)| c for a chained decode step:
+    with codes uniform in [-127, 127] (rms about 73.6) an output of a K-long
+    row then has about the rms of its input, so 121 chained matmuls neither
+    overflow nor vanish."""
+    return 1.0 / (73.6 * float(np.sqrt(k)))

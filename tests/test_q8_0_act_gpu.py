@@ -66,3 +66,21 @@ def test_quantize_then_gemv_chain_and_flag():
     codes, scales = oracle.split_q8_0_blocks(oracle.quantize_act_q8_0(x), k)
     ref, S = oracle.q8q8_gemv(host(W), codes, scales, n)
     assert_within(host(Y0), ref, S, TOL_FP32, "quantize_act_q8_0 -> q8q8_gemv_q8_0")
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 4864, 896), (1, 896, 4864), (3, 37, 160), (8, 129, 2048)])
+def test_q8_0_block_dots_bit_exact(m, n, k):
+    """The int32 block dots of the GEMV on Q8_0 activation blocks equal the
+    oracle's exact dots on the blocks' codes."""
+    g = syn.rng(7 * n + k + m)
+    W = syn.q8_0_weights(g, n, k, qlo=-128, qhi=127)[0]
+    x = syn.act_f32(g, m, k)
+    xb = oracle.quantize_act_q8_0(x)
+    isum = qmm.qmm_q8q8_block_dots_q8_0(dev(W), dev(xb), k, n)
+    torch.cuda.synchronize()
+    codes, _ = oracle.split_q8_0_blocks(xb, k)
+    ref = oracle.q8q8_block_dots(W, codes, n)
+    got = host(isum)
+    bad = int((got != ref).sum())
+    assert bad == 0, f"{bad} of {ref.size} block dots differ"
+    assert qmm.device_status() == 0

@@ -128,3 +128,32 @@ def test_fused_empty_and_zero_k():
     Y0, _, _ = qmm.qmm_q8q8_gemv_fused(dev(W2), x2, 0)
     assert Y0.shape == (1, 0)
     assert qmm.device_status() == 0
+
+
+@pytest.mark.parametrize("m,n,k", [
+    (1, 4864, 896), (1, 896, 4864),           # the two Q8xQ8 decode shapes, resident kernel
+    (1, 1185, 896), (1, 37, 256),              # ragged splits, fewer rows than CTAs
+    (1, 151936, 896), (3, 129, 2048),          # quantise-then-stream forms
+])
+def test_fused_block_dots_bit_exact(m, n, k):
+    """The int32 block dots of the fused Q8xQ8 path (the kernel qmm_q8q8_gemv_fused
+    runs, in its dump instance) equal the oracle's exact dots on the oracle's
+    codes; Y, QX and DX equal qmm_q8q8_gemv_fused's bit for bit."""
+    g = syn.rng(11 * n + k + m)
+    W, _, _ = syn.q8_0_weights(g, n, k, qlo=-128, qhi=127)
+    x = syn.act_f32(g, m, k)
+    x[0, :32] = np.float32(-2.5)                              # equal magnitudes: codes of +-127
+    Y, QX, DX, isum = qmm.qmm_q8q8_gemv_fused_dots(dev(W), dev(x), n)
+    Yf, QXf, DXf = qmm.qmm_q8q8_gemv_fused(dev(W), dev(x), n)
+    torch.cuda.synchronize()
+    qr, dr = oracle.quantize_act_q8(x)
+    assert np.array_equal(host(QX), qr) and np.array_equal(host(DX).view(np.uint32), dr.view(np.uint32))
+    win = (0, m, 0, min(n, 8192))
+    ref = oracle.q8q8_block_dots(W, qr, n, window=win)
+    got = host(isum)[:, :win[3], :]
+    assert got.shape == ref.shape
+    bad = int((got != ref).sum())
+    assert bad == 0, f"{bad} of {ref.size} block dots differ"
+    assert torch.equal(Y.view(torch.int32), Yf.view(torch.int32))
+    assert torch.equal(QX, QXf) and torch.equal(DX.view(torch.int32), DXf.view(torch.int32))
+    assert qmm.device_status() == 0
