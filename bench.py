@@ -3,9 +3,12 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-components]
 
 One step = the 121 weight matmuls of one decode token (24 layers x {qkv 896->1152,
-wo 896->896, gate 896->4864, up 896->4864, down 4864->896} + lm_head 896->151936),
-each a qmm_q8_gemv call (M=1, Q8_0 blocks, fp32 activations), stream-ordered and
-replayed as one CUDA graph with programmatic dependent launch. Weights are seeded
+wo 896->896, gate 896->4864, up 896->4864, down 4864->896} + lm_head 896->151936)
+on Q8_0 blocks with fp32 activations (M=1), stream-ordered and replayed as one CUDA
+graph with programmatic dependent launch. Default schedule ("multi", 97 launches):
+gate and up of each layer, which read the same activation vector, share one
+qmm_q8_gemv_multi launch; every other matmul is one qmm_q8_gemv_ex call.
+`--schedule gemv` issues the 121 matmuls as 121 qmm_q8_gemv_ex calls. Weights are seeded
 synthetic tensors with the shapes of that model (no trained weights are used);
 they total 524,833,792 bytes per step, more than the 126 MB L2, so no flush is
 needed between steps. value = decode tokens/s (steps/s) summed over ranks.
@@ -385,22 +388,19 @@ def component_lm_head(qmm, step: DecodeStep, dev_peak_gbs, reps=20):
     return out
 
 
-def component_step_multi(qmm, step: DecodeStep, dev_peak_gbs, reps=200):
-    """The decode step's matmul set with gate and up of each layer sharing one
-    activation vector in one qmm_q8_gemv_multi launch (97 launches instead of
-    121; same bytes). A variant next to the headline, which keeps 121 GEMVs."""
+def component_step_schedule(qmm, step: DecodeStep, schedule: str, dev_peak_gbs, reps=200):
+    """The decode step's matmul set under another schedule than the headline's
+    ("gemv": 121 qmm_q8_gemv_ex launches; "multi": gate and up of each layer in
+    one qmm_q8_gemv_multi launch, 97 launches; same bytes)."""
     import torch
 
     s = torch.cuda.Stream()
-    flags = qmm.QMM_FLAG_EARLY_WEIGHTS
-    step.launch_multi(qmm, s.cuda_stream, flags)
-    torch.cuda.synchronize()
-    gr = capture(lambda h: step.launch_multi(qmm, h, flags), s)
+    gr = step_graph(qmm, step, s, schedule, qmm.QMM_FLAG_EARLY_WEIGHTS)
     time_graph(gr, s, 20)
     ms = time_graph(gr, s, reps)
     del gr
     bytes_ = sum(n * (k // 32) * 34 + k * 4 + n * 4 for _, n, k in step.shapes)
-    return {"ms_per_step": round(ms, 5), "tok_s": round(1e3 / ms, 2), "launches": 97,
+    return {"ms_per_step": round(ms, 5), "tok_s": round(1e3 / ms, 2), "launches": step.launches(schedule),
             "GB_s": round(bytes_ / ms / 1e6, 1), "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4)}
 
 
@@ -798,7 +798,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None, help="launch one named kernel (see run_case) instead of the benchmark")
     ap.add_argument("--reps", type=int, default=3)
-    ap.add_argument("--schedule", default="gemv", choices=["gemv", "multi"],
+    ap.add_argument("--schedule", default="multi", choices=["gemv", "multi"],
                     help="decode-step schedule: 121 qmm_q8_gemv_ex launches, or gate+up of each layer in one "
                          "qmm_q8_gemv_multi launch (97)")
     args = ap.parse_args(argv)
@@ -899,7 +899,9 @@ def main(argv=None):
     components = None
     if rank == 0 and world == 1 and not args.no_components:
         components = {"lm_head_896x151936": component_lm_head(qmm, step, pk["hbm_gbs"]),
-                      "decode_step_gate_up_multi": component_step_multi(qmm, step, pk["hbm_gbs"]),
+                      ("decode_step_121_gemv" if args.schedule == "multi" else "decode_step_gate_up_multi"):
+                          component_step_schedule(qmm, step, "gemv" if args.schedule == "multi" else "multi",
+                                                  pk["hbm_gbs"]),
                       "decode_step_per_k_q8q8": component_step_auto(qmm, step, pk["hbm_gbs"]),
                       "single_gemv_896x1152": component_single_gemv(qmm, pk["hbm_gbs"]),
                       "q4_gateup_m8_k5120_n17408": component_gateup(qmm, pk["hbm_gbs"]),

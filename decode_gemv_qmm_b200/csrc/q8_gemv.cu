@@ -1221,6 +1221,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *empty = full + kMaxStages;
   int *emax = reinterpret_cast<int *>(empty + kMaxStages);
+  int *wmax = emax + 2;  // [kDigitWarps]: each consumer warp's largest block exponent
   uint2 *tab = reinterpret_cast<uint2 *>(smem + p.tab_off);     // [KB][32 lanes] B registers
   float *ftab = reinterpret_cast<float *>(smem + p.ftab_off);   // [KB] 2^(E_b - E)
   int *ebt = reinterpret_cast<int *>(smem + p.eb_off);          // [KB] E_b
@@ -1334,20 +1335,35 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   pdl_wait();
   const int ctid = tid - 32;  // 0 .. 255
   const int units = p.KB * 8;  // (block, t, half): four activations each
-  // pass 1: block exponents and the vector's largest
-  for (int u = ctid; u < units; u += 32 * kDigitWarps) {
-    const int b = u >> 3;
-    const float4 v = __ldg(reinterpret_cast<const float4 *>(p.X) + u);
-    const uint32_t m = max(max(__float_as_uint(v.x) & 0x7fffffffu, __float_as_uint(v.y) & 0x7fffffffu),
-                           max(__float_as_uint(v.z) & 0x7fffffffu, __float_as_uint(v.w) & 0x7fffffffu));
+  // pass 1: block exponents (the eight units of a block are eight lanes of a
+  // warp: a shuffle max, one writer) and the vector's largest (per warp, then
+  // over the warps; shared-memory atomics on one address would serialise)
+  int wmaxE = 1;
+  for (int base = (warp - 1) * 32; base < units; base += 32 * kDigitWarps) {  // warp-uniform: it shuffles
+    const int u = base + lane;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (u < units) v = __ldg(reinterpret_cast<const float4 *>(p.X) + u);
+    uint32_t m = max(max(__float_as_uint(v.x) & 0x7fffffffu, __float_as_uint(v.y) & 0x7fffffffu),
+                     max(__float_as_uint(v.z) & 0x7fffffffu, __float_as_uint(v.w) & 0x7fffffffu));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
     const int E = max(static_cast<int>(m >> 23), 1);
-    atomicMax(&ebt[b], E);
-    atomicMax(emax, E);
+    wmaxE = max(wmaxE, E);
+    if (u < units && (u & 7) == 0) ebt[u >> 3] = E;
   }
+  wmaxE = __reduce_max_sync(0xffffffffu, wmaxE);
+  if (lane == 0) wmax[warp - 1] = wmaxE;
   asm volatile("bar.sync 1, %0;" ::"n"(32 * kDigitWarps) : "memory");
+  if (ctid == 0) {  // read by the producer after the consumers release their first stage
+    int e = 1;
+    for (int w = 0; w < kDigitWarps; ++w) e = max(e, wmax[w]);
+    *emax = e;
+  }
   // pass 2: the digits, transposed into B registers: lane (k, t) of block b
   // holds digit k of activations 8t..8t+3 (word 0) and 8t+4..8t+7 (word 1)
-  const int Emax = *emax;
+  int Emax = 1;
+  for (int w = 0; w < kDigitWarps; ++w) Emax = max(Emax, wmax[w]);
   for (int u = ctid; u < units; u += 32 * kDigitWarps) {
     const int b = u >> 3, t = (u >> 1) & 3, h = u & 1;
     const int Eb = ebt[b];
