@@ -785,6 +785,79 @@ def run_case(spec: str, reps: int, seed: int):
     return 0
 
 
+# --------------------------------------------------------------------------- tensor parallel (column shards)
+
+def run_tensor_parallel(args):
+    """The decode step with every weight matrix's rows split over the ranks
+    (decode_gemv_qmm_b200.shard: rank r owns rows [r N / G, (r + 1) N / G) of
+    each matrix, computes its slice with qmm_q8_gemv and the slices are
+    all-gathered after each matmul). Strong scaling: all ranks work on the same
+    token, value = steps/s of the whole job. Launches are eager (the NCCL
+    all-gathers are not captured in a CUDA graph)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import decode_gemv_qmm_b200 as qmm
+    from decode_gemv_qmm_b200 import shard
+
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    shapes = syn.decode_step_shapes()
+    Wl, Xs, Yl = [], [], []
+    for i, (_, n, k) in enumerate(shapes):
+        g = syn.rng(syn.sub_seed(args.seed, i))
+        wb, _, _ = syn.q8_0_weights(g, n, k)
+        x = syn.act_f32(g, 1, k)
+        r0, r1 = shard.row_range(n, rank, world)
+        Wl.append(torch.from_numpy(np.ascontiguousarray(shard.weight_shard(wb, n, k, rank, world))).to(dev))
+        Xs.append(torch.from_numpy(x).to(dev))
+        Yl.append(torch.empty((1, r1 - r0), dtype=torch.float32, device=dev))
+
+    def step():
+        outs = []
+        for i, (_, n, k) in enumerate(shapes):
+            qmm.qmm_q8_gemv(Wl[i], Xs[i], Yl[i].shape[1], Yl[i], flags=qmm.QMM_FLAG_EARLY_WEIGHTS)
+            outs.append(shard.gather_rows(Yl[i], n, rank, world))
+        return outs
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    if rank == 0:
+        wb, xb, yb = step_bytes()
+        line = {"metric": METRIC, "value": round(args.steps / (ms / 1000.0), 2), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic",
+                "config": {"workload": WORKLOAD, "M": 1, "weight_format": "Q8_0", "bytes_per_step": wb + xb + yb,
+                           "parallelism": f"tp{world} (column shards, all-gather after each matmul; eager)"},
+                "gpu_launches": len(shapes) * args.steps}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 # --------------------------------------------------------------------------- main
 
 def main(argv=None):
@@ -801,6 +874,8 @@ def main(argv=None):
     ap.add_argument("--schedule", default="multi", choices=["gemv", "multi"],
                     help="decode-step schedule: 121 qmm_q8_gemv_ex launches, or gate+up of each layer in one "
                          "qmm_q8_gemv_multi launch (97)")
+    ap.add_argument("--parallel", default="dp", choices=["dp", "tp"],
+                    help="N > 1: data-parallel replicas (default) or column-sharded weights (tp)")
     args = ap.parse_args(argv)
     if args.case:
         return run_case(args.case, args.reps, args.seed)
@@ -808,6 +883,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.parallel == "tp":
+        return run_tensor_parallel(args)
 
     import torch
 
