@@ -47,6 +47,7 @@
 // (writing G, then U) and a third launch applying silu(G) * U with the same
 // device function, so the fused output equals the unfused one bit for bit.
 #include <algorithm>
+#include <type_traits>
 
 #include "qmm_common.cuh"
 #include "qmm_internal.h"
@@ -340,78 +341,88 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
       for (int k = 0; k < 4; ++k) acc[i][mat][k] = 0.f;
 
   const int64_t row_bytes = 18ll * p.KB;
-  for (int j = 0; j < nstages; ++j) {
-    const int s = j % kStages;
-    if (!DIRECT && !mbar_wait(&full[s], static_cast<uint32_t>(j / kStages) & 1u)) {
-      if (lane == 0) atomicOr(&g_q4_status, kDevTimeoutFull);
-      if (split == 1) return;  // the producer gives up on this warp's missing arrival and drains
-      break;                   // split K: still meet the cluster barriers
-    }
-    const int kb = (j_lo + j) * kBlocksPerStage + wb;  // this warp's block
-    if (kb < p.KB) {
-      // activations of block kb for token g
-      float4 x0, x1;
-      if (!DIRECT) {
-        const uint32_t xa = smem_u32(stages + s * kStageBytes + wb * 1024) + g * 128;
-        x0 = lds_f4(xa + 16u * (t ^ g));
-        x1 = lds_f4(xa + 16u * ((4 + t) ^ g));
-      } else if (g < p.M) {
-        const float4 *xp = reinterpret_cast<const float4 *>(p.X + static_cast<int64_t>(g) * p.K + 32 * kb);
-        x0 = __ldg(xp + t);
-        x1 = __ldg(xp + 4 + t);
-      } else {
-        x0 = x1 = make_float4(0.f, 0.f, 0.f, 0.f);
+  // The stage loop, compiled once per parity of this warp's block (fixed for
+  // the whole kernel): odd blocks start 2 bytes past a 4-byte boundary, so
+  // their code words are aligned; even ones need a funnel shift. Returns 0, or
+  // on a timeout 1 (leave) / 2 (split K: go on to the cluster barriers).
+  auto stage_loop = [&](auto parity) -> int {
+    constexpr bool kOdd = decltype(parity)::value;
+    for (int j = 0; j < nstages; ++j) {
+      const int s = j % kStages;
+      if (!DIRECT && !mbar_wait(&full[s], static_cast<uint32_t>(j / kStages) & 1u)) {
+        if (lane == 0) atomicOr(&g_q4_status, kDevTimeoutFull);
+        return split == 1 ? 1 : 2;  // 1: leave (the producer gives up on this warp's missing
+                                    // arrival and drains); 2: split K, still meet the cluster barriers
       }
-      const BFrag bf = make_bfrag(x0, x1);
-#pragma unroll
-      for (int mat = 0; mat < 2; ++mat) {
-        if (mat >= NMAT) break;
-#pragma unroll
-        for (int ii = 0; ii < kTilesMax / kHalves; ++ii) {
-          const int i = ii * kHalves + th;  // this warp's share of the row tiles
-          // Staged tiles: no exit, so the loads of all tiles can be issued
-          // together; a tile past ntiles reads stale stage bytes and its
-          // accumulators are never used.
-          if (DIRECT && i >= ntiles) break;
-          uint32_t vg, vh;
-          float dg, dh;
-          if (!DIRECT) {
-            // row r of the tile at r * 144 bytes; block `wb` at 18 * wb
-            const uint32_t tb = smem_u32(stages + s * kStageBytes + kXStageBytes + (mat * kTilesMax + i) * kTileBytes);
-            const uint32_t ag = tb + g * kRowStageBytes + 18 * wb, ah = ag + 8 * kRowStageBytes;
-            if (wb & 1) {  // block starts 2 bytes past a 4-byte boundary: qs word aligned
-              vg = lds_u32(ag + 2 + 4 * t);
-              vh = lds_u32(ah + 2 + 4 * t);
-            } else {
-              vg = __funnelshift_r(lds_u32(ag + 4 * t), lds_u32(ag + 4 * t + 4), 16);
-              vh = __funnelshift_r(lds_u32(ah + 4 * t), lds_u32(ah + 4 * t + 4), 16);
-            }
-            dg = half_bits_to_float(lds_u16(ag));
-            dh = half_bits_to_float(lds_u16(ah));
-          } else {
-            const int64_t rg = 16ll * (tile0 + i) + g, rh = rg + 8;
-            const uint8_t *Wm = p.W[mat];
-            auto word = [&](int64_t r, float &d) -> uint32_t {
-              if (r >= p.N) {
-                d = 0.f;
-                return 0x88888888u;  // nibbles 8 -> value 0
+      const int kb = (j_lo + j) * kBlocksPerStage + wb;  // this warp's block
+      if (kb < p.KB) {
+        // activations of block kb for token g
+        float4 x0, x1;
+        if (!DIRECT) {
+          const uint32_t xa = smem_u32(stages + s * kStageBytes + wb * 1024) + g * 128;
+          x0 = lds_f4(xa + 16u * (t ^ g));
+          x1 = lds_f4(xa + 16u * ((4 + t) ^ g));
+        } else if (g < p.M) {
+          const float4 *xp = reinterpret_cast<const float4 *>(p.X + static_cast<int64_t>(g) * p.K + 32 * kb);
+          x0 = __ldg(xp + t);
+          x1 = __ldg(xp + 4 + t);
+        } else {
+          x0 = x1 = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        const BFrag bf = make_bfrag(x0, x1);
+  #pragma unroll
+        for (int mat = 0; mat < 2; ++mat) {
+          if (mat >= NMAT) break;
+  #pragma unroll
+          for (int ii = 0; ii < kTilesMax / kHalves; ++ii) {
+            const int i = ii * kHalves + th;  // this warp's share of the row tiles
+            // Staged tiles: no exit, so the loads of all tiles can be issued
+            // together; a tile past ntiles reads stale stage bytes and its
+            // accumulators are never used.
+            if (DIRECT && i >= ntiles) break;
+            uint32_t vg, vh;
+            float dg, dh;
+            if (!DIRECT) {
+              // row r of the tile at r * 144 bytes; block `wb` at 18 * wb
+              const uint32_t tb = smem_u32(stages + s * kStageBytes + kXStageBytes + (mat * kTilesMax + i) * kTileBytes);
+              const uint32_t ag = tb + g * kRowStageBytes + 18 * wb, ah = ag + 8 * kRowStageBytes;
+              if constexpr (kOdd) {  // block starts 2 bytes past a 4-byte boundary: qs word aligned
+                vg = lds_u32(ag + 2 + 4 * t);
+                vh = lds_u32(ah + 2 + 4 * t);
+              } else {
+                vg = __funnelshift_r(lds_u32(ag + 4 * t), lds_u32(ag + 4 * t + 4), 16);
+                vh = __funnelshift_r(lds_u32(ah + 4 * t), lds_u32(ah + 4 * t + 4), 16);
               }
-              const uint16_t *bp = reinterpret_cast<const uint16_t *>(Wm + r * row_bytes + 18ll * kb);
-              d = half_bits_to_float(__ldg(bp));
-              return static_cast<uint32_t>(__ldg(bp + 1 + 2 * t)) | (static_cast<uint32_t>(__ldg(bp + 2 + 2 * t)) << 16);
-            };
-            vg = word(rg, dg);
-            vh = word(rh, dh);
+              dg = half_bits_to_float(lds_u16(ag));
+              dh = half_bits_to_float(lds_u16(ah));
+            } else {
+              const int64_t rg = 16ll * (tile0 + i) + g, rh = rg + 8;
+              const uint8_t *Wm = p.W[mat];
+              auto word = [&](int64_t r, float &d) -> uint32_t {
+                if (r >= p.N) {
+                  d = 0.f;
+                  return 0x88888888u;  // nibbles 8 -> value 0
+                }
+                const uint16_t *bp = reinterpret_cast<const uint16_t *>(Wm + r * row_bytes + 18ll * kb);
+                d = half_bits_to_float(__ldg(bp));
+                return static_cast<uint32_t>(__ldg(bp + 1 + 2 * t)) | (static_cast<uint32_t>(__ldg(bp + 2 + 2 * t)) << 16);
+              };
+              vg = word(rg, dg);
+              vh = word(rh, dh);
+            }
+            tile_block(acc[ii][mat], vg, vh, dg, dh, bf);
           }
-          tile_block(acc[ii][mat], vg, vh, dg, dh, bf);
         }
       }
+      if (!DIRECT) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
     }
-    if (!DIRECT) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-    }
-  }
+    return 0;
+  };
+  const int loop_rc = (wb & 1) ? stage_loop(std::true_type{}) : stage_loop(std::false_type{});
+  if (loop_rc == 1) return;
 
   // ------------------------------------------ cross-warp sum, SwiGLU epilogue
   // Every consumer has passed its last stage, so the stage memory is free.
