@@ -421,7 +421,12 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1) q4_gateup_kernel(const _
     }
     return 0;
   };
-  const int loop_rc = (wb & 1) ? stage_loop(std::true_type{}) : stage_loop(std::false_type{});
+  int loop_rc;
+  if constexpr (DIRECT) {  // reads global memory: the parity does not matter
+    loop_rc = stage_loop(std::false_type{});
+  } else {
+    loop_rc = (wb & 1) ? stage_loop(std::true_type{}) : stage_loop(std::false_type{});
+  }
   if (loop_rc == 1) return;
 
   // ------------------------------------------ cross-warp sum, SwiGLU epilogue

@@ -1335,9 +1335,11 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   pdl_wait();
   const int ctid = tid - 32;  // 0 .. 255
   const int units = p.KB * 8;  // (block, t, half): four activations each
-  // pass 1: block exponents (the eight units of a block are eight lanes of a
-  // warp: a shuffle max, one writer) and the vector's largest (per warp, then
-  // over the warps; shared-memory atomics on one address would serialise)
+  // One pass over x: block exponents (the eight units of a block are eight
+  // lanes of a warp: a shuffle max), then the unit's digits, transposed into B
+  // registers (lane (k, t) of block b holds digit k of activations 8t..8t+3 in
+  // word 0 and 8t+4..8t+7 in word 1); the vector's largest exponent per warp,
+  // then over the warps (shared-memory atomics on one address would serialise).
   int wmaxE = 1;
   for (int base = (warp - 1) * 32; base < units; base += 32 * kDigitWarps) {  // warp-uniform: it shuffles
     const int u = base + lane;
@@ -1348,44 +1350,39 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
     m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    const int E = max(static_cast<int>(m >> 23), 1);
-    wmaxE = max(wmaxE, E);
-    if (u < units && (u & 7) == 0) ebt[u >> 3] = E;
+    const int Eb = max(static_cast<int>(m >> 23), 1);
+    wmaxE = max(wmaxE, Eb);
+    if (u < units) {
+      const int b = u >> 3, t = (u >> 1) & 3, h = u & 1;
+      if ((u & 7) == 0) ebt[b] = Eb;
+      const uint64_t bias = 0x8080808080808080ull;
+      const uint64_t d0 = (static_cast<uint64_t>(x_fixed(v.x, Eb)) + bias) ^ bias;
+      const uint64_t d1 = (static_cast<uint64_t>(x_fixed(v.y, Eb)) + bias) ^ bias;
+      const uint64_t d2 = (static_cast<uint64_t>(x_fixed(v.z, Eb)) + bias) ^ bias;
+      const uint64_t d3 = (static_cast<uint64_t>(x_fixed(v.w, Eb)) + bias) ^ bias;
+      uint32_t *tb = reinterpret_cast<uint32_t *>(tab + b * 32);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {  // digits 0..3, then 4..7
+        const uint32_t w0 = static_cast<uint32_t>(d0 >> (32 * half)), w1 = static_cast<uint32_t>(d1 >> (32 * half));
+        const uint32_t w2 = static_cast<uint32_t>(d2 >> (32 * half)), w3 = static_cast<uint32_t>(d3 >> (32 * half));
+        const uint32_t l01 = __byte_perm(w0, w1, 0x5140u), h01 = __byte_perm(w0, w1, 0x7362u);
+        const uint32_t l23 = __byte_perm(w2, w3, 0x5140u), h23 = __byte_perm(w2, w3, 0x7362u);
+        const uint32_t dig[4] = {__byte_perm(l01, l23, 0x5410u), __byte_perm(l01, l23, 0x7632u),
+                                 __byte_perm(h01, h23, 0x5410u), __byte_perm(h01, h23, 0x7632u)};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) tb[2 * ((4 * half + k) * 4 + t) + h] = dig[k];  // lane 4k' + t, word h
+      }
+    }
   }
   wmaxE = __reduce_max_sync(0xffffffffu, wmaxE);
   if (lane == 0) wmax[warp - 1] = wmaxE;
   asm volatile("bar.sync 1, %0;" ::"n"(32 * kDigitWarps) : "memory");
-  if (ctid == 0) {  // read by the producer after the consumers release their first stage
-    int e = 1;
-    for (int w = 0; w < kDigitWarps; ++w) e = max(e, wmax[w]);
-    *emax = e;
-  }
-  // pass 2: the digits, transposed into B registers: lane (k, t) of block b
-  // holds digit k of activations 8t..8t+3 (word 0) and 8t+4..8t+7 (word 1)
   int Emax = 1;
   for (int w = 0; w < kDigitWarps; ++w) Emax = max(Emax, wmax[w]);
-  for (int u = ctid; u < units; u += 32 * kDigitWarps) {
-    const int b = u >> 3, t = (u >> 1) & 3, h = u & 1;
-    const int Eb = ebt[b];
-    const float4 v = __ldg(reinterpret_cast<const float4 *>(p.X) + u);
-    const uint64_t bias = 0x8080808080808080ull;
-    const uint64_t d0 = (static_cast<uint64_t>(x_fixed(v.x, Eb)) + bias) ^ bias;
-    const uint64_t d1 = (static_cast<uint64_t>(x_fixed(v.y, Eb)) + bias) ^ bias;
-    const uint64_t d2 = (static_cast<uint64_t>(x_fixed(v.z, Eb)) + bias) ^ bias;
-    const uint64_t d3 = (static_cast<uint64_t>(x_fixed(v.w, Eb)) + bias) ^ bias;
-    uint32_t *tb = reinterpret_cast<uint32_t *>(tab + b * 32);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {  // digits 0..3, then 4..7
-      const uint32_t w0 = static_cast<uint32_t>(d0 >> (32 * half)), w1 = static_cast<uint32_t>(d1 >> (32 * half));
-      const uint32_t w2 = static_cast<uint32_t>(d2 >> (32 * half)), w3 = static_cast<uint32_t>(d3 >> (32 * half));
-      const uint32_t l01 = __byte_perm(w0, w1, 0x5140u), h01 = __byte_perm(w0, w1, 0x7362u);
-      const uint32_t l23 = __byte_perm(w2, w3, 0x5140u), h23 = __byte_perm(w2, w3, 0x7362u);
-      const uint32_t dig[4] = {__byte_perm(l01, l23, 0x5410u), __byte_perm(l01, l23, 0x7632u),
-                               __byte_perm(h01, h23, 0x5410u), __byte_perm(h01, h23, 0x7632u)};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) tb[2 * ((4 * half + k) * 4 + t) + h] = dig[k];  // lane 4k' + t, word h
-    }
-    if (t == 0 && h == 0) ftab[b] = Eb - Emax >= -126 ? __int_as_float((127 + Eb - Emax) << 23) : 0.f;
+  if (ctid == 0) *emax = Emax;  // read by the producer after the consumers release their first stage
+  for (int b = ctid; b < p.KB; b += 32 * kDigitWarps) {
+    const int eb = ebt[b] - Emax;
+    ftab[b] = eb >= -126 ? __int_as_float((127 + eb) << 23) : 0.f;
   }
   asm volatile("bar.sync 1, %0;" ::"n"(32 * kDigitWarps) : "memory");
 
