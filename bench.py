@@ -256,11 +256,20 @@ class DecodeStep:
                 raise qmm.QmmError(st, "qmm_q8_gemv_auto")
 
     def schedule(self, name: str):
-        """The launch function of a named schedule ("gemv": 121 launches, "multi": 97)."""
+        """The launch function of a named schedule ("gemv": 121 launches, "multi": 97,
+        "auto": 121 qmm_q8_gemv_auto calls sharing the step's code/scale buffers)."""
+        if name == "auto":
+            if not hasattr(self, "_qx"):
+                import torch
+
+                kmax = max(k for _, _, k in self.shapes)
+                self._qx = torch.empty(kmax, dtype=torch.int8, device=self.X.device)
+                self._dx = torch.empty(kmax // 32, dtype=torch.float32, device=self.X.device)
+            return lambda qmm, h, flags: self.launch_auto(qmm, h, flags, self._qx, self._dx)
         return {"gemv": self.launch, "multi": self.launch_multi}[name]
 
     def launches(self, name: str) -> int:
-        return len(self.shapes) if name == "gemv" else len(self.shapes) - QWEN_LAYERS
+        return len(self.shapes) - QWEN_LAYERS if name == "multi" else len(self.shapes)
 
     def x_of(self, i: int, Y_host=None):
         """Host copy of matmul i's input vector (from Y_host, the step's outputs, in chain mode)."""
@@ -408,23 +417,9 @@ def component_step_auto(qmm, step: DecodeStep, dev_peak_gbs, reps=200):
     """The decode step's matmul set through the per-K choice (qmm_q8_gemv_auto):
     short-K GEMVs as fused Q8xQ8 on quantised activations, long-K ones fp32 --
     a different numerical contract from the headline's fp32 activations."""
-    import torch
-
-    kmax = max(k for _, _, k in step.shapes)
-    qx = torch.empty(kmax, dtype=torch.int8, device="cuda")
-    dx = torch.empty(kmax // 32, device="cuda")
-    s = torch.cuda.Stream()
-    flags = qmm.QMM_FLAG_EARLY_WEIGHTS
-    step.launch_auto(qmm, s.cuda_stream, flags, qx, dx)
-    torch.cuda.synchronize()
-    gr = capture(lambda h: step.launch_auto(qmm, h, flags, qx, dx), s)
-    time_graph(gr, s, 20)
-    ms = time_graph(gr, s, reps)
-    del gr
-    bytes_ = sum(n * (k // 32) * 34 + k * 4 + n * 4 for _, n, k in step.shapes)
-    return {"ms_per_step": round(ms, 5), "tok_s": round(1e3 / ms, 2),
-            "GB_s": round(bytes_ / ms / 1e6, 1), "frac_hbm": round(bytes_ / ms / 1e6 / dev_peak_gbs, 4),
-            "note": "qkv, wo, gate, up as fused Q8xQ8 (quantised activations); down and lm_head fp32"}
+    out = component_step_schedule(qmm, step, "auto", dev_peak_gbs, reps)
+    out["note"] = "qkv, wo, gate, up as fused Q8xQ8 (quantised activations); down and lm_head fp32"
+    return out
 
 
 def component_gateup(qmm, dev_peak_gbs, m=8, n=17408, k=5120, reps=10):

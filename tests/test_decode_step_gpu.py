@@ -117,3 +117,36 @@ def test_chained_step_magnitudes_stay_bounded():
         rms = float(np.sqrt(np.mean(np.square(y.astype(np.float64)))))
         assert 0.05 < rms < 20.0, f"{name}: rms {rms}"
     del graph
+
+
+def test_decode_step_auto_schedule_matches_oracle():
+    """The per-K schedule the benchmark also times (qmm_q8_gemv_auto on every
+    matmul, one code/scale buffer for the whole step): qkv, wo, gate and up
+    (K = 896, slices on chip) are the Q8xQ8 product of the activations
+    quantised per block, down (K = 4864) and lm_head (slice too large) the
+    fp32 GEMV. Each output is compared with the oracle of the form it took,
+    on a chained step, after replays of the graph."""
+    step = bench.DecodeStep(0, torch.device("cuda", 0), keep_host=True, chain=True)
+    stream = torch.cuda.Stream()
+    graph = bench.step_graph(qmm, step, stream, "auto", qmm.QMM_FLAG_EARLY_WEIGHTS)
+    step.Y.fill_(float("nan"))
+    torch.cuda.synchronize()
+    Y = run_graph(step, graph, stream, 2)
+    assert np.all(np.isfinite(Y))
+    for i, (name, n, k) in enumerate(step.shapes):
+        got = Y[int(step.y_offsets[i]):int(step.y_offsets[i + 1])]
+        x = step.x_of(i, Y)
+        kind = name.split(".")[-1]
+        if kind in ("qkv", "wo", "gate", "up"):
+            qx, dx = oracle.quantize_act_q8(x)
+            ref, S = oracle.q8q8_gemv(step.host_w[i], qx, dx, n)
+        elif n > 8192:
+            parts = [oracle.gemv(syn.Q8_0, step.host_w[i], x, n, window=(0, 1, n0, min(n, n0 + 16384)))
+                     for n0 in range(0, n, 16384)]
+            ref = np.concatenate([p[0] for p in parts], axis=1)
+            S = np.concatenate([p[1] for p in parts], axis=1)
+        else:
+            ref, S = oracle.gemv(syn.Q8_0, step.host_w[i], x, n)
+        assert_within(got, ref[0], S[0], TOL_FP32, f"auto {name}")
+    assert qmm.device_status() == 0
+    del graph
