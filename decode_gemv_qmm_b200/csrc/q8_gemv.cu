@@ -54,6 +54,7 @@
 // activation vector in one launch), and the fused Q8xQ8 resident kernel that
 // quantises the activations itself.
 #include <algorithm>
+#include <type_traits>
 
 #include "qmm_common.cuh"
 #include "qmm_internal.h"
@@ -1150,15 +1151,23 @@ __global__ void __launch_bounds__(256, 2) q8_gemv_mma_kernel(const __grid_consta
 //    becomes the integer x_int = M_j 2^(E_j - E_b + 38) (rounded to nearest
 //    for elements 2^38 below the block's largest exponent E_b), |x_int| <
 //    2^62, written as eight balanced base-256 digits in [-128, 127]: the
-//    bytes of (x_int + 0x8080..80) xor 0x8080..80. Digit k of the eight
-//    activations of a lane's k slots forms B column k.
+//    bytes of (x_int + 0x8080..80) xor 0x8080..80. Digit k of the block's
+//    activations forms B column k (k order within the block as stored).
 //  * C column k = sum_j q_j digit_k(x_j): exact int32 (|C| < 2^20). Thread
-//    (g, t) holds digits 2t, 2t+1 for rows g and g + 8 and adds
-//    (C_2t 2^16t + C_2t+1 2^(16t+8)) * d * 2^(E_b - E) in fp32 (E the largest
-//    E_b of the vector); the four digit lanes are summed at the end and the
-//    row total is scaled by 2^(E - 188). The only rounding is fp32's: the
-//    activation representation is exact for every element within 2^38 of its
-//    block maximum.
+//    (g, t) holds digits 2t, 2t+1 of its two rows; C_2t + 256 C_2t+1 is an
+//    exact int32 (< 2^28), converted once and scaled by d * 2^(E_b - E + 16t)
+//    in fp32 (E the largest E_b of the vector); the four digit lanes are
+//    summed at the end and the row total is scaled by 2^(E - 188). Apart from
+//    fp32 rounding the activation representation is exact for every element
+//    within 2^38 of its block maximum.
+//  * Shared-memory layout: a stage is a verbatim copy of consecutive rows
+//    (34-byte blocks). MMA rows g and g + 8 of a tile are the tile's rows 2g
+//    and 2g + 1: with the 952-byte rows of K = 896 the eight rows 2g start
+//    28 banks apart, so every code load of a warp touches 32 distinct banks
+//    (consecutive rows put all lanes on even banks, 2- to 3-way conflicts).
+//    When rows are 4-byte multiples the codes of odd blocks are word-aligned
+//    (two loads per row) and those of even blocks start 2 bytes past a word
+//    (four loads and two byte permutes); the loop takes blocks in pairs.
 //  * Rows come in 16-row tiles; 32 rows (two tiles) per stage for K <= 1024,
 //    16 otherwise. Eight consumer warps split a stage as (tile, K slice); the
 //    producer warp sums the K slices of each row in slice order when the
@@ -1182,10 +1191,12 @@ struct alignas(64) DParams {
   int stages;
   int stage_bytes;
   int tab_off, ftab_off, eb_off, red_off, stage_off;  // shared-memory offsets
+  int rows_aligned;  // row_bytes % 4 == 0 (even KB): parity-specialised code loads
   int prefetch_before_wait;
 };
 
 constexpr int kDigitWarps = 8;
+constexpr int kMaxSliceBlocks = 16;  // blocks of one K slice: ceil(64 / 4) at K <= 2048
 
 __device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                            uint32_t b0, uint32_t b1) {
@@ -1210,10 +1221,6 @@ __device__ __forceinline__ long long x_fixed(float x, int Eb) {
   return (b >> 31) ? -static_cast<long long>(v) : static_cast<long long>(v);
 }
 
-__device__ __forceinline__ float int_exact_f(int v) {  // |v| < 2^22
-  return __int_as_float(v + 0x4B400000) - 12582912.0f;
-}
-
 template <int TPS, bool MULTI>
 __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(const __grid_constant__ DParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1223,7 +1230,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   int *emax = reinterpret_cast<int *>(empty + kMaxStages);
   int *wmax = emax + 2;  // [kDigitWarps]: each consumer warp's largest block exponent
   uint2 *tab = reinterpret_cast<uint2 *>(smem + p.tab_off);     // [KB][32 lanes] B registers
-  float *ftab = reinterpret_cast<float *>(smem + p.ftab_off);   // [KB] 2^(E_b - E)
+  float *fwt = reinterpret_cast<float *>(smem + p.ftab_off);    // [warp][block of its K slice][t] 2^(E_b - E + 16t)
   int *ebt = reinterpret_cast<int *>(smem + p.eb_off);          // [KB] E_b
   float *red = reinterpret_cast<float *>(smem + p.red_off);     // [stage][kSlices][16 TPS rows]
   uint8_t *stage_mem = smem + p.stage_off;
@@ -1337,9 +1344,9 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   const int units = p.KB * 8;  // (block, t, half): four activations each
   // One pass over x: block exponents (the eight units of a block are eight
   // lanes of a warp: a shuffle max), then the unit's digits, transposed into B
-  // registers (lane (k, t) of block b holds digit k of activations 8t..8t+3 in
-  // word 0 and 8t+4..8t+7 in word 1); the vector's largest exponent per warp,
-  // then over the warps (shared-memory atomics on one address would serialise).
+  // registers (lane (k, t) of block b holds digit k of activations 4t..4t+3 in
+  // word 0 and 16+4t..16+4t+3 in word 1); the vector's largest exponent per
+  // warp, then over the warps (shared-memory atomics on one address would serialise).
   int wmaxE = 1;
   for (int base = (warp - 1) * 32; base < units; base += 32 * kDigitWarps) {  // warp-uniform: it shuffles
     const int u = base + lane;
@@ -1353,7 +1360,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     const int Eb = max(static_cast<int>(m >> 23), 1);
     wmaxE = max(wmaxE, Eb);
     if (u < units) {
-      const int b = u >> 3, t = (u >> 1) & 3, h = u & 1;
+      const int b = u >> 3, t = u & 3, h = (u >> 2) & 1;  // activations 4(u & 7) .. 4(u & 7) + 3
       if ((u & 7) == 0) ebt[b] = Eb;
       const uint64_t bias = 0x8080808080808080ull;
       const uint64_t d0 = (static_cast<uint64_t>(x_fixed(v.x, Eb)) + bias) ^ bias;
@@ -1380,17 +1387,21 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   int Emax = 1;
   for (int w = 0; w < kDigitWarps; ++w) Emax = max(Emax, wmax[w]);
   if (ctid == 0) *emax = Emax;  // read by the producer after the consumers release their first stage
-  for (int b = ctid; b < p.KB; b += 32 * kDigitWarps) {
-    const int eb = ebt[b] - Emax;
-    ftab[b] = eb >= -126 ? __int_as_float((127 + eb) << 23) : 0.f;
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(32 * kDigitWarps) : "memory");
 
   const int cw = warp - 1;
   const int tl = cw % TPS, ks = cw / TPS;  // this warp's tile of the stage and K slice
   const int kb0 = ks * p.KB / kSlices, kb1 = (ks + 1) * p.KB / kSlices;
   const int g = lane >> 2, t = lane & 3;
-  const float w0 = __int_as_float((127 + 16 * t) << 23), w1 = __int_as_float((127 + 16 * t + 8) << 23);
+  // The warp's own block factors 2^(E_b - E) 2^(16t) (zero for blocks more
+  // than 2^126 below the vector's largest), per block of its K slice and
+  // digit-lane pair t; no CTA barrier needed, the warp reads only these.
+  float *fw = fwt + cw * (kMaxSliceBlocks * 4);
+  for (int i = lane; i < 4 * (kb1 - kb0); i += 32) {
+    const int eb = ebt[kb0 + (i >> 2)] - Emax;
+    fw[i] = eb >= -126 ? __int_as_float((127 + eb) << 23) * __int_as_float((127 + 16 * (i & 3)) << 23) : 0.f;
+  }
+  __syncwarp();
+
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % S;
     if (!mbar_wait(&full[s], static_cast<uint32_t>(c / S) & 1u)) {
@@ -1401,31 +1412,59 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     const int64_t r0 = ch.r0;
     const int rows = ch.rows;
     const uint32_t base = smem_u32(stage_mem) + s * p.stage_bytes + static_cast<uint32_t>((r0 * p.row_bytes) & 15);
-    const int ra = tl * 16 + g, rb = ra + 8;  // rows of this lane
-    const bool oka = ra < rows, okb = rb < rows;
+    // MMA rows g and g + 8 are the tile's rows 2g and 2g + 1 (bank spread);
+    // rows past the chunk read its last row and are never written out
+    const int ra = tl * 16 + 2 * g, rb = ra + 1;
     const uint32_t pa = base + static_cast<uint32_t>(min(ra, rows - 1) * p.row_bytes);
     const uint32_t pb = base + static_cast<uint32_t>(min(rb, rows - 1) * p.row_bytes);
     float2 acc = make_float2(0.f, 0.f);  // rows ra, rb
-#pragma unroll 4
-    for (int b = kb0; b < kb1; ++b) {
-      // codes 8t..8t+7 of both rows (2-byte aligned) and their block scales
-      const uint32_t ca = pa + 34u * b, cb = pb + 34u * b;
-      const uint32_t ma = (ca + 2u + 8u * t) & 2u, mb = (cb + 2u + 8u * t) & 2u;
-      const uint32_t xa = ca + 2u + 8u * t - ma, xb = cb + 2u + 8u * t - mb;
-      const uint32_t a0 = lds_u32(xa), a1w = lds_u32(xa + 4), a2 = lds_u32(xa + 8);
-      const uint32_t b0w = lds_u32(xb), b1w = lds_u32(xb + 4), b2w = lds_u32(xb + 8);
-      const uint32_t A0 = oka ? __funnelshift_r(a0, a1w, ma << 3) : 0u, A2 = oka ? __funnelshift_r(a1w, a2, ma << 3) : 0u;
-      const uint32_t A1 = okb ? __funnelshift_r(b0w, b1w, mb << 3) : 0u, A3 = okb ? __funnelshift_r(b1w, b2w, mb << 3) : 0u;
+    // Block b of both rows: codes k = 4t..4t+3 (A0, A1) and 16+4t..16+4t+3
+    // (A2, A3). FORM 0: codes word-aligned; 1: codes 2 bytes past a word
+    // (byte permutes of aligned words); 2: alignment known at run time only.
+    auto block = [&](auto form, int b) {
+      constexpr int kForm = decltype(form)::value;
+      const uint32_t ca = pa + 34u * b, cb = pb + 34u * b;  // block starts (scale d)
+      uint32_t A0, A1, A2, A3;
+      if constexpr (kForm == 0) {
+        A0 = lds_u32(ca + 2u + 4u * t);
+        A2 = lds_u32(ca + 18u + 4u * t);
+        A1 = lds_u32(cb + 2u + 4u * t);
+        A3 = lds_u32(cb + 18u + 4u * t);
+      } else if constexpr (kForm == 1) {
+        const uint32_t ea = ca + 4u * t, eb = cb + 4u * t;
+        A0 = __byte_perm(lds_u32(ea), lds_u32(ea + 4u), 0x5432u);
+        A2 = __byte_perm(lds_u32(ea + 16u), lds_u32(ea + 20u), 0x5432u);
+        A1 = __byte_perm(lds_u32(eb), lds_u32(eb + 4u), 0x5432u);
+        A3 = __byte_perm(lds_u32(eb + 16u), lds_u32(eb + 20u), 0x5432u);
+      } else {
+        const uint32_t xa = ca + 2u + 4u * t, xb = cb + 2u + 4u * t;
+        const uint32_t sa = (xa & 3u) << 3, sb = (xb & 3u) << 3, ya = xa & ~3u, yb = xb & ~3u;
+        A0 = __funnelshift_r(lds_u32(ya), lds_u32(ya + 4u), sa);
+        A2 = __funnelshift_r(lds_u32(ya + 16u), lds_u32(ya + 20u), sa);
+        A1 = __funnelshift_r(lds_u32(yb), lds_u32(yb + 4u), sb);
+        A3 = __funnelshift_r(lds_u32(yb + 16u), lds_u32(yb + 20u), sb);
+      }
       const float2 dd = make_float2(half_bits_to_float(lds_u16(ca)), half_bits_to_float(lds_u16(cb)));
       const uint2 B = tab[b * 32 + lane];
       int cc[4];
       imma_16832(cc, A0, A1, A2, A3, B.x, B.y);
-      // this lane's two digits of both rows, then the block scale
-      const float2 lo = make_float2(int_exact_f(cc[0]), int_exact_f(cc[2]));
-      const float2 hi = make_float2(int_exact_f(cc[1]), int_exact_f(cc[3]));
-      const float2 v = __ffma2_rn(hi, make_float2(w1, w1), __fmul2_rn(lo, make_float2(w0, w0)));
-      const float f = ftab[b];
+      // this lane's digits 2t, 2t+1 of both rows as one exact int32 (< 2^28)
+      const float2 v = make_float2(__int2float_rn(cc[0] + cc[1] * 256), __int2float_rn(cc[2] + cc[3] * 256));
+      const float f = fw[4 * (b - kb0) + t];
       acc = __ffma2_rn(v, __fmul2_rn(dd, make_float2(f, f)), acc);
+    };
+    if (p.rows_aligned) {  // rows are whole words: odd blocks aligned, even ones 2 bytes past
+      int b = kb0;
+      if (b < kb1 && (b & 1)) block(std::integral_constant<int, 0>{}, b++);
+#pragma unroll 2
+      for (; b + 1 < kb1; b += 2) {
+        block(std::integral_constant<int, 1>{}, b);
+        block(std::integral_constant<int, 0>{}, b + 1);
+      }
+      if (b < kb1) block(std::integral_constant<int, 1>{}, b);
+    } else {
+#pragma unroll 4
+      for (int b = kb0; b < kb1; ++b) block(std::integral_constant<int, 2>{}, b);
     }
     // the four digit lanes of each row
     acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
@@ -1843,7 +1882,8 @@ bool try_launch_digits(const DevInfo &dev, int nproj, const int64_t *N, const vo
   p.stage_bytes = align_up(16ll * tps * p.row_bytes + 64, 128);
   p.tab_off = 1024;
   p.ftab_off = p.tab_off + 256 * KB;
-  p.eb_off = p.ftab_off + 4 * KB;
+  p.eb_off = p.ftab_off + kDigitWarps * kMaxSliceBlocks * 4 * 4;
+  p.rows_aligned = (p.row_bytes % 4) == 0 ? 1 : 0;
   p.red_off = align_up(p.eb_off + 4ll * KB, 16);
   p.stage_off = align_up(p.red_off + 4ll * kMaxStages * 16 * kDigitWarps, 128);  // K-slice partials
   constexpr int kBudget = 113 * 1024;  // two CTAs per SM
