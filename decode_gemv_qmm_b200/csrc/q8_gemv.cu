@@ -1156,10 +1156,12 @@ __global__ void __launch_bounds__(256, 2) q8_gemv_mma_kernel(const __grid_consta
 //  * C column k = sum_j q_j digit_k(x_j): exact int32 (|C| < 2^20). Thread
 //    (g, t) holds digits 2t, 2t+1 of its two rows; C_2t + 256 C_2t+1 is an
 //    exact int32 (< 2^28), converted once and scaled by d * 2^(E_b - E + 16t)
-//    in fp32 (E the largest E_b of the vector); the four digit lanes are
-//    summed at the end and the row total is scaled by 2^(E - 188). Apart from
-//    fp32 rounding the activation representation is exact for every element
-//    within 2^38 of its block maximum.
+//    in fp32 (E the largest E_b of the warp's K slice); the four digit lanes
+//    are summed, and the producer scales each slice's partial by 2^(E - 188)
+//    and adds the slices in order. Apart from fp32 rounding the activation
+//    representation is exact for every element within 2^38 of its block
+//    maximum. Each K slice's activations are converted by the warps that use
+//    them (a named barrier per slice, no CTA-wide barrier).
 //  * Shared-memory layout: a stage is a verbatim copy of consecutive rows
 //    (34-byte blocks). MMA rows g and g + 8 of a tile are the tile's rows 2g
 //    and 2g + 1: with the 952-byte rows of K = 896 the eight rows 2g start
@@ -1197,6 +1199,7 @@ struct alignas(64) DParams {
 
 constexpr int kDigitWarps = 8;
 constexpr int kMaxSliceBlocks = 16;  // blocks of one K slice: ceil(64 / 4) at K <= 2048
+constexpr int kTabStride = 36;       // uint2 per block of B registers: 32 lanes + pad (conflict-free stores)
 
 __device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                            uint32_t b0, uint32_t b1) {
@@ -1227,9 +1230,9 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   uint8_t *smem = smem_raw;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *empty = full + kMaxStages;
-  int *emax = reinterpret_cast<int *>(empty + kMaxStages);
-  int *wmax = emax + 2;  // [kDigitWarps]: each consumer warp's largest block exponent
-  uint2 *tab = reinterpret_cast<uint2 *>(smem + p.tab_off);     // [KB][32 lanes] B registers
+  int *ewt = reinterpret_cast<int *>(empty + kMaxStages);  // [K slice] its largest block exponent
+  int *ewp = ewt + 8;                                       // [consumer warp] the same over its units
+  uint2 *tab = reinterpret_cast<uint2 *>(smem + p.tab_off);     // [KB][kTabStride]: 32 lanes' B registers + pad
   float *fwt = reinterpret_cast<float *>(smem + p.ftab_off);    // [warp][block of its K slice][t] 2^(E_b - E + 16t)
   int *ebt = reinterpret_cast<int *>(smem + p.eb_off);          // [KB] E_b
   float *red = reinterpret_cast<float *>(smem + p.red_off);     // [stage][kSlices][16 TPS rows]
@@ -1272,7 +1275,6 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kDigitWarps);
     }
-    *emax = 1;
     fence_mbar_init();
   }
   for (int b = tid; b < p.KB; b += blockDim.x) ebt[b] = 1;
@@ -1304,31 +1306,45 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
       if (!p.prefetch_before_wait) pdl_wait();
       for (int c = 0; c < prologue; ++c) issue(c);
     }
+    Chunk ch = nchunks > 0 ? chunk(0) : Chunk{0, 0, 0};
     pdl_wait();
     bool ok = true;
     int issued = prologue;
+    float f1[kSlices], f2[kSlices];  // 2^(E_slice - 188) in two exact steps, per K slice
+    int s = 0;
+    uint32_t ph = 0;
     for (int c = 0; c < nchunks && ok; ++c) {
-      ok = mbar_wait(&empty[c % S], static_cast<uint32_t>(c / S) & 1u);
+      ok = mbar_wait(&empty[s], ph);
       if (!ok) break;
-      // rows of chunk c: sum the K slices in order, scale by 2^(E - 188) (two exact steps)
-      const int s = c % S;
-      const Chunk ch = chunk(c);
+      if (c == 0) {  // the slice exponents were written before the consumers' first release
+#pragma unroll
+        for (int k = 0; k < kSlices; ++k) {
+          const int e = ewt[k] - 188, e1 = max(e, -120);
+          f1[k] = __int_as_float((127 + e1) << 23);
+          f2[k] = __int_as_float((127 + e - e1) << 23);
+        }
+      }
+      // rows of chunk c: each K slice's partial at its own scale, added in slice order
       const int64_t r0 = ch.r0;
       const int rows = ch.rows;
       float *Y = MULTI ? p.Yp[ch.proj] : p.Yp[0];
-      const int e = *emax - 188, e1 = max(e, -120);
-      const float f1 = __int_as_float((127 + e1) << 23), f2 = __int_as_float((127 + e - e1) << 23);
       const float *rb = red + s * kSlices * kRows;
       for (int r = lane; r < rows; r += 32) {
-        float v = rb[r];
-        for (int k = 1; k < kSlices; ++k) v += rb[k * kRows + r];
-        Y[r0 + r] = (v * f1) * f2;
+        float v = (rb[r] * f1[0]) * f2[0];
+#pragma unroll
+        for (int k = 1; k < kSlices; ++k) v += (rb[k * kRows + r] * f1[k]) * f2[k];
+        Y[r0 + r] = v;
       }
       __syncwarp();
       if (lane == 0 && issued < nchunks) {
         issue(issued);
         ++issued;
       }
+      if (++s == S) {
+        s = 0;
+        ph ^= 1u;
+      }
+      if (c + 1 < nchunks) ch = chunk(c + 1);
     }
     if (!ok && lane == 0) {  // error path: record, then drain copies still in flight
       atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
@@ -1339,19 +1355,23 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   }
 
   // -------------------------------------------------------------- consumers
+  const int cw = warp - 1;
+  const int tl = cw % TPS, ks = cw / TPS;  // this warp's tile of the stage and K slice
+  const int kb0 = ks * p.KB / kSlices, kb1 = (ks + 1) * p.KB / kSlices;
+  const int g = lane >> 2, t = lane & 3;
+  Chunk ch = nchunks > 0 ? chunk(0) : Chunk{0, 0, 0};
   pdl_wait();
-  const int ctid = tid - 32;  // 0 .. 255
-  const int units = p.KB * 8;  // (block, t, half): four activations each
-  // One pass over x: block exponents (the eight units of a block are eight
-  // lanes of a warp: a shuffle max), then the unit's digits, transposed into B
-  // registers (lane (k, t) of block b holds digit k of activations 4t..4t+3 in
-  // word 0 and 16+4t..16+4t+3 in word 1); the vector's largest exponent per
-  // warp, then over the warps (shared-memory atomics on one address would serialise).
+  // One pass over this K slice's activations, shared by its TPS warps: block
+  // exponents (the eight units of a block are eight lanes of a warp: a
+  // shuffle max), then each unit's digits, transposed into B registers (lane
+  // (k, t) of block b holds digit k of activations 4t..4t+3 in word 0 and
+  // 16+4t..16+4t+3 in word 1); the slice's largest block exponent E_w.
   int wmaxE = 1;
-  for (int base = (warp - 1) * 32; base < units; base += 32 * kDigitWarps) {  // warp-uniform: it shuffles
+  const int u_end = 8 * kb1;
+  for (int base = 8 * kb0 + 32 * tl; base < u_end; base += 32 * TPS) {  // warp-uniform: it shuffles
     const int u = base + lane;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (u < units) v = __ldg(reinterpret_cast<const float4 *>(p.X) + u);
+    if (u < u_end) v = __ldg(reinterpret_cast<const float4 *>(p.X) + u);
     uint32_t m = max(max(__float_as_uint(v.x) & 0x7fffffffu, __float_as_uint(v.y) & 0x7fffffffu),
                      max(__float_as_uint(v.z) & 0x7fffffffu, __float_as_uint(v.w) & 0x7fffffffu));
     m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
@@ -1359,7 +1379,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
     const int Eb = max(static_cast<int>(m >> 23), 1);
     wmaxE = max(wmaxE, Eb);
-    if (u < units) {
+    if (u < u_end) {
       const int b = u >> 3, t = u & 3, h = (u >> 2) & 1;  // activations 4(u & 7) .. 4(u & 7) + 3
       if ((u & 7) == 0) ebt[b] = Eb;
       const uint64_t bias = 0x8080808080808080ull;
@@ -1367,7 +1387,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
       const uint64_t d1 = (static_cast<uint64_t>(x_fixed(v.y, Eb)) + bias) ^ bias;
       const uint64_t d2 = (static_cast<uint64_t>(x_fixed(v.z, Eb)) + bias) ^ bias;
       const uint64_t d3 = (static_cast<uint64_t>(x_fixed(v.w, Eb)) + bias) ^ bias;
-      uint32_t *tb = reinterpret_cast<uint32_t *>(tab + b * 32);
+      uint32_t *tb = reinterpret_cast<uint32_t *>(tab + b * kTabStride);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {  // digits 0..3, then 4..7
         const uint32_t w0 = static_cast<uint32_t>(d0 >> (32 * half)), w1 = static_cast<uint32_t>(d1 >> (32 * half));
@@ -1382,33 +1402,36 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     }
   }
   wmaxE = __reduce_max_sync(0xffffffffu, wmaxE);
-  if (lane == 0) wmax[warp - 1] = wmaxE;
-  asm volatile("bar.sync 1, %0;" ::"n"(32 * kDigitWarps) : "memory");
-  int Emax = 1;
-  for (int w = 0; w < kDigitWarps; ++w) Emax = max(Emax, wmax[w]);
-  if (ctid == 0) *emax = Emax;  // read by the producer after the consumers release their first stage
-
-  const int cw = warp - 1;
-  const int tl = cw % TPS, ks = cw / TPS;  // this warp's tile of the stage and K slice
-  const int kb0 = ks * p.KB / kSlices, kb1 = (ks + 1) * p.KB / kSlices;
-  const int g = lane >> 2, t = lane & 3;
-  // The warp's own block factors 2^(E_b - E) 2^(16t) (zero for blocks more
-  // than 2^126 below the vector's largest), per block of its K slice and
-  // digit-lane pair t; no CTA barrier needed, the warp reads only these.
+  if (lane == 0) ewp[cw] = wmaxE;
+  if constexpr (TPS == 2) {  // the slice's two warps: named barrier 2 + ks (immediate ids)
+    switch (ks) {
+      case 0: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+      case 1: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+      case 2: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+      default: asm volatile("bar.sync 5, 64;" ::: "memory"); break;
+    }
+  } else {
+    __syncwarp();
+  }
+  int Ew = ewp[ks * TPS];
+  if constexpr (TPS == 2) Ew = max(Ew, ewp[ks * TPS + 1]);
+  if (tl == 0 && lane == 0) ewt[ks] = Ew;  // read by the producer after the first release
+  // The warp's block factors 2^(E_b - E_w) 2^(16t) (zero for blocks more than
+  // 2^126 below the slice's largest), per block of its slice and digit pair t.
   float *fw = fwt + cw * (kMaxSliceBlocks * 4);
   for (int i = lane; i < 4 * (kb1 - kb0); i += 32) {
-    const int eb = ebt[kb0 + (i >> 2)] - Emax;
+    const int eb = ebt[kb0 + (i >> 2)] - Ew;
     fw[i] = eb >= -126 ? __int_as_float((127 + eb) << 23) * __int_as_float((127 + 16 * (i & 3)) << 23) : 0.f;
   }
   __syncwarp();
 
+  int s = 0;
+  uint32_t ph = 0;
   for (int c = 0; c < nchunks; ++c) {
-    const int s = c % S;
-    if (!mbar_wait(&full[s], static_cast<uint32_t>(c / S) & 1u)) {
+    if (!mbar_wait(&full[s], ph)) {
       if (lane == 0) atomicOr(&g_q8_gemv_status, kDevTimeoutFull);
       return;  // the producer times out on this warp's missing arrival and drains
     }
-    const Chunk ch = chunk(c);
     const int64_t r0 = ch.r0;
     const int rows = ch.rows;
     const uint32_t base = smem_u32(stage_mem) + s * p.stage_bytes + static_cast<uint32_t>((r0 * p.row_bytes) & 15);
@@ -1445,7 +1468,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
         A3 = __funnelshift_r(lds_u32(yb + 16u), lds_u32(yb + 20u), sb);
       }
       const float2 dd = make_float2(half_bits_to_float(lds_u16(ca)), half_bits_to_float(lds_u16(cb)));
-      const uint2 B = tab[b * 32 + lane];
+      const uint2 B = tab[b * kTabStride + lane];
       int cc[4];
       imma_16832(cc, A0, A1, A2, A3, B.x, B.y);
       // this lane's digits 2t, 2t+1 of both rows as one exact int32 (< 2^28)
@@ -1478,6 +1501,11 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == S) {
+      s = 0;
+      ph ^= 1u;
+    }
+    if (c + 1 < nchunks) ch = chunk(c + 1);
   }
 }
 
@@ -1881,7 +1909,7 @@ bool try_launch_digits(const DevInfo &dev, int nproj, const int64_t *N, const vo
   p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
   p.stage_bytes = align_up(16ll * tps * p.row_bytes + 64, 128);
   p.tab_off = 1024;
-  p.ftab_off = p.tab_off + 256 * KB;
+  p.ftab_off = p.tab_off + 8 * kTabStride * KB;
   p.eb_off = p.ftab_off + kDigitWarps * kMaxSliceBlocks * 4 * 4;
   p.rows_aligned = (p.row_bytes % 4) == 0 ? 1 : 0;
   p.red_off = align_up(p.eb_off + 4ll * KB, 16);
