@@ -704,6 +704,7 @@ def run_case(spec: str, reps: int, seed: int):
     numbers it prints are not benchmark values.
 
     gemv:N:K            qmm_q8_gemv, M=1
+    multi:N1,N2,..:K    qmm_q8_gemv_multi, M=1 (projections of one activation vector)
     q8q8:N:K            qmm_quantize_act_q8 + qmm_q8q8_gemv, M=1
     q8q8f:N:K           qmm_q8q8_gemv_fused, M=1
     q4gemv:M:N:K        qmm_q4_gemv
@@ -725,6 +726,12 @@ def run_case(spec: str, reps: int, seed: int):
         x = torch.from_numpy(syn.act_f32(g, 1, k)).cuda()
         y = torch.empty(1, n, device="cuda")
         launches.append(lambda: qmm.qmm_q8_gemv(W, x, n, y))
+    elif parts[0] == "multi":
+        ns, k = [int(v) for v in parts[1].split(",")], int(parts[2])
+        Ws = [torch.from_numpy(syn.q8_0_weights(g, n, k)[0]).cuda() for n in ns]
+        x = torch.from_numpy(syn.act_f32(g, 1, k)).cuda()
+        ys = [torch.empty(1, n, device="cuda") for n in ns]
+        launches.append(lambda: qmm.qmm_q8_gemv_multi(Ws, x, ns, ys))
     elif parts[0] == "q8q8":
         n, k = int(parts[1]), int(parts[2])
         W = torch.from_numpy(syn.q8_0_weights(g, n, k)[0]).cuda()

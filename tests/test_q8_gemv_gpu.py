@@ -225,3 +225,50 @@ def test_single_row_integer_streaming_shapes(n, k):
     # M = 1 with many rows per CTA and K <= 2048: raw codes x 8-digit activations on the
     # integer tensor cores
     check(1, n, k, seed=61 + n + k)
+
+
+def _slice_scaled_inputs(g, n, k, big_first):
+    """Weights whose codes are zero over the first quarter of K, and activations of
+    ~1e30 there and ~1e-30 elsewhere (or the reverse scales with the zero codes
+    over the last three quarters): the output then comes from the tiny-magnitude
+    part alone while the vector's largest block exponent sits in the other part."""
+    W, _, _ = syn.q8_0_weights(g, n, k)
+    kb = k // 32
+    rows = W.reshape(n, kb, 34)
+    x = syn.act_f32(g, 1, k).astype(np.float64)
+    q = k // 4
+    if big_first:
+        rows[:, :kb // 4, 2:] = 0           # codes of the huge quarter
+        x[0, :q] *= 1e30
+        x[0, q:] *= 1e-30
+    else:
+        rows[:, kb // 4:, 2:] = 0           # codes of the huge three quarters
+        x[0, :q] *= 1e-30
+        x[0, q:] *= 1e30
+    return rows.reshape(-1).copy(), x.astype(np.float32)
+
+
+@pytest.mark.parametrize("big_first", [True, False], ids=["huge_first_quarter", "huge_last_quarters"])
+@pytest.mark.parametrize("n,k", [(12000, 896), (9472, 2048)])
+def test_integer_kernel_exponent_range_across_k(n, k, big_first):
+    # The integer tensor-core kernel scales each K slice by its own largest block
+    # exponent: a slice of ~1e30 activations times zero codes must not wipe out the
+    # ~1e-30 contributions of the other slices (2^-200 below the vector's maximum).
+    g = syn.rng(71 + n + k + big_first)
+    W, x = _slice_scaled_inputs(g, n, k, big_first)
+    y = run(W, x, n)
+    ref, S = oracle.gemv(syn.Q8_0, W, x, n)
+    assert np.all(np.abs(ref) > 0)
+    assert_within(y, ref, S, TOL_FP32, f"N={n} K={k} big_first={big_first}")
+
+
+def test_projection_table_exponent_range_across_k():
+    g = syn.rng(75)
+    k, ns = 896, [4864, 4864]
+    W0, x = _slice_scaled_inputs(g, ns[0], k, True)
+    W1 = W0.reshape(ns[0], -1)[::-1].reshape(-1).copy()   # same zeroed codes, other rows order
+    Ys = qmm.qmm_q8_gemv_multi([dev(W0), dev(W1)], dev(x), ns)
+    torch.cuda.synchronize()
+    for W, Y, n in zip((W0, W1), Ys, ns):
+        ref, S = oracle.gemv(syn.Q8_0, W, x, n)
+        assert_within(host(Y), ref, S, TOL_FP32, "projection table, huge first quarter")
