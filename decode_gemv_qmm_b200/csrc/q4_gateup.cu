@@ -557,6 +557,10 @@ qmm_status launch_q4_gateup(const DevInfo &dev, int M, int64_t N, int K, const v
 
 qmm_status launch_q4_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
                           cudaStream_t stream, uint32_t flags) {
+  // one token: raw codes on the integer tensor cores (a fraction of this
+  // kernel's per-weight work, which serves eight tokens)
+  qmm_status st;
+  if (M == 1 && launch_q4_gemv_digits(dev, N, K, W, X, Y, stream, flags, &st)) return st;
   const void *Wp[1] = {W};
   return launch_proj(dev, M, N, K, Wp, 1, X, Y, stream, flags);
 }

@@ -1193,12 +1193,16 @@ struct alignas(64) DParams {
   int stages;
   int stage_bytes;
   int tab_off, ftab_off, eb_off, red_off, stage_off;  // shared-memory offsets
-  int rows_aligned;  // row_bytes % 4 == 0 (even KB): parity-specialised code loads
+  int rows_aligned;  // block starts are even and rows whole words: parity-specialised code loads
+  int padded;        // rows copied in groups of 2^lg_sub rows, group g at g * sub_pitch
+  int lg_sub, sub_pitch;
+  uint8_t rowmap[16];  // MMA row m of a 16-row tile -> row of the tile in memory order
+  int wexp;          // power of two of the code scale (Q4_0 codes enter as 16 (q - 8): -4)
   int prefetch_before_wait;
 };
 
-constexpr int kDigitWarps = 8;
-constexpr int kMaxSliceBlocks = 16;  // blocks of one K slice: ceil(64 / 4) at K <= 2048
+constexpr int kDigitWarps = 8;  // consumer warps of a CTA when two CTAs share an SM (16 with one)
+constexpr int kMaxSliceBlocks = 32;  // blocks of one K slice (the launcher checks the bound)
 constexpr int kTabStride = 36;       // uint2 per block of B registers: 32 lanes + pad (conflict-free stores)
 
 __device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -1209,36 +1213,43 @@ __device__ __forceinline__ void imma_16832(int (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
-// x * 2^(38 - E_b) as a signed 64-bit integer (x = M 2^(E - 150)).
-__device__ __forceinline__ long long x_fixed(float x, int Eb) {
-  const uint32_t b = __float_as_uint(x);
-  int E = static_cast<int>((b >> 23) & 0xffu);
-  uint64_t M = b & 0x7fffffu;
-  if (E == 0) E = 1;
-  else M |= 0x800000u;
-  const int s = E - Eb + 38;
-  uint64_t v;
-  if (s >= 0) v = M << s;
-  else if (s > -26) v = (M + (uint64_t(1) << (-s - 1))) >> (-s);
-  else v = 0;
-  return (b >> 31) ? -static_cast<long long>(v) : static_cast<long long>(v);
+// The eight balanced base-256 digits of x_int = x 2^(188 - E_b) (x = M 2^(E - 150):
+// exact for elements within 2^38 of the block maximum, rounded to nearest below
+// that), as the bytes of (x_int + 0x8080..80) xor 0x8080..80. fa fb = 2^(156 - E_b),
+// two normal powers of two. In fp32, every step exact: |x| fa fb = |x_int| / 2^32
+// (< 2^30), its integer part is the high word and the fraction times 2^32 the low
+// word of |x_int|; the sign is applied in two's complement with the bias added.
+__device__ __forceinline__ uint64_t x_digits(float x, float fa, float fb) {
+  const float xa = (fabsf(x) * fa) * fb;
+  const uint32_t hw = __float2uint_rz(xa);
+  const uint32_t lw = __float2uint_rn((xa - truncf(xa)) * 4294967296.0f);
+  const uint64_t mag = (static_cast<uint64_t>(hw) << 32) | lw;
+  const uint64_t neg = static_cast<uint64_t>(static_cast<int64_t>(static_cast<int32_t>(__float_as_uint(x)) >> 31));
+  const uint64_t bias = 0x8080808080808080ull;
+  return (((mag ^ neg) + (neg & 1u)) + bias) ^ bias;
 }
 
-template <int TPS, bool MULTI>
-__global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(const __grid_constant__ DParams p) {
+// WT: QMM_Q8_0 (rows verbatim in shared memory, MMA rows interleaved) or
+// QMM_Q4_0 (one GEMV; rows copied in groups placed so that the eight rows of
+// an MMA half start on distinct banks; codes widened to 16 (q - 8), the factor
+// 16 undone by wexp).
+// NW: consumer warps (8 when two CTAs share an SM, 16 when one CTA has it).
+template <int TPS, bool MULTI, int WT, int NW>
+__global__ void __launch_bounds__((NW + 1) * 32) q8_gemv_digits_kernel(const __grid_constant__ DParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *empty = full + kMaxStages;
   int *ewt = reinterpret_cast<int *>(empty + kMaxStages);  // [K slice] its largest block exponent
-  int *ewp = ewt + 8;                                       // [consumer warp] the same over its units
+  int *ewp = ewt + 16;                                      // [consumer warp] the same over its units
   uint2 *tab = reinterpret_cast<uint2 *>(smem + p.tab_off);     // [KB][kTabStride]: 32 lanes' B registers + pad
   float *fwt = reinterpret_cast<float *>(smem + p.ftab_off);    // [warp][block of its K slice][t] 2^(E_b - E + 16t)
   int *ebt = reinterpret_cast<int *>(smem + p.eb_off);          // [KB] E_b
   float *red = reinterpret_cast<float *>(smem + p.red_off);     // [stage][kSlices][16 TPS rows]
   uint8_t *stage_mem = smem + p.stage_off;
   constexpr int kRows = 16 * TPS;
-  constexpr int kSlices = kDigitWarps / TPS;
+  constexpr int kSlices = NW / TPS;
+  constexpr uint32_t kBB = WT == QMM_Q8_0 ? 34u : 18u;  // bytes per block
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // whole chunks per CTA: a chunk costs the same however few of its rows are
@@ -1273,7 +1284,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kDigitWarps);
+      mbar_init(&empty[s], NW);
     }
     fence_mbar_init();
   }
@@ -1287,6 +1298,15 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
       const int s = c % S;
       const Chunk ch = chunk(c);
       const uint8_t *W = MULTI ? p.Wp[ch.proj] : p.Wp[0];
+      if (p.padded) {  // rows are 16-byte multiples: one copy per group of rows
+        uint8_t *dst = stage_mem + static_cast<int64_t>(s) * p.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(p.row_bytes * ch.rows));
+        const int gr = 1 << p.lg_sub;
+        for (int r = 0, gi = 0; r < ch.rows; r += gr, ++gi)
+          bulk_g2s(dst + gi * p.sub_pitch, W + (ch.r0 + r) * p.row_bytes,
+                   static_cast<uint32_t>(p.row_bytes * min(gr, ch.rows - r)), &full[s], policy);
+        return;
+      }
       const int64_t b0 = ch.r0 * p.row_bytes, b1 = (ch.r0 + ch.rows) * p.row_bytes;
       const int64_t a0 = b0 & ~int64_t(15);
       int64_t a1 = (b1 + 15) & ~int64_t(15);
@@ -1319,7 +1339,7 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
       if (c == 0) {  // the slice exponents were written before the consumers' first release
 #pragma unroll
         for (int k = 0; k < kSlices; ++k) {
-          const int e = ewt[k] - 188, e1 = max(e, -120);
+          const int e = ewt[k] - 188 + p.wexp, e1 = max(e, -120);
           f1[k] = __int_as_float((127 + e1) << 23);
           f2[k] = __int_as_float((127 + e - e1) << 23);
         }
@@ -1368,10 +1388,14 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   // 16+4t..16+4t+3 in word 1); the slice's largest block exponent E_w.
   int wmaxE = 1;
   const int u_end = 8 * kb1;
+  const float4 *X4 = reinterpret_cast<const float4 *>(p.X);
+  float4 vn = make_float4(0.f, 0.f, 0.f, 0.f);  // the next pass's activations, loaded a pass ahead
+  if (8 * kb0 + 32 * tl + lane < u_end) vn = __ldg(X4 + 8 * kb0 + 32 * tl + lane);
   for (int base = 8 * kb0 + 32 * tl; base < u_end; base += 32 * TPS) {  // warp-uniform: it shuffles
     const int u = base + lane;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (u < u_end) v = __ldg(reinterpret_cast<const float4 *>(p.X) + u);
+    const float4 v = vn;
+    vn = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (u + 32 * TPS < u_end) vn = __ldg(X4 + u + 32 * TPS);
     uint32_t m = max(max(__float_as_uint(v.x) & 0x7fffffffu, __float_as_uint(v.y) & 0x7fffffffu),
                      max(__float_as_uint(v.z) & 0x7fffffffu, __float_as_uint(v.w) & 0x7fffffffu));
     m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
@@ -1382,11 +1406,10 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     if (u < u_end) {
       const int b = u >> 3, t = u & 3, h = (u >> 2) & 1;  // activations 4(u & 7) .. 4(u & 7) + 3
       if ((u & 7) == 0) ebt[b] = Eb;
-      const uint64_t bias = 0x8080808080808080ull;
-      const uint64_t d0 = (static_cast<uint64_t>(x_fixed(v.x, Eb)) + bias) ^ bias;
-      const uint64_t d1 = (static_cast<uint64_t>(x_fixed(v.y, Eb)) + bias) ^ bias;
-      const uint64_t d2 = (static_cast<uint64_t>(x_fixed(v.z, Eb)) + bias) ^ bias;
-      const uint64_t d3 = (static_cast<uint64_t>(x_fixed(v.w, Eb)) + bias) ^ bias;
+      const int ke = 156 - Eb, ka = min(ke, 127);
+      const float fa = __int_as_float((127 + ka) << 23), fb = __int_as_float((127 + ke - ka) << 23);
+      const uint64_t d0 = x_digits(v.x, fa, fb), d1 = x_digits(v.y, fa, fb);
+      const uint64_t d2 = x_digits(v.z, fa, fb), d3 = x_digits(v.w, fa, fb);
       uint32_t *tb = reinterpret_cast<uint32_t *>(tab + b * kTabStride);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {  // digits 0..3, then 4..7
@@ -1408,7 +1431,11 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
       case 0: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
       case 1: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
       case 2: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
-      default: asm volatile("bar.sync 5, 64;" ::: "memory"); break;
+      case 3: asm volatile("bar.sync 5, 64;" ::: "memory"); break;
+      case 4: asm volatile("bar.sync 6, 64;" ::: "memory"); break;
+      case 5: asm volatile("bar.sync 7, 64;" ::: "memory"); break;
+      case 6: asm volatile("bar.sync 8, 64;" ::: "memory"); break;
+      default: asm volatile("bar.sync 9, 64;" ::: "memory"); break;
     }
   } else {
     __syncwarp();
@@ -1425,6 +1452,11 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
   }
   __syncwarp();
 
+  // MMA rows g and g + 8 of tile tl. Q8_0 (verbatim rows of 952 bytes): the
+  // tile's rows 2g and 2g + 1; Q4_0 (grouped rows): rowmap[g], rowmap[g + 8],
+  // chosen on the host so that each MMA half's eight rows start on distinct banks.
+  const int ra = WT == QMM_Q8_0 ? tl * 16 + 2 * g : tl * 16 + p.rowmap[g];
+  const int rb = WT == QMM_Q8_0 ? ra + 1 : tl * 16 + p.rowmap[g + 8];
   int s = 0;
   uint32_t ph = 0;
   for (int c = 0; c < nchunks; ++c) {
@@ -1434,21 +1466,43 @@ __global__ void __launch_bounds__((kDigitWarps + 1) * 32) q8_gemv_digits_kernel(
     }
     const int64_t r0 = ch.r0;
     const int rows = ch.rows;
-    const uint32_t base = smem_u32(stage_mem) + s * p.stage_bytes + static_cast<uint32_t>((r0 * p.row_bytes) & 15);
-    // MMA rows g and g + 8 are the tile's rows 2g and 2g + 1 (bank spread);
+    const uint32_t base = smem_u32(stage_mem) + s * p.stage_bytes +
+                          (p.padded ? 0u : static_cast<uint32_t>((r0 * p.row_bytes) & 15));
     // rows past the chunk read its last row and are never written out
-    const int ra = tl * 16 + 2 * g, rb = ra + 1;
-    const uint32_t pa = base + static_cast<uint32_t>(min(ra, rows - 1) * p.row_bytes);
-    const uint32_t pb = base + static_cast<uint32_t>(min(rb, rows - 1) * p.row_bytes);
+    auto row_off = [&](int r) -> uint32_t {
+      r = min(r, rows - 1);
+      if constexpr (WT == QMM_Q8_0) return static_cast<uint32_t>(r * p.row_bytes);
+      else return static_cast<uint32_t>((r >> p.lg_sub) * p.sub_pitch + (r & ((1 << p.lg_sub) - 1)) * p.row_bytes);
+    };
+    const uint32_t pa = base + row_off(ra), pb = base + row_off(rb);
     float2 acc = make_float2(0.f, 0.f);  // rows ra, rb
     // Block b of both rows: codes k = 4t..4t+3 (A0, A1) and 16+4t..16+4t+3
     // (A2, A3). FORM 0: codes word-aligned; 1: codes 2 bytes past a word
     // (byte permutes of aligned words); 2: alignment known at run time only.
     auto block = [&](auto form, int b) {
       constexpr int kForm = decltype(form)::value;
-      const uint32_t ca = pa + 34u * b, cb = pb + 34u * b;  // block starts (scale d)
+      const uint32_t ca = pa + kBB * b, cb = pb + kBB * b;  // block starts (scale d)
       uint32_t A0, A1, A2, A3;
-      if constexpr (kForm == 0) {
+      if constexpr (WT == QMM_Q4_0) {
+        // bytes 4t..4t+3 of the packed codes: low nibbles are elements 4t..4t+3,
+        // high nibbles 16+4t..16+4t+3; each becomes the int8 16 (q - 8)
+        uint32_t wa, wb;
+        if constexpr (kForm == 0) {
+          wa = lds_u32(ca + 2u + 4u * t);
+          wb = lds_u32(cb + 2u + 4u * t);
+        } else if constexpr (kForm == 1) {
+          wa = __byte_perm(lds_u32(ca + 4u * t), lds_u32(ca + 4u * t + 4u), 0x5432u);
+          wb = __byte_perm(lds_u32(cb + 4u * t), lds_u32(cb + 4u * t + 4u), 0x5432u);
+        } else {
+          const uint32_t xa = ca + 2u + 4u * t, xb = cb + 2u + 4u * t;
+          wa = __funnelshift_r(lds_u32(xa & ~3u), lds_u32((xa & ~3u) + 4u), (xa & 3u) << 3);
+          wb = __funnelshift_r(lds_u32(xb & ~3u), lds_u32((xb & ~3u) + 4u), (xb & 3u) << 3);
+        }
+        A0 = ((wa << 4) & 0xF0F0F0F0u) ^ 0x80808080u;
+        A2 = (wa & 0xF0F0F0F0u) ^ 0x80808080u;
+        A1 = ((wb << 4) & 0xF0F0F0F0u) ^ 0x80808080u;
+        A3 = (wb & 0xF0F0F0F0u) ^ 0x80808080u;
+      } else if constexpr (kForm == 0) {
         A0 = lds_u32(ca + 2u + 4u * t);
         A2 = lds_u32(ca + 18u + 4u * t);
         A1 = lds_u32(cb + 2u + 4u * t);
@@ -1877,11 +1931,63 @@ bool try_launch_mma(const DevInfo &dev, int64_t N, int K, const void *W, const f
 
 // Integer tensor-core streaming variant for M = 1, K <= 2048 and enough rows
 // for two CTAs per SM (returns false when the shape does not suit it).
+// Row placement in shared memory and the MMA row order. Verbatim rows (Q8_0):
+// one copy per chunk, MMA rows g, g + 8 = tile rows 2g, 2g + 1. Grouped rows
+// (Q4_0, rows of 16-byte multiples): the tile's rows come in copies of 2^lg
+// consecutive rows, copy i at i * sub_pitch; the largest groups (fewest
+// copies: many small bulk copies are slow) and smallest gap for which the
+// tile's rows split into two halves of eight whose start banks (4-word
+// groups) are all distinct; rowmap lists half 0, then half 1. tile_span:
+// shared-memory bytes a 16-row tile takes.
+bool place_rows(DParams &p, int &tile_span) {
+  if (!p.padded) {
+    for (int g = 0; g < 8; ++g) {
+      p.rowmap[g] = static_cast<uint8_t>(2 * g);
+      p.rowmap[g + 8] = static_cast<uint8_t>(2 * g + 1);
+    }
+    tile_span = 16 * static_cast<int>(p.row_bytes);
+    return true;
+  }
+  const int64_t rb = p.row_bytes;
+  for (int lg = 4; lg >= 0; --lg) {
+    const int gr = 1 << lg;
+    for (int gap = 0; gap < 128; gap += 16) {
+      const int64_t pitch = gr * rb + gap;
+      int first[8], second[8], seen[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      bool ok = true;
+      for (int r = 0; r < 16 && ok; ++r) {
+        const int bank = static_cast<int>((((r >> lg) * pitch + (r & (gr - 1)) * rb) / 4) % 32) / 4;
+        if (seen[bank] == 0) first[bank] = r;
+        else if (seen[bank] == 1) second[bank] = r;
+        else ok = false;
+        ++seen[bank];
+      }
+      for (int b = 0; b < 8 && ok; ++b) ok = seen[b] == 2;
+      if (!ok) continue;
+      for (int b = 0; b < 8; ++b) {
+        p.rowmap[b] = static_cast<uint8_t>(first[b]);
+        p.rowmap[b + 8] = static_cast<uint8_t>(second[b]);
+      }
+      p.lg_sub = lg;
+      p.sub_pitch = static_cast<int>(pitch);
+      tile_span = static_cast<int>((16 >> lg) * pitch);
+      return true;
+    }
+  }
+  return false;
+}
+
 bool try_launch_digits(const DevInfo &dev, int nproj, const int64_t *N, const void *const *W, int K, const float *X,
-                       float *const *Y, bool single, cudaStream_t stream, uint32_t flags, qmm_status *out) {
-  if (K > 2048 || nproj < 1 || nproj > kMaxProj) return false;
+                       float *const *Y, bool single, cudaStream_t stream, uint32_t flags, qmm_status *out,
+                       int wtype = QMM_Q8_0) {
+  const bool q4 = wtype == QMM_Q4_0;
+  if (nproj < 1 || nproj > kMaxProj) return false;
+  if (!q4 && K > 2048) return false;
+  // Q4_0: one GEMV whose rows are 16-byte multiples (copied in groups of rows)
+  if (q4 && (nproj != 1 || K % 256 != 0 || K > 8192)) return false;
   const int KB = K / 32;
   const int tps = K <= 1024 ? 2 : 1;
+  if ((KB + 16 / tps - 1) / (16 / tps) > kMaxSliceBlocks) return false;  // checked again below for 8 warps
   DParams p{};
   int64_t chunks = 0;
   for (int i = 0; i < nproj; ++i) {
@@ -1893,34 +1999,52 @@ bool try_launch_digits(const DevInfo &dev, int nproj, const int64_t *N, const vo
   }
   p.chunk0[nproj] = chunks;
   p.nproj = nproj;
-  int grid = 2 * dev.sms;
-  if (single) {
+  p.X = X;
+  p.K = K;
+  p.KB = KB;
+  p.row_bytes = (q4 ? 18ll : 34ll) * KB;
+  p.padded = q4 ? 1 : 0;
+  int tile_span = 16 * static_cast<int>(p.row_bytes);  // bytes of a 16-row tile in shared memory
+  if (!place_rows(p, tile_span)) return false;
+  p.wexp = q4 ? -4 : 0;
+  p.tps = tps;
+  p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
+  p.stage_bytes = align_up(static_cast<int64_t>(tps) * tile_span + 64, 128);
+  p.rows_aligned = (p.row_bytes % 4) == 0 ? 1 : 0;
+  auto layout = [&](int warps) {  // shared-memory offsets for `warps` consumer warps
+    p.tab_off = 1024;
+    p.ftab_off = p.tab_off + 8 * kTabStride * KB;
+    p.eb_off = p.ftab_off + warps * kMaxSliceBlocks * 4 * 4;
+    p.red_off = align_up(p.eb_off + 4ll * KB, 16);
+    p.stage_off = align_up(p.red_off + 4ll * kMaxStages * 16 * warps, 128);  // K-slice partials
+  };
+  // two CTAs of eight consumer warps per SM when two stages fit in half the
+  // shared memory; Q4_0 rows of long K may take one CTA of sixteen per SM
+  constexpr int kHalfBudget = 113 * 1024;
+  int per_sm = 2, budget = kHalfBudget, nw = kDigitWarps;
+  layout(nw);
+  if (p.stage_off + 2 * p.stage_bytes > kHalfBudget) {
+    if (!q4) return false;
+    per_sm = 1;
+    budget = 2 * kHalfBudget;
+    nw = 16;
+    layout(nw);
+  }
+  if ((KB + nw / tps - 1) / (nw / tps) > kMaxSliceBlocks) return false;
+  int grid = per_sm * dev.sms;
+  if (single && !q4) {
     if (N[0] < static_cast<int64_t>(grid) * 32) return false;  // one GEMV takes this kernel only for many rows
   } else {
     grid = static_cast<int>(std::min<int64_t>(grid, chunks));  // every CTA at least one chunk
   }
   if (grid < 1) return false;
-  p.X = X;
-  p.K = K;
-  p.KB = KB;
-  p.row_bytes = 34ll * KB;
   p.grid = grid;
-  p.tps = tps;
-  p.prefetch_before_wait = (flags & kPrefetchBeforeWait) ? 1 : 0;
-  p.stage_bytes = align_up(16ll * tps * p.row_bytes + 64, 128);
-  p.tab_off = 1024;
-  p.ftab_off = p.tab_off + 8 * kTabStride * KB;
-  p.eb_off = p.ftab_off + kDigitWarps * kMaxSliceBlocks * 4 * 4;
-  p.rows_aligned = (p.row_bytes % 4) == 0 ? 1 : 0;
-  p.red_off = align_up(p.eb_off + 4ll * KB, 16);
-  p.stage_off = align_up(p.red_off + 4ll * kMaxStages * 16 * kDigitWarps, 128);  // K-slice partials
-  constexpr int kBudget = 113 * 1024;  // two CTAs per SM
-  p.stages = std::min(kMaxStages, (kBudget - p.stage_off) / p.stage_bytes);
+  p.stages = std::min(kMaxStages, (budget - p.stage_off) / p.stage_bytes);
   if (p.stages < 2) return false;
   const size_t smem = static_cast<size_t>(p.stage_off) + static_cast<size_t>(p.stages) * p.stage_bytes;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3((kDigitWarps + 1) * 32);
+  cfg.blockDim = dim3((nw + 1) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1930,24 +2054,35 @@ bool try_launch_digits(const DevInfo &dev, int nproj, const int64_t *N, const vo
   cfg.numAttrs = 1;
   // the projection table is a compile-time choice: one matrix keeps the plain loop
   const bool multi = nproj > 1;
-  void (*kern)(DParams) = tps == 2 ? (multi ? q8_gemv_digits_kernel<2, true> : q8_gemv_digits_kernel<2, false>)
-                                   : (multi ? q8_gemv_digits_kernel<1, true> : q8_gemv_digits_kernel<1, false>);
-  static DeviceFlags configured[2][2];
+  void (*kern)(DParams) =
+      q4 ? (nw == 16 ? (tps == 2 ? q8_gemv_digits_kernel<2, false, QMM_Q4_0, 16> : q8_gemv_digits_kernel<1, false, QMM_Q4_0, 16>)
+                     : (tps == 2 ? q8_gemv_digits_kernel<2, false, QMM_Q4_0, 8> : q8_gemv_digits_kernel<1, false, QMM_Q4_0, 8>))
+         : (tps == 2 ? (multi ? q8_gemv_digits_kernel<2, true, QMM_Q8_0, 8> : q8_gemv_digits_kernel<2, false, QMM_Q8_0, 8>)
+                     : (multi ? q8_gemv_digits_kernel<1, true, QMM_Q8_0, 8> : q8_gemv_digits_kernel<1, false, QMM_Q8_0, 8>));
+  static DeviceFlags configured[2][2][2][2];
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  if (!configured[tps - 1][multi].done(dev_id)) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBudget);
+  if (!configured[q4][nw == 16][tps - 1][multi].done(dev_id)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * kHalfBudget);
     if (e != cudaSuccess) {
       *out = cuda_check(e, "q8_gemv attribute");
       return true;
     }
-    configured[tps - 1][multi].set(dev_id);
+    configured[q4][nw == 16][tps - 1][multi].set(dev_id);
   }
   *out = cuda_check(cudaLaunchKernelEx(&cfg, kern, p), "q8_gemv launch");
   return true;
 }
 
 }  // namespace
+
+bool launch_q4_gemv_digits(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, float *Y,
+                           cudaStream_t stream, uint32_t flags, qmm_status *out) {
+  const int64_t n1[1] = {N};
+  const void *w1[1] = {W};
+  float *y1[1] = {Y};
+  return try_launch_digits(dev, 1, n1, w1, K, X, y1, true, stream, flags, out, QMM_Q4_0);
+}
 
 qmm_status launch_q8_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
                           cudaStream_t stream, uint32_t flags) {

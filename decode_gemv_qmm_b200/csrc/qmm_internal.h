@@ -77,9 +77,15 @@ qmm_status launch_quantize_act_q8(const DevInfo &dev, int64_t M, int K, const fl
 
 qmm_status launch_q4_gateup(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
                             const float *X, float *Y, cudaStream_t stream, uint32_t flags);
-// One Q4_0 projection Y = X . dequant(W)^T (the gate/up kernel with one matrix).
+// One Q4_0 projection Y = X . dequant(W)^T: M = 1 with K a multiple of 256 on
+// the integer tensor-core GEMV (q8_gemv.cu), otherwise the gate/up kernel with
+// one matrix.
 qmm_status launch_q4_gemv(const DevInfo &dev, int M, int64_t N, int K, const void *W, const float *X, float *Y,
                           cudaStream_t stream, uint32_t flags);
+// The M = 1 Q4_0 GEMV on the integer tensor-core kernel; false when the shape
+// does not suit it (then nothing was launched).
+bool launch_q4_gemv_digits(const DevInfo &dev, int64_t N, int K, const void *W, const float *X, float *Y,
+                           cudaStream_t stream, uint32_t flags, qmm_status *out);
 qmm_status launch_q4_gateup_unfused(const DevInfo &dev, int M, int64_t N, int K, const void *Wg, const void *Wu,
                                     const float *X, float *G, float *U, float *Y, cudaStream_t stream);
 

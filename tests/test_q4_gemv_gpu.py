@@ -1,10 +1,13 @@
 """qmm_q4_gemv (decode GEMV / small-M matmul on Q4_0 blocks) against the CPU oracle.
 
-Outputs must lie within 1e-5 * sum_k |w_k x_k| of the oracle, and equal the
-gate projection of qmm_q4_gateup_unfused bit for bit (same kernel, one matrix).
-Shapes cover M = 1 and M = 8, the down projection of the gate/up workload
-(K = 17408, N = 5120), ragged rows, and K that is not a multiple of 256 (the
-kernel's direct-load path).
+Outputs must lie within 1e-5 * sum_k |w_k x_k| of the oracle. For M > 1 the
+call is the gate/up kernel with one matrix and equals the gate projection of
+qmm_q4_gateup_unfused bit for bit; M = 1 with K a multiple of 256 (up to the
+shared-memory limit) runs the integer tensor-core GEMV instead (codes widened
+to 16 (q - 8), activations as base-256 digits). Shapes cover M = 1 and M = 8,
+the down projection of the gate/up workload (K = 17408, N = 5120), ragged
+rows, and K that is not a multiple of 256 (the gate/up kernel's direct-load
+path).
 """
 import numpy as np
 import pytest
@@ -43,6 +46,10 @@ def check(m, n, k, seed, flags=0):
     (1, 5120, 17408),
     (1, 16, 256), (3, 17, 512), (8, 33, 256), (5, 1000, 1024), (1, 4097, 2048),
     (1, 5, 32), (8, 40, 96), (4, 17, 288),   # K % 256 != 0: direct loads
+    (1, 3000, 768),     # M = 1 integer kernel: 32-row chunks, rows not padded (odd 16-byte count)
+    (1, 2001, 4096),    # 16-row chunks, padded rows, ragged last chunk
+    (1, 37, 7680),      # the longest K the integer kernel takes (one CTA per SM)
+    (1, 1000, 8192),    # beyond it: the gate/up kernel with one matrix
 ])
 def test_q4_gemv_matches_oracle(m, n, k):
     check(m, n, k, seed=m + 2 * n + 3 * k)
@@ -69,3 +76,25 @@ def test_q4_gemv_empty_and_zero_k():
     assert torch.count_nonzero(Y).item() == 0
     assert qmm.qmm_q4_gemv(torch.zeros(16, dtype=torch.uint8, device="cuda"),
                            torch.zeros(1, 32, device="cuda"), 0).shape == (1, 0)
+
+
+def test_q4_gemv_m1_early_weights_same_bits_and_dynamic_range():
+    g = syn.rng(22)
+    n, k = 17408, 5120
+    W = syn.q4_0_weights(g, n, k)[0]
+    x = syn.act_f32(g, 1, k)
+    Wd, xd = dev(W), dev(x)
+    Y0 = qmm.qmm_q4_gemv(Wd, xd, n)
+    Y1 = qmm.qmm_q4_gemv(Wd, xd, n, flags=qmm.QMM_FLAG_EARLY_WEIGHTS)
+    torch.cuda.synchronize()
+    assert torch.equal(Y0.view(torch.int32), Y1.view(torch.int32))
+    n = 4096
+    W = np.ascontiguousarray(W[:n])
+    for name, scale in (("tiny", 1e-33), ("huge", 1e30), ("mixed", None)):
+        xs = x * (10.0 ** g.uniform(-4, 4, size=x.shape)) if scale is None else x * scale
+        xs = xs.astype(np.float32)
+        Y = qmm.qmm_q4_gemv(dev(W), dev(xs), n)
+        torch.cuda.synchronize()
+        ref, S = oracle_gemv(W, xs, n)
+        assert_within(host(Y), ref, S, TOL_FP32, f"q4_gemv M=1 x={name}")
+    assert qmm.device_status() == 0
