@@ -312,9 +312,13 @@ QMM_API qmm_status qmm_q4_swiglu_gateup_ex(int64_t M, int64_t N, int64_t K, int 
  *
  *   Y[m][n] = sum_b d[n][b] * sum_j (q[n][b][j] - 8) * X[m][32b + j]   (fp32 accumulation)
  *
- * It runs the fused gate/up kernel with one matrix, so each output equals
- * the corresponding gate (or up) projection of qmm_q4_swiglu_gateup's
- * unfused form bit for bit.
+ * For M >= 2 (and M = 1 with K not a multiple of 256, or K > 7680) it runs the
+ * fused gate/up kernel with one matrix, so each output equals the
+ * corresponding gate (or up) projection of qmm_q4_swiglu_gateup's unfused form
+ * bit for bit. M = 1 otherwise runs the integer tensor-core GEMV on the raw
+ * codes (the activations as base-256 digits, as in qmm_q8_gemv's lm_head
+ * form); the result is within the same fp32 tolerance, not bit-equal to the
+ * gate/up kernel's.
  *
  *   M      1 .. QMM_MAX_DECODE_M (0 = empty call)
  *   W      N * K/32 Q4_0 blocks (16-byte aligned)
