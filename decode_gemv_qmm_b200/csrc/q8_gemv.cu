@@ -1252,13 +1252,23 @@ __global__ void __launch_bounds__((NW + 1) * 32) q8_gemv_digits_kernel(const __g
   constexpr uint32_t kBB = WT == QMM_Q8_0 ? 34u : 18u;  // bytes per block
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // whole chunks per CTA: a chunk costs the same however few of its rows are
-  // valid, so an even split of rows (every CTA ending in a one-row chunk)
-  // costs a chunk per CTA more than an even split of chunks
-  const int64_t tchunks = MULTI ? p.chunk0[p.nproj] : (p.Np[0] + kRows - 1) / kRows;
-  const int64_t c_begin = static_cast<int64_t>(blockIdx.x) * tchunks / p.grid;
-  const int64_t c_end = static_cast<int64_t>(blockIdx.x + 1) * tchunks / p.grid;
-  const int nchunks = static_cast<int>(c_end - c_begin);
+  // Work split: the projection table by whole chunks (a chunk never spans two
+  // matrices); one matrix by whole 16-row tiles, so that a CTA may end in a
+  // one-tile chunk (half the bytes of a two-tile chunk: the busiest CTAs of a
+  // long launch carry half a chunk more, not a whole one). An even split of
+  // rows would end every CTA in a ragged chunk that streams nearly as long.
+  int64_t c_begin = 0, r_begin = 0, r_end = 0;
+  int nchunks;
+  if constexpr (MULTI) {
+    const int64_t tchunks = p.chunk0[p.nproj];
+    c_begin = static_cast<int64_t>(blockIdx.x) * tchunks / p.grid;
+    nchunks = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * tchunks / p.grid - c_begin);
+  } else {
+    const int64_t tiles = (p.Np[0] + 15) / 16;
+    r_begin = 16 * (static_cast<int64_t>(blockIdx.x) * tiles / p.grid);
+    r_end = min(p.Np[0], 16 * (static_cast<int64_t>(blockIdx.x + 1) * tiles / p.grid));
+    nchunks = static_cast<int>((r_end - r_begin + kRows - 1) / kRows);
+  }
   const int S = p.stages;
   // chunk c of this CTA: its projection, first row and valid rows
   struct Chunk {
@@ -1266,7 +1276,6 @@ __global__ void __launch_bounds__((NW + 1) * 32) q8_gemv_digits_kernel(const __g
     int64_t r0;
     int rows;
   };
-  const int64_t r_begin = c_begin * kRows, r_end = min(p.Np[0], c_end * kRows);  // one matrix
   auto chunk = [&](int c) -> Chunk {
     if constexpr (MULTI) {
       const int64_t gc = c_begin + c;
